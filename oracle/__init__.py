@@ -1,0 +1,245 @@
+"""CPU oracle for the BitLinear W1.58A8 forward -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA
+library; the product path never calls it.
+
+Each function states the passage it follows.  Sources (web pages):
+
+* DataCamp blog "MatMul-free language models" (Dutch), section "MatMul
+  vervangen door ternaire bewerkingen" -- absmean ternarisation; -1/0/+1
+  multiplies become negate/zero/pass-through.  Figure item "RMS norm" --
+  activations are normalised before quantisation.  Section "Kerncomponenten:
+  MLGRU en GLU" -- the MatMul-free GLU (two BitLinears, SiLU, elementwise
+  product, a third BitLinear).
+* unite.ai "Microsofts Inference Framework bringt 1-Bit grosse Sprachmodelle
+  auf lokale Geraete" (German), section "Mathematische Grundlagen", eq. 2
+  "Aktivierungsquantisierung" and eq. 3 "BitLinear-Betrieb".
+
+Pins (tests/test_oracle_pins.py): a hand-worked 4x4 example, closed forms of
+the Gaussian absmean statistics, invariants, brute force on tiny inputs and
+reduction of the contraction to numpy's int64 matmul; the exact |W| sum is
+checked against ``math.fsum``.  Parity unpinned: ``silu_mul`` beyond its
+binary64 error bound (exp is a library routine on both sides).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = ctypes.CDLL(_build.build())
+
+_f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+_i8p = np.ctypeslib.ndpointer(np.int8, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+_u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
+_u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+_i64 = ctypes.c_int64
+
+_lib.orc_exact_abs_sum.argtypes = [_f32p, _i64]
+_lib.orc_exact_abs_sum.restype = ctypes.c_double
+_lib.orc_absmean_beta.argtypes = [_f32p, _i64, _i64]
+_lib.orc_absmean_beta.restype = ctypes.c_float
+_lib.orc_ternarize.argtypes = [_f32p, _i64, _i64, ctypes.c_float, ctypes.c_float, _i8p]
+_lib.orc_pack.argtypes = [_i8p, _i64, _i64, _u32p]
+_lib.orc_unpack.argtypes = [_u32p, _i64, _i64, _i8p]
+_lib.orc_unpack.restype = _i64
+_lib.orc_quant_act.argtypes = [_f32p, _i64, _i64, _i8p, _f32p]
+_lib.orc_ternary_acc.argtypes = [_i8p, _i64, _i64, _i8p, _i64, _i32p]
+_lib.orc_rescale_f32.argtypes = [_i32p, _i64, _i64, ctypes.c_float, _f32p, _f32p]
+_lib.orc_rescale_f64.argtypes = [_i32p, _i64, _i64, ctypes.c_float, _f32p, _f64p]
+_lib.orc_f32_to_bf16.argtypes = [_f32p, _i64, _u16p]
+_lib.orc_rms_rho.argtypes = [_f32p, _i64, ctypes.c_double]
+_lib.orc_rms_rho.restype = ctypes.c_float
+_lib.orc_silu_mul.argtypes = [_f32p, _f32p, _i64, _f32p]
+
+EPS_W = np.float32(1e-5)      # divisor guard of the ternariser
+Q_B = 127                     # int8 activation range [-127, 127]
+GAMMA_FLOOR = np.float32(1e-5)
+RMS_EPS = 1e-6                # RMSNorm epsilon of the decoder block
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def exact_abs_sum(w: np.ndarray) -> float:
+    """Exact sum of |w| over binary32 values, correctly rounded to binary64."""
+    w = _c(w, np.float32).ravel()
+    return float(_lib.orc_exact_abs_sum(w, w.size))
+
+
+def absmean_beta(W: np.ndarray) -> np.float32:
+    """absmean scale, one per matrix (MatMul-free blog, "MatMul vervangen door
+    ternaire bewerkingen"): beta = mean |W|, the exact mean rounded to binary64
+    then binary32."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    return np.float32(_lib.orc_absmean_beta(W, N, K))
+
+
+def ternarize(W: np.ndarray, beta, eps=EPS_W) -> np.ndarray:
+    """W_t = clip(round(W / (beta + eps)), -1, 1), binary32 divide, ties to even
+    (MatMul-free blog, "MatMul vervangen door ternaire bewerkingen")."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    out = np.empty((N, K), np.int8)
+    _lib.orc_ternarize(W, N, K, np.float32(beta), np.float32(eps), out)
+    return out
+
+
+def quantize_weights(W: np.ndarray, eps=EPS_W):
+    """absmean ternarisation of a full-precision matrix -> (W_t int8, beta fp32)."""
+    beta = absmean_beta(W)
+    return ternarize(W, beta, eps), beta
+
+
+def pack(W_t: np.ndarray) -> np.ndarray:
+    """2-bit codes c = w + 1, trit k = 16j + 4s + b of a row at bits 8b + 2s of word j."""
+    W_t = _c(W_t, np.int8)
+    N, K = W_t.shape
+    assert K % 16 == 0
+    out = np.empty((N, K // 16), np.uint32)
+    _lib.orc_pack(W_t, N, K, out)
+    return out
+
+
+def unpack(W_p: np.ndarray, K: int):
+    """Inverse of :func:`pack`; returns (W_t, number of invalid code-3 fields)."""
+    W_p = _c(W_p, np.uint32)
+    N = W_p.shape[0]
+    out = np.empty((N, K), np.int8)
+    bad = _lib.orc_unpack(W_p, N, K, out)
+    return out, int(bad)
+
+
+def quant_act(x: np.ndarray):
+    """Per-token absmax int8 quantiser (unite.ai page, eq. 2 "Aktivierungs-
+    quantisierung") with Q_b = 127: gamma = max(||x_m||_inf, 1e-5),
+    s = 127 / gamma, x_hat = clip(rint(x * s), -127, 127), all binary32."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    xq = np.empty((M, K), np.int8)
+    g = np.empty(M, np.float32)
+    _lib.orc_quant_act(x, M, K, xq, g)
+    return xq, g
+
+
+def ternary_acc(x_q: np.ndarray, W_t: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k W_t[n, k] x_hat[m, k] by literal add / subtract / skip
+    (MatMul-free blog: multiplying by -1, 0, 1 is negation, zero, identity)."""
+    x_q = _c(x_q, np.int8)
+    W_t = _c(W_t, np.int8)
+    M, K = x_q.shape
+    N = W_t.shape[0]
+    assert W_t.shape[1] == K
+    acc = np.empty((M, N), np.int32)
+    _lib.orc_ternary_acc(x_q, M, K, W_t, N, acc)
+    return acc
+
+
+def rescale_f32(acc, beta, gamma) -> np.ndarray:
+    """unite.ai eq. 3 "BitLinear-Betrieb": y = acc * (beta * gamma / 127),
+    binary32 with f = (beta * gamma) / 127 formed first."""
+    acc = _c(acc, np.int32)
+    M, N = acc.shape
+    y = np.empty((M, N), np.float32)
+    _lib.orc_rescale_f32(acc, M, N, np.float32(beta), _c(gamma, np.float32), y)
+    return y
+
+
+def rescale_f64(acc, beta, gamma) -> np.ndarray:
+    """The same rescale in binary64 (the reference the 1e-6 tolerance is taken against)."""
+    acc = _c(acc, np.int32)
+    M, N = acc.shape
+    y = np.empty((M, N), np.float64)
+    _lib.orc_rescale_f64(acc, M, N, np.float32(beta), _c(gamma, np.float32), y)
+    return y
+
+
+def to_bf16(y: np.ndarray) -> np.ndarray:
+    """binary32 -> bf16 bit patterns, round to nearest, ties to even."""
+    y = _c(y, np.float32)
+    out = np.empty(y.shape, np.uint16)
+    _lib.orc_f32_to_bf16(y.ravel(), y.size, out.reshape(-1))
+    return out
+
+
+def forward(x: np.ndarray, W_t: np.ndarray, beta):
+    """Whole BitLinear forward from fp32 activations and ternary weights.
+
+    Returns a dict with x_q, gamma, acc, y (binary32 op order) and y64."""
+    x_q, gamma = quant_act(x)
+    acc = ternary_acc(x_q, W_t)
+    return {"x_q": x_q, "gamma": gamma, "acc": acc,
+            "y": rescale_f32(acc, beta, gamma), "y64": rescale_f64(acc, beta, gamma)}
+
+
+# ---------------------------------------------------------------------------
+# Decoder block at batch-1 decode (hidden 2560, intermediate 6912).
+# ---------------------------------------------------------------------------
+
+def rms_rho(x: np.ndarray) -> np.float32:
+    """RMSNorm scalar with gain 1 (MatMul-free blog, figure item "RMS norm"):
+    rho = 1 / sqrt(mean(x^2) + 1e-6), binary64, rounded once to binary32."""
+    x = _c(x, np.float32).ravel()
+    return np.float32(_lib.orc_rms_rho(x, x.size, RMS_EPS))
+
+
+def quant_act_rmsnorm(x: np.ndarray):
+    """Quantiser of RMSNorm(x) for one token.  absmax quantisation is invariant
+    under a positive scale of the token, so Q(rho * x) has the codes of Q(x)
+    and the scale gamma_eff = rho * gamma(x) (binary32 multiply)."""
+    x_q, g = quant_act(x)
+    rho = rms_rho(x)
+    return x_q, (g * rho).astype(np.float32), rho
+
+
+def silu_mul(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """SiLU(gate) * up in binary64, rounded once to binary32 (the GLU of the
+    MatMul-free blog, section "Kerncomponenten: MLGRU en GLU")."""
+    gate = _c(gate, np.float32).ravel()
+    up = _c(up, np.float32).ravel()
+    out = np.empty(gate.size, np.float32)
+    _lib.orc_silu_mul(gate, up, gate.size, out)
+    return out
+
+
+def bitlinear_rms(x_row: np.ndarray, W_t: np.ndarray, beta):
+    """One projection of the block: RMSNorm folded into the quantiser, ternary
+    contraction, binary32 rescale."""
+    x_q, g_eff, _ = quant_act_rmsnorm(x_row.reshape(1, -1))
+    acc = ternary_acc(x_q, W_t)
+    return {"x_q": x_q, "gamma": g_eff, "acc": acc, "y": rescale_f32(acc, beta, g_eff)}
+
+
+def block_decode(x: np.ndarray, tern: dict) -> dict:
+    """One decoder block for one token.  ``tern[p] = (W_t, beta)`` for p in
+    q, k, v, o, gate, up, down.
+
+    Attention over the single token in the context is softmax of one score,
+    i.e. weight 1 on v, so the attention output equals v.  Residual adds are
+    binary32.  Every BitLinear input is RMS-normalised before quantisation."""
+    x = _c(x, np.float32).reshape(1, -1)
+    out = {}
+    q = bitlinear_rms(x, *tern["q"])          # all three share one x_hat
+    k = bitlinear_rms(x, *tern["k"])
+    v = bitlinear_rms(x, *tern["v"])
+    out.update(q=q["y"], k=k["y"], v=v["y"], x_q_attn=q["x_q"], gamma_attn=q["gamma"])
+    attn = v["y"]
+    o = bitlinear_rms(attn, *tern["o"])
+    h1 = (x + o["y"]).astype(np.float32)
+    gate = bitlinear_rms(h1, *tern["gate"])
+    up = bitlinear_rms(h1, *tern["up"])
+    u = silu_mul(gate["y"], up["y"]).reshape(1, -1)
+    down = bitlinear_rms(u, *tern["down"])
+    h2 = (h1 + down["y"]).astype(np.float32)
+    out.update(o=o["y"], h1=h1, gate=gate["y"], up=up["y"], u=u, down=down["y"], out=h2,
+               x_q_o=o["x_q"], x_q_mlp=gate["x_q"], x_q_down=down["x_q"],
+               acc_down=down["acc"])
+    return out
