@@ -1,0 +1,208 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the B200 (sm_100a) BitLinear
+ * W1.58A8 forward: ternary weights {-1, 0, +1} with one scale per matrix,
+ * int8 activations quantised per token by absmax, int32 accumulation and a
+ * fused rescale.
+ *
+ * Sources (web pages):
+ *   [MMF] DataCamp blog "MatMul-free language models" (Dutch): section
+ *         "MatMul vervangen door ternaire bewerkingen" (absmean ternarisation;
+ *         a multiply by -1/0/+1 is a negate/zero/pass-through), figure item
+ *         "RMS norm" (normalise activations before quantisation), section
+ *         "Kerncomponenten: MLGRU en GLU" (the MatMul-free GLU).
+ *   [BNC] unite.ai "Microsofts Inference Framework bringt 1-Bit grosse
+ *         Sprachmodelle auf lokale Geraete" (German): section "Ternaeres
+ *         Gewichtssystem" (1.58-bit ternary weights), section "Mathematische
+ *         Grundlagen" eq. 2 "Aktivierungsquantisierung" and eq. 3
+ *         "BitLinear-Betrieb", section "Implementierungshinweise" (the
+ *         quantise -> ternary matmul -> scale shape of a forward call).
+ *
+ * Conventions for every call:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller (the
+ *     library allocates nothing and frees nothing), 16-byte aligned.  Outputs
+ *     must not overlap inputs.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work on it and never synchronise, except
+ *     bitlinear_device_status(), which says so.
+ *   - Shapes: M tokens, K input features, N output features.  x is [M, K]
+ *     row-major, W is [N, K] row-major (nn.Linear out x in), y is [M, N]
+ *     row-major.  Sizes are int64_t and must be >= 1.
+ *   - Arguments are validated on the host before any launch; on error nothing
+ *     is launched and a nonzero bl_status is returned.  Device faults are not
+ *     used for error reporting.  Non-finite inputs (NaN, Inf) give
+ *     unspecified results.
+ *   - A nonzero return after a launch (BL_ERR_CUDA) carries the CUDA error of
+ *     the launch; the stream is otherwise left as it was.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int bl_status;
+
+enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,       /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,      /* a size is < 1, too large, or violates a divisibility rule */
+    BL_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned */
+    BL_ERR_DTYPE = 4,      /* unknown dtype or combine enum */
+    BL_ERR_WORKSPACE = 5,  /* workspace NULL or smaller than the *_workspace() size */
+    BL_ERR_DEVICE = 6,     /* no CUDA device, or current device is not compute capability 10.x */
+    BL_ERR_CUDA = 7,       /* a launch or runtime call failed */
+    BL_ERR_TIMEOUT = 8,    /* a bounded on-device wait expired (reported by bitlinear_device_status) */
+    BL_ERR_ALIAS = 9       /* an output overlaps an input */
+};
+
+enum { BL_F32 = 0, BL_BF16 = 1 };
+
+/* Largest K accepted (keeps every int32 partial of the contraction exact). */
+#define BL_MAX_K 262144
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bitlinear_status_string(bl_status s);
+
+/* ------------------------------------------------------------------------ */
+/* Offline weight preparation                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace bitlinear_quantize_weights needs (any N, K). */
+size_t bitlinear_quantize_weights_workspace(int64_t N, int64_t K);
+
+/*
+ * absmean ternarisation, [MMF] "MatMul vervangen door ternaire bewerkingen":
+ *   beta   = mean over all N*K elements of |W|          (one scale per matrix)
+ *   W_t    = clip(round(W / (beta + eps)), -1, 1)        (ties to even)
+ * beta is the exact sum of |W| rounded to binary64, divided by N*K in
+ * binary64 and rounded to binary32.  The sum is taken in fixed point: with
+ * E the binary32 exponent of max|W|, every |w| is truncated to a multiple of
+ * 2^(E-38-23) (exact for |w| >= 2^-38 max|W|) and the integers are added
+ * exactly, so the result does not depend on thread order.  The divisor
+ * beta + eps and the quotient are binary32 (IEEE add, IEEE divide).
+ *   W    [N, K] float32, device, read only
+ *   W_t  [N, K] int8 out, values in {-1, 0, 1}
+ *   beta [1] float32 out (stays on the device)
+ *   ws   >= bitlinear_quantize_weights_workspace(N, K) bytes of device scratch
+ *        (contents on entry do not matter; calls sharing a ws must not overlap)
+ * eps must be finite and >= 0 (1e-5 in the workloads); an all-zero W gives
+ * beta = 0 and W_t = 0.
+ */
+bl_status bitlinear_quantize_weights(const float* W, int64_t N, int64_t K, float eps,
+                                     int8_t* W_t, float* beta, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/*
+ * 2-bit packing of ternary weights ([BNC] "Ternaeres Gewichtssystem": three
+ * states per weight, stored here in 2 bits, 16 per uint32).  Code c = w + 1
+ * in {0, 1, 2}.  For row n and word j, the trit at k = 16j + 4s + b
+ * (s, b in 0..3) sits at bits [8b + 2s, 8b + 2s + 1] of W_p[n, j], so that
+ * (word >> 2s) & 0x03030303 holds the codes of k = 16j+4s .. 16j+4s+3 in
+ * its four bytes.  An all-zero group of 16 trits packs to 0x55555555.
+ *   W_t [N, K] int8 in, values must be in {-1, 0, 1} (others: unspecified)
+ *   W_p [N, K/16] uint32 out
+ * K % 16 == 0.
+ */
+bl_status bitlinear_pack(const int8_t* W_t, int64_t N, int64_t K, uint32_t* W_p, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Per-token forward                                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Per-token absmax int8 activation quantiser, [BNC] eq. 2
+ * "Aktivierungsquantisierung" with Q_b = 127 and a symmetric clamp:
+ *   gamma_m = max(max_k |x[m, k]|, 1e-5)                  (binary32)
+ *   s_m     = 127 / gamma_m                               (binary32 IEEE divide)
+ *   x_q     = clip(rint(x[m, k] * s_m), -127, 127)        (binary32 multiply, ties to even)
+ *   x     [M, K] float32 (x_dtype BL_F32) or bfloat16 (BL_BF16), in
+ *   x_q   [M, K] int8 out
+ *   gamma [M] float32 out
+ * K % 16 == 0, K <= BL_MAX_K.
+ */
+bl_status bitlinear_quant_act(const void* x, int x_dtype, int64_t M, int64_t K,
+                              int8_t* x_q, float* gamma, void* stream);
+
+/* Bytes of device workspace bitlinear_forward needs for this shape (may be 0). */
+size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K);
+
+/*
+ * BitLinear forward on quantised inputs, [BNC] eq. 3 "BitLinear-Betrieb",
+ * with the multiplies of [MMF] replaced by add / subtract / skip:
+ *   acc[m, n] = sum_k W_t[n, k] * x_q[m, k]               (int32, exact)
+ *   y[m, n]   = (float)acc[m, n] * ((beta * gamma_m) / 127)  (binary32, this order)
+ * and for y_dtype BL_BF16 the binary32 value rounded to nearest-even bf16.
+ *   x_q   [M, K] int8, gamma [M] float32, W_p [N, K/16] uint32 (bitlinear_pack
+ *         layout), beta [1] float32 -- all inputs
+ *   y     [M, N] float32 or bfloat16 out
+ *   ws    >= bitlinear_forward_workspace(M, N, K) bytes (may be NULL when that is 0)
+ * K % 64 == 0, K <= BL_MAX_K.  M <= 64 runs the decode GEMV (CUDA cores);
+ * larger M runs the prefill GEMM (tcgen05 int8 tensor cores).  Both give
+ * identical results.
+ */
+bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
+                            const uint32_t* W_p, const float* beta, int64_t N,
+                            void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Inspection variant of bitlinear_forward: writes the int32 accumulators
+ * acc[M, N] = sum_k W_t[n, k] * x_q[m, k] instead of y (same kernels, same
+ * dispatch, rescale skipped).  For exact comparisons in tests.
+ */
+bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K,
+                                const uint32_t* W_p, int64_t N, int32_t* acc,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decoder-block glue                                                        */
+/* ------------------------------------------------------------------------ */
+
+enum { BL_COMBINE_NONE = 0, BL_COMBINE_ADD = 1, BL_COMBINE_SILU_MUL = 2 };
+
+/*
+ * Fused combine + RMSNorm + int8 quantiser for the decoder block, one token
+ * per row.  [MMF] figure item "RMS norm": activations are RMS-normalised
+ * (gain 1) before quantisation; [MMF] "Kerncomponenten: MLGRU en GLU": the
+ * GLU gates one BitLinear output with SiLU of the other.
+ *   h[m, k] = a                                  (BL_COMBINE_NONE)
+ *           = a + b            (binary32 add)     (BL_COMBINE_ADD)
+ *           = (float)(silu(a) * b), silu(a) = a / (1 + exp(-a)), in binary64
+ *                                                 (BL_COMBINE_SILU_MUL)
+ *   rho_m   = (float)(1 / sqrt(mean_k h^2 + 1e-6))    (binary64, then rounded)
+ * absmax quantisation is invariant under the positive per-token scale rho,
+ * so the codes are those of bitlinear_quant_act applied to h, and
+ *   gamma[m] = rho_m * max(max_k |h[m, k]|, 1e-5)       (binary32 multiply).
+ *   a, b  [M, K] float32 in (b unused and may be NULL for BL_COMBINE_NONE)
+ *   h     [M, K] float32 out, may be NULL (not written)
+ *   x_q   [M, K] int8 out, may be NULL together with gamma (then only h is
+ *         produced and no norm is computed)
+ *   gamma [M] float32 out
+ * K % 16 == 0, K <= BL_MAX_K.
+ */
+bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, int64_t M, int64_t K,
+                                  float* h, int8_t* x_q, float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics                                                               */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word on the current device.  Returns BL_ERR_TIMEOUT if any kernel since the
+ * last call gave up a bounded wait (the kernel then returned early and its
+ * outputs are unspecified), BL_ERR_CUDA on a CUDA error, else BL_OK.
+ */
+bl_status bitlinear_device_status(void* stream);
+
+/* Number of SMs of the current device as seen by the library (0 if none). */
+int bitlinear_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,291 @@
+"""Thin Python binding of libbitlinear.so (argument marshalling only).
+
+Every function below checks dtypes, shapes and devices of torch tensors,
+allocates outputs with torch (device memory is PyTorch's job here), passes raw
+pointers and the current CUDA stream through the C ABI declared in
+``include/bitlinear.h``, and raises ``BitLinearError`` on a nonzero status.
+All arithmetic happens in the library's CUDA kernels.  There is no fallback:
+if the shared library is missing or no sm_100 device is present, calls fail.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+BL_F32, BL_BF16 = 0, 1
+COMBINE = {"none": 0, "add": 1, "silu_mul": 2}
+EPS_W = 1e-5
+
+_STATUS = {0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGN", 4: "BL_ERR_DTYPE",
+           5: "BL_ERR_WORKSPACE", 6: "BL_ERR_DEVICE", 7: "BL_ERR_CUDA", 8: "BL_ERR_TIMEOUT", 9: "BL_ERR_ALIAS"}
+
+# every symbol the header declares: (name, restype, argtypes)
+_P, _I64, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "bitlinear_status_string": (ctypes.c_char_p, [_I]),
+    "bitlinear_quantize_weights_workspace": (_SZ, [_I64, _I64]),
+    "bitlinear_quantize_weights": (_I, [_P, _I64, _I64, _F, _P, _P, _P, _SZ, _P]),
+    "bitlinear_pack": (_I, [_P, _I64, _I64, _P, _P]),
+    "bitlinear_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
+    "bitlinear_forward_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_forward": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_device_status": (_I, [_P]),
+    "bitlinear_num_sms": (_I, []),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitlinear.so from the package directory (built by build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m ternary_weight_linear_forward_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().bitlinear_status_string(int(s)).decode()
+
+
+def _check(fn: str, s: int):
+    if s != 0:
+        raise BitLinearError(fn, s)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, ndim, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------------
+# entry points
+# --------------------------------------------------------------------------
+
+def quantize_weights(W: torch.Tensor, eps: float = EPS_W, stream=None):
+    """absmean ternarisation -> (W_t int8 [N, K], beta float32 [1]) on W's device."""
+    _need(W, torch.float32, 2, "W")
+    N, K = W.shape
+    W_t = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    beta = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
+    nws = lib().bitlinear_quantize_weights_workspace(N, K)
+    ws = torch.empty(nws, dtype=torch.uint8, device=W.device)
+    _check("bitlinear_quantize_weights",
+           lib().bitlinear_quantize_weights(_ptr(W), N, K, float(eps), _ptr(W_t), _ptr(beta), _ptr(ws), nws,
+                                            _stream(stream)))
+    return W_t, beta
+
+
+def pack(W_t: torch.Tensor, stream=None) -> torch.Tensor:
+    """2-bit packing, 16 trits per uint32 -> W_p int32 [N, K/16] (bit pattern of uint32)."""
+    _need(W_t, torch.int8, 2, "W_t")
+    N, K = W_t.shape
+    W_p = torch.empty((N, K // 16 if K % 16 == 0 else 1), dtype=torch.int32, device=W_t.device)
+    _check("bitlinear_pack", lib().bitlinear_pack(_ptr(W_t), N, K, _ptr(W_p), _stream(stream)))
+    return W_p
+
+
+def quant_act(x: torch.Tensor, out=None, stream=None):
+    """Per-token absmax int8 quantiser -> (x_q int8 [M, K], gamma float32 [M])."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, 2, "x")
+    M, K = x.shape
+    if out is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+        gamma = torch.empty(max(M, 4), dtype=torch.float32, device=x.device)[:M]
+    else:
+        x_q, gamma = out
+    dt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_quant_act",
+           lib().bitlinear_quant_act(_ptr(x), dt, M, K, _ptr(x_q), _ptr(gamma), _stream(stream)))
+    return x_q, gamma
+
+
+def forward_workspace(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_forward_workspace(M, N, K))
+
+
+def forward(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,
+            out_dtype=torch.float32, out=None, ws=None, stream=None) -> torch.Tensor:
+    """y = BitLinear(x_q) with the fused rescale; float32 or bfloat16 output."""
+    _need(x_q, torch.int8, 2, "x_q")
+    _need(W_p, torch.int32, 2, "W_p")
+    _need(gamma, torch.float32, 1, "gamma")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x_q.shape
+    N = W_p.shape[0]
+    if W_p.shape[1] * 16 != K:
+        raise ValueError("W_p must be [N, K/16]")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = forward_workspace(M, N, K)
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward",
+           lib().bitlinear_forward(_ptr(x_q), _ptr(gamma), M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                   _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """int32 accumulators acc[m, n] = sum_k W_t[n, k] x_q[m, k] (same kernels as forward)."""
+    _need(x_q, torch.int8, 2, "x_q")
+    _need(W_p, torch.int32, 2, "W_p")
+    M, K = x_q.shape
+    N = W_p.shape[0]
+    if W_p.shape[1] * 16 != K:
+        raise ValueError("W_p must be [N, K/16]")
+    acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
+    nws = forward_workspace(M, N, K)
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward_acc",
+           lib().bitlinear_forward_acc(_ptr(x_q), M, K, _ptr(W_p), N, _ptr(acc), _ptr(ws),
+                                       0 if ws is None else ws.numel(), _stream(stream)))
+    return acc
+
+
+def quant_act_rms(a: torch.Tensor, b: torch.Tensor | None = None, combine: str = "none", h=None,
+                  quantize: bool = True, want_h: bool = False, out=None, stream=None):
+    """Fused combine (none/add/silu_mul) + RMSNorm-folded int8 quantiser.
+
+    Returns (h or None, x_q or None, gamma or None)."""
+    _need(a, torch.float32, 2, "a")
+    if b is not None:
+        _need(b, torch.float32, 2, "b")
+    M, K = a.shape
+    if want_h and h is None:
+        h = torch.empty_like(a)
+    if quantize:
+        if out is None:
+            x_q = torch.empty((M, K), dtype=torch.int8, device=a.device)
+            gamma = torch.empty(max(M, 4), dtype=torch.float32, device=a.device)[:M]
+        else:
+            x_q, gamma = out
+    else:
+        x_q = gamma = None
+    _check("bitlinear_quant_act_rms",
+           lib().bitlinear_quant_act_rms(_ptr(a), _ptr(b), COMBINE[combine], M, K, _ptr(h), _ptr(x_q),
+                                         _ptr(gamma), _stream(stream)))
+    return h, x_q, gamma
+
+
+def device_status(stream=None):
+    """Synchronise the stream and raise if a kernel gave up a bounded wait."""
+    _check("bitlinear_device_status", lib().bitlinear_device_status(_stream(stream)))
+
+
+def num_sms() -> int:
+    return int(lib().bitlinear_num_sms())
+
+
+# --------------------------------------------------------------------------
+# convenience layer objects (still only marshalling around the C ABI)
+# --------------------------------------------------------------------------
+
+class BitLinear:
+    """A prepared ternary layer: packed weights W_p [N, K/16] and scale beta [1]."""
+
+    def __init__(self, W_p: torch.Tensor, beta: torch.Tensor):
+        self.W_p, self.beta = W_p, beta
+        self.N, self.K = W_p.shape[0], W_p.shape[1] * 16
+
+    @classmethod
+    def from_float(cls, W: torch.Tensor, eps: float = EPS_W):
+        W_t, beta = quantize_weights(W, eps)
+        return cls(pack(W_t), beta)
+
+    def __call__(self, x: torch.Tensor, out_dtype=torch.float32, out=None) -> torch.Tensor:
+        x_q, gamma = quant_act(x)
+        return forward(x_q, gamma, self.W_p, self.beta, out_dtype=out_dtype, out=out)
+
+
+class DecoderBlock:
+    """One ternary decoder block at batch-1 decode (seven BitLinear projections).
+
+    h1 = x + o(v(x)) where attention over the single token returns v; out =
+    h1 + down(SiLU(gate(h1)) * up(h1)); every projection input is
+    RMS-normalised (gain 1) inside the fused quantiser."""
+
+    PROJ = ("q", "k", "v", "o", "gate", "up", "down")
+
+    def __init__(self, layers: dict):
+        self.layers = layers
+        self.hidden = layers["q"].K
+        self.inter = layers["gate"].N
+        dev = layers["q"].W_p.device
+        H, F = self.hidden, self.inter
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.buf = {
+            "xq_h": torch.empty((1, H), dtype=torch.int8, device=dev),
+            "g_h": torch.empty(4, **f32)[:1],
+            "xq_f": torch.empty((1, F), dtype=torch.int8, device=dev),
+            "g_f": torch.empty(4, **f32)[:1],
+            "q": torch.empty((1, H), **f32), "k": torch.empty((1, H), **f32), "v": torch.empty((1, H), **f32),
+            "o": torch.empty((1, H), **f32), "h1": torch.empty((1, H), **f32),
+            "gate": torch.empty((1, F), **f32), "up": torch.empty((1, F), **f32),
+            "u": torch.empty((1, F), **f32), "down": torch.empty((1, H), **f32),
+            "out": torch.empty((1, H), **f32),
+        }
+
+    @classmethod
+    def from_float(cls, weights: dict, eps: float = EPS_W):
+        return cls({p: BitLinear.from_float(weights[p], eps) for p in cls.PROJ})
+
+    def __call__(self, x: torch.Tensor, keep_u: bool = True) -> dict:
+        b, L = self.buf, self.layers
+        xh = (b["xq_h"], b["g_h"])
+        xf = (b["xq_f"], b["g_f"])
+        quant_act_rms(x, out=xh)
+        for p in ("q", "k", "v"):
+            forward(*xh, L[p].W_p, L[p].beta, out=b[p])
+        quant_act_rms(b["v"], out=xh)                     # attention over one token = v
+        forward(*xh, L["o"].W_p, L["o"].beta, out=b["o"])
+        quant_act_rms(x, b["o"], "add", h=b["h1"], out=xh)
+        forward(*xh, L["gate"].W_p, L["gate"].beta, out=b["gate"])
+        forward(*xh, L["up"].W_p, L["up"].beta, out=b["up"])
+        quant_act_rms(b["gate"], b["up"], "silu_mul", h=b["u"] if keep_u else None, out=xf)
+        forward(*xf, L["down"].W_p, L["down"].beta, out=b["down"])
+        quant_act_rms(b["h1"], b["down"], "add", h=b["out"], quantize=False)
+        return b

@@ -1,0 +1,275 @@
+// api.cu -- the extern "C" boundary of libbitlinear: host-side validation,
+// device checks and dispatch.  Every entry point is declared, with its
+// defining passage, in include/bitlinear.h.
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace bl {
+
+__device__ int g_dev_error = 0;
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+
+struct DevState {
+    std::once_flag once;
+    bool ok = false;
+    DevInfo info = {0, 0};
+};
+DevState g_dev[MAX_DEVICES];
+
+// Current device, checked once per device: present and compute capability 10.x.
+bl_status current_device(DevInfo& out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+        cudaGetLastError();
+        return BL_ERR_DEVICE;
+    }
+    DevState& s = g_dev[dev];
+    std::call_once(s.once, [&]() {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        if (prop.major != 10) return;
+        s.info.num_sms = prop.multiProcessorCount;
+        s.info.max_smem_optin = (int)prop.sharedMemPerBlockOptin;
+        s.ok = true;
+    });
+    if (!s.ok) return BL_ERR_DEVICE;
+    out = s.info;
+    return BL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+bl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// N, K limits shared by the weight calls
+bl_status check_nk(int64_t N, int64_t K, int64_t k_mult) {
+    if (N < 1 || K < 1 || K % k_mult != 0 || K > BL_MAX_K || N > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+bl_status check_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
+                        const float* beta, int64_t N, const void* y, size_t y_elem) {
+    if (!x_q || !W_p || !y || (y_elem != 4 && (!gamma || !beta))) return BL_ERR_NULL;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    if (!aligned16(x_q) || !aligned16(W_p) || !aligned16(y) || (gamma && !aligned16(gamma)) ||
+        (beta && !aligned16(beta)))
+        return BL_ERR_ALIGN;
+    const size_t ybytes = (size_t)M * N * y_elem;
+    if (overlap(y, ybytes, x_q, (size_t)M * K) || overlap(y, ybytes, W_p, (size_t)N * (K / 16) * 4) ||
+        overlap(y, ybytes, gamma, gamma ? (size_t)M * 4 : 0) || overlap(y, ybytes, beta, beta ? 4 : 0))
+        return BL_ERR_ALIAS;
+    return BL_OK;
+}
+
+constexpr int GEMV_MAX_M = 64;
+
+bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
+                      const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes, void* stream) {
+    const size_t need = bitlinear_forward_workspace(M, N, K);
+    if (need && (!ws || ws_bytes < need)) return BL_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return BL_ERR_ALIGN;
+    DevInfo dev;
+    bl_status s = current_device(dev);
+    if (s) return s;
+    cudaError_t e;
+    if (M <= GEMV_MAX_M)
+        e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
+    else
+        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
+    return from_cuda(e);
+}
+
+}  // namespace
+
+cudaError_t ensure_smem_optin(const void* kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<const void*, int>, size_t>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto& d : done)
+        if (d.first.first == kernel && d.first.second == dev && d.second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    for (auto& d : done)
+        if (d.first.first == kernel && d.first.second == dev) {
+            d.second = bytes;
+            return cudaSuccess;
+        }
+    done.push_back({{kernel, dev}, bytes});
+    return cudaSuccess;
+}
+
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" {
+
+const char* bitlinear_status_string(bl_status s) {
+    switch (s) {
+        case BL_OK: return "ok";
+        case BL_ERR_NULL: return "null pointer";
+        case BL_ERR_SHAPE: return "invalid shape";
+        case BL_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case BL_ERR_DTYPE: return "invalid dtype or combine mode";
+        case BL_ERR_WORKSPACE: return "workspace missing or too small";
+        case BL_ERR_DEVICE: return "no compute capability 10.x CUDA device";
+        case BL_ERR_CUDA: return "CUDA launch or runtime error";
+        case BL_ERR_TIMEOUT: return "bounded device wait expired";
+        case BL_ERR_ALIAS: return "output overlaps an input";
+    }
+    return "unknown status";
+}
+
+size_t bitlinear_quantize_weights_workspace(int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return quantize_weights_ws_bytes();
+}
+
+bl_status bitlinear_quantize_weights(const float* W, int64_t N, int64_t K, float eps, int8_t* W_t, float* beta,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    if (!W || !W_t || !beta) return BL_ERR_NULL;
+    bl_status s = check_nk(N, K, 16);
+    if (s) return s;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return BL_ERR_SHAPE;
+    if (!ws || ws_bytes < quantize_weights_ws_bytes()) return BL_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(W_t) || !aligned16(beta) || !aligned16(ws)) return BL_ERR_ALIGN;
+    const size_t n = (size_t)N * K;
+    if (overlap(W_t, n, W, n * 4) || overlap(beta, 4, W, n * 4) || overlap(W_t, n, beta, 4) ||
+        overlap(ws, ws_bytes, W, n * 4) || overlap(ws, ws_bytes, W_t, n) || overlap(ws, ws_bytes, beta, 4))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_quantize_weights(W, (long long)n, eps, W_t, beta, ws, dev.num_sms, as_stream(stream)));
+}
+
+bl_status bitlinear_pack(const int8_t* W_t, int64_t N, int64_t K, uint32_t* W_p, void* stream) {
+    if (!W_t || !W_p) return BL_ERR_NULL;
+    bl_status s = check_nk(N, K, 16);
+    if (s) return s;
+    if (!aligned16(W_t) || !aligned16(W_p)) return BL_ERR_ALIGN;
+    const size_t n = (size_t)N * K;
+    if (overlap(W_p, n / 4, W_t, n)) return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_pack(W_t, (long long)(n / 16), W_p, dev.num_sms, as_stream(stream)));
+}
+
+bl_status bitlinear_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, int8_t* x_q, float* gamma,
+                              void* stream) {
+    if (!x || !x_q || !gamma) return BL_ERR_NULL;
+    if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_DTYPE;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(1, K, 16);
+    if (s) return s;
+    if (!aligned16(x) || !aligned16(x_q) || !aligned16(gamma)) return BL_ERR_ALIGN;
+    const size_t xb = (size_t)M * K * (x_dtype == BL_BF16 ? 2 : 4);
+    if (overlap(x_q, (size_t)M * K, x, xb) || overlap(gamma, (size_t)M * 4, x, xb) ||
+        overlap(gamma, (size_t)M * 4, x_q, (size_t)M * K))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream)));
+}
+
+size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K) {
+    if (M <= GEMV_MAX_M) return 0;
+    return gemm_ws_bytes(M, N, K);
+}
+
+bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
+                            const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                            void* stream) {
+    if (y_dtype != BL_F32 && y_dtype != BL_BF16) {
+        if (!x_q || !gamma || !W_p || !beta || !y) return BL_ERR_NULL;
+        return BL_ERR_DTYPE;
+    }
+    const size_t ye = y_dtype == BL_F32 ? 4 : 2;
+    if (!gamma || !beta) return BL_ERR_NULL;
+    bl_status s = check_forward(x_q, gamma, M, K, W_p, beta, N, y, ye);
+    if (s) return s;
+    return run_forward(x_q, gamma, M, K, W_p, beta, N, y, y_dtype == BL_F32 ? Y_F32 : Y_BF16, ws, ws_bytes, stream);
+}
+
+bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,
+                                int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
+    bl_status s = check_forward(x_q, nullptr, M, K, W_p, nullptr, N, acc, 4);
+    if (s) return s;
+    return run_forward(x_q, nullptr, M, K, W_p, nullptr, N, acc, Y_ACC, ws, ws_bytes, stream);
+}
+
+bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, int64_t M, int64_t K, float* h,
+                                  int8_t* x_q, float* gamma, void* stream) {
+    if (combine != BL_COMBINE_NONE && combine != BL_COMBINE_ADD && combine != BL_COMBINE_SILU_MUL)
+        return BL_ERR_DTYPE;
+    if (!a || (combine != BL_COMBINE_NONE && !b)) return BL_ERR_NULL;
+    if ((x_q == nullptr) != (gamma == nullptr)) return BL_ERR_NULL;
+    if (!x_q && !h) return BL_ERR_NULL;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(1, K, 16);
+    if (s) return s;
+    if (!aligned16(a) || (b && !aligned16(b)) || (h && !aligned16(h)) || (x_q && !aligned16(x_q)) ||
+        (gamma && !aligned16(gamma)))
+        return BL_ERR_ALIGN;
+    const size_t fb = (size_t)M * K * 4;
+    const void* ins[2] = {a, combine != BL_COMBINE_NONE ? b : nullptr};
+    for (const void* in : ins) {
+        if (!in) continue;
+        if (overlap(h, h ? fb : 0, in, fb) || overlap(x_q, x_q ? (size_t)M * K : 0, in, fb) ||
+            overlap(gamma, gamma ? (size_t)M * 4 : 0, in, fb))
+            return BL_ERR_ALIAS;
+    }
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_quant_act_rms(a, combine != BL_COMBINE_NONE ? b : nullptr, combine, M, K, h, x_q, gamma,
+                                          as_stream(stream)));
+}
+
+bl_status bitlinear_device_status(void* stream) {
+    DevInfo dev;
+    bl_status s = current_device(dev);
+    if (s) return s;
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BL_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+    if (v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+        return BL_ERR_TIMEOUT;
+    }
+    return BL_OK;
+}
+
+int bitlinear_num_sms(void) {
+    DevInfo dev;
+    if (current_device(dev)) return 0;
+    return dev.num_sms;
+}
+
+}  // extern "C"

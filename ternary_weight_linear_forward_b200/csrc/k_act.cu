@@ -1,0 +1,209 @@
+// k_act.cu -- per-token absmax int8 activation quantisers.
+//
+// unite.ai "Microsofts Inference Framework bringt 1-Bit grosse Sprachmodelle
+// auf lokale Geraete", "Mathematische Grundlagen", eq. 2
+// "Aktivierungsquantisierung": x_hat = Clip(x * Q_b / gamma, ...), gamma =
+// ||x||_inf.  Here Q_b = 127, gamma is per token and floored at 1e-5, the
+// scale s = 127 / gamma is formed first (IEEE divide) and x * s is rounded to
+// nearest-even and clamped to [-127, 127].
+//
+// One CTA per token row: pass 1 reduces max |x| (and, for the RMSNorm form,
+// sum x^2 in binary64), pass 2 re-reads the row from L1/L2 and writes 16
+// codes per thread per step with one 16-byte store.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace bl {
+
+namespace {
+
+constexpr int ACT_THREADS = 256;
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+    return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
+           ((uint32_t)(d & 0xFF) << 24);
+}
+
+__device__ __forceinline__ int q8(float v, float s) {
+    int r = __float2int_rn(__fmul_rn(v, s));
+    return min(max(r, -127), 127);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 16 consecutive activations of group g (k = 16g .. 16g+15) as fp32.
+template <bool BF16>
+__device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
+    if (BF16) {
+        const uint4* p = reinterpret_cast<const uint4*>(row) + 2 * g;
+        uint4 a = __ldg(p), b = __ldg(p + 1);
+        uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[2 * i] = bf16lo(w[i]);
+            v[2 * i + 1] = bf16hi(w[i]);
+        }
+    } else {
+        const float4* p = reinterpret_cast<const float4*>(row) + 4 * g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float4 f = __ldg(p + i);
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+    }
+}
+
+__device__ __forceinline__ void store16(int8_t* row_q, int g, const float (&v)[16], float s) {
+    uint4 o;
+    o.x = pack4(q8(v[0], s), q8(v[1], s), q8(v[2], s), q8(v[3], s));
+    o.y = pack4(q8(v[4], s), q8(v[5], s), q8(v[6], s), q8(v[7], s));
+    o.z = pack4(q8(v[8], s), q8(v[9], s), q8(v[10], s), q8(v[11], s));
+    o.w = pack4(q8(v[12], s), q8(v[13], s), q8(v[14], s), q8(v[15], s));
+    reinterpret_cast<uint4*>(row_q)[g] = o;
+}
+
+// block-wide max of non-negative floats (compared as bit patterns)
+__device__ __forceinline__ float block_max_nonneg(float v, unsigned* sm) {
+    unsigned u = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) sm[warp] = u;
+    __syncthreads();
+    unsigned r = lane < ACT_THREADS / 32 ? sm[lane] : 0u;
+    r = __reduce_max_sync(0xffffffffu, r);
+    __syncthreads();
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ double block_sum_f64(double v, double* sm) {
+    for (int off = 16; off; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    double r = lane < ACT_THREADS / 32 ? sm[lane] : 0.0;
+    for (int off = 16; off; off >>= 1) r = __dadd_rn(r, __shfl_xor_sync(0xffffffffu, r, off));
+    __syncthreads();
+    return r;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(ACT_THREADS) quant_act_kernel(const void* __restrict__ x, int K,
+                                                                int8_t* __restrict__ x_q, float* __restrict__ gamma) {
+    __shared__ unsigned sm[ACT_THREADS / 32];
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long row = blockIdx.x;
+    const char* xr = reinterpret_cast<const char*>(x) + row * (long long)K * (BF16 ? 2 : 4);
+    const int G = K / 16;
+    float amax = 0.0f;
+    for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
+        float v[16];
+        load16<BF16>(xr, g, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+    amax = block_max_nonneg(amax, sm);
+    const float gm = fmaxf(amax, 1e-5f);
+    const float s = __fdiv_rn(127.0f, gm);
+    int8_t* qr = x_q + row * (long long)K;
+    for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
+        float v[16];
+        load16<BF16>(xr, g, v);
+        store16(qr, g, v, s);
+    }
+    if (threadIdx.x == 0) gamma[row] = gm;
+}
+
+// h = combine(a, b) for 16 consecutive elements of group g.
+__device__ __forceinline__ void combine16(const float* ar, const float* br, int combine, int g, float (&h)[16]) {
+    const float4* pa = reinterpret_cast<const float4*>(ar) + 4 * g;
+    const float4* pb = reinterpret_cast<const float4*>(br) + 4 * g;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float4 va = __ldg(pa + i);
+        float av[4] = {va.x, va.y, va.z, va.w};
+        if (combine == C_NONE) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[4 * i + j] = av[j];
+        } else {
+            float4 vb = __ldg(pb + i);
+            float bv[4] = {vb.x, vb.y, vb.z, vb.w};
+            if (combine == C_ADD) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) h[4 * i + j] = __fadd_rn(av[j], bv[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    double gd = (double)av[j];
+                    double sg = __ddiv_rn(gd, __dadd_rn(1.0, exp(-gd)));
+                    h[4 * i + j] = __double2float_rn(__dmul_rn(sg, (double)bv[j]));
+                }
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(ACT_THREADS) quant_act_rms_kernel(const float* __restrict__ a,
+                                                                    const float* __restrict__ b, int combine, int K,
+                                                                    float* __restrict__ h, int8_t* __restrict__ x_q,
+                                                                    float* __restrict__ gamma) {
+    __shared__ unsigned smu[ACT_THREADS / 32];
+    __shared__ double smd[ACT_THREADS / 32];
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long row = blockIdx.x;
+    const float* ar = a + row * (long long)K;
+    const float* br = b ? b + row * (long long)K : nullptr;
+    float* hr = h ? h + row * (long long)K : nullptr;
+    const int G = K / 16;
+    float amax = 0.0f;
+    double ss = 0.0;
+    for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
+        float v[16];
+        combine16(ar, br, combine, g, v);
+        if (hr) {
+            float4* ph = reinterpret_cast<float4*>(hr) + 4 * g;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ph[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            amax = fmaxf(amax, fabsf(v[i]));
+            ss = __dadd_rn(ss, __dmul_rn((double)v[i], (double)v[i]));
+        }
+    }
+    if (!x_q) return;
+    amax = block_max_nonneg(amax, smu);
+    ss = block_sum_f64(ss, smd);
+    const float gm = fmaxf(amax, 1e-5f);
+    const float s = __fdiv_rn(127.0f, gm);
+    const double ms = __dadd_rn(__ddiv_rn(ss, (double)K), 1e-6);
+    const float rho = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(ms)));
+    int8_t* qr = x_q + row * (long long)K;
+    for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
+        float v[16];
+        combine16(ar, br, combine, g, v);
+        store16(qr, g, v, s);
+    }
+    if (threadIdx.x == 0) gamma[row] = __fmul_rn(rho, gm);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
+                             cudaStream_t st) {
+    if (bf16)
+        return launch_pdl(quant_act_kernel<true>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
+    return launch_pdl(quant_act_kernel<false>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
+}
+
+cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,
+                                 int8_t* x_q, float* gamma, cudaStream_t st) {
+    return launch_pdl(quant_act_rms_kernel, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, a, b, combine, (int)K, h,
+                      x_q, gamma);
+}
+
+}  // namespace bl

@@ -1,0 +1,66 @@
+// kernels.cuh -- host-side launchers of libbitlinear's kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace bl {
+
+constexpr int PREP_MAX_GRID = 1024;
+
+// Output modes of the forward kernels.
+enum YMode : int { Y_F32 = 0, Y_BF16 = 1, Y_ACC = 2 };
+
+// Combine modes of the block-glue quantiser (match BL_COMBINE_*).
+enum Combine : int { C_NONE = 0, C_ADD = 1, C_SILU_MUL = 2 };
+
+struct DevInfo {
+    int num_sms;
+    int max_smem_optin;
+};
+
+// k_prep.cu
+size_t quantize_weights_ws_bytes();
+cudaError_t launch_quantize_weights(const float* W, long long n, float eps, int8_t* W_t, float* beta, void* ws,
+                                    int num_sms, cudaStream_t st);
+cudaError_t launch_pack(const int8_t* W_t, long long nwords, uint32_t* W_p, int num_sms, cudaStream_t st);
+
+// k_act.cu
+cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
+                             cudaStream_t st);
+cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,
+                                 int8_t* x_q, float* gamma, cudaStream_t st);
+
+// k_gemv.cu  (M <= 64, CUDA cores)
+cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
+                        int N, void* y, YMode mode, const DevInfo& dev, cudaStream_t st);
+
+// k_gemm.cu  (M > 64, tcgen05 int8 tensor cores)
+size_t gemm_ws_bytes(long long M, long long N, long long K);
+cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st);
+
+// Raise a kernel's dynamic shared-memory limit once per device (api.cu).
+cudaError_t ensure_smem_optin(const void* kernel, size_t bytes);
+
+// launch helper: every per-token kernel is launched with programmatic stream
+// serialisation so it can start while its predecessor drains.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace bl

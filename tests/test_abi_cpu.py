@@ -1,0 +1,142 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects invalid arguments on the host before touching a
+device (no compute is launched here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_weight_linear_forward_b200 as bl
+from ternary_weight_linear_forward_b200 import bitlinear as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+OK, NULL, SHAPE, ALIGN, DTYPE, WS, DEVICE, CUDA, TIMEOUT, ALIAS = range(10)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_four_core_calls():
+    names = declared_functions()
+    for core in ("bitlinear_quantize_weights", "bitlinear_pack", "bitlinear_quant_act", "bitlinear_forward"):
+        assert core in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = bl.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in B.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings():
+    for s in range(10):
+        assert bl.status_string(s)
+    assert bl.status_string(0) == "ok"
+    assert bl.status_string(12345) == "unknown status"
+
+
+# fake, never-dereferenced device addresses: 16-byte aligned and disjoint
+A1, A2, A3, A4, A5, A6 = (0x10000000 * i for i in range(1, 7))
+L = None
+
+
+def _L():
+    global L
+    if L is None:
+        L = bl.lib()
+    return L
+
+
+def P(x):
+    return ctypes.c_void_p(x)
+
+
+def test_forward_validation_order():
+    f = _L().bitlinear_forward
+    assert f(None, P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == NULL
+    assert f(P(A1), P(A2), 1, 1000, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == SHAPE   # K % 64
+    assert f(P(A1), P(A2), 0, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == SHAPE   # M < 1
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 0, P(A5), 0, None, 0, None) == SHAPE    # N < 1
+    assert f(P(A1), P(A2), 1, 2 ** 19, P(A3), P(A4), 8, P(A5), 0, None, 0, None) == SHAPE  # K > max
+    assert f(P(A1 + 8), P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == ALIGN
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 7, None, 0, None) == DTYPE
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A1), 0, None, 0, None) == ALIAS
+    # prefill path needs a workspace
+    assert _L().bitlinear_forward_workspace(2048, 4096, 4096) >= 2048 * 4
+    assert f(P(A1), P(A2), 2048, 1024, P(A3), P(A4), 64, P(A5), 1, None, 0, None) == WS
+    # everything valid: without a CUDA device the call stops at the device check
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DEVICE
+
+
+def test_forward_acc_validation():
+    f = _L().bitlinear_forward_acc
+    assert f(None, 1, 1024, P(A3), 64, P(A5), None, 0, None) == NULL
+    assert f(P(A1), 1, 1040, P(A3), 64, P(A5), None, 0, None) == SHAPE
+    assert f(P(A1), 1, 1024, P(A3), 64, P(A5 + 4), None, 0, None) == ALIGN
+    assert f(P(A1), 1, 1024, P(A3), 64, P(A5), None, 0, None) == DEVICE
+
+
+def test_quantize_weights_validation():
+    f = _L().bitlinear_quantize_weights
+    ws = _L().bitlinear_quantize_weights_workspace(16, 16)
+    assert ws > 0
+    assert f(None, 16, 16, 1e-5, P(A2), P(A3), P(A4), ws, None) == NULL
+    assert f(P(A1), 16, 8, 1e-5, P(A2), P(A3), P(A4), ws, None) == SHAPE      # K % 16
+    assert f(P(A1), 16, 16, -1.0, P(A2), P(A3), P(A4), ws, None) == SHAPE     # eps < 0
+    assert f(P(A1), 16, 16, float("nan"), P(A2), P(A3), P(A4), ws, None) == SHAPE
+    assert f(P(A1), 16, 16, 1e-5, P(A2), P(A3), P(A4), ws - 1, None) == WS
+    assert f(P(A1), 16, 16, 1e-5, P(A2), P(A3), None, 0, None) == WS
+    assert f(P(A1), 16, 16, 1e-5, P(A2 + 1), P(A3), P(A4), ws, None) == ALIGN
+    assert f(P(A1), 16, 16, 1e-5, P(A1), P(A3), P(A4), ws, None) == ALIAS
+    assert f(P(A1), 16, 16, 1e-5, P(A2), P(A3), P(A4), ws, None) == DEVICE
+
+
+def test_pack_and_quant_act_validation():
+    pk = _L().bitlinear_pack
+    assert pk(None, 4, 16, P(A2), None) == NULL
+    assert pk(P(A1), 4, 24, P(A2), None) == SHAPE
+    assert pk(P(A1), 4, 16, P(A2 + 4), None) == ALIGN
+    assert pk(P(A1), 4, 16, P(A1), None) == ALIAS
+    assert pk(P(A1), 4, 16, P(A2), None) == DEVICE
+    qa = _L().bitlinear_quant_act
+    assert qa(P(A1), 0, 1, 1024, None, P(A3), None) == NULL
+    assert qa(P(A1), 2, 1, 1024, P(A2), P(A3), None) == DTYPE
+    assert qa(P(A1), 1, 1, 1000, P(A2), P(A3), None) == SHAPE
+    assert qa(P(A1), 1, 0, 1024, P(A2), P(A3), None) == SHAPE
+    assert qa(P(A1 + 2), 1, 1, 1024, P(A2), P(A3), None) == ALIGN
+    assert qa(P(A1), 0, 1, 1024, P(A1 + 16), P(A3), None) == ALIAS
+    assert qa(P(A1), 1, 1, 1024, P(A2), P(A3), None) == DEVICE
+
+
+def test_quant_act_rms_validation():
+    f = _L().bitlinear_quant_act_rms
+    assert f(P(A1), None, 9, 1, 64, None, P(A2), P(A3), None) == DTYPE
+    assert f(P(A1), None, 1, 1, 64, None, P(A2), P(A3), None) == NULL       # add needs b
+    assert f(P(A1), None, 0, 1, 64, None, P(A2), None, None) == NULL        # x_q without gamma
+    assert f(P(A1), None, 0, 1, 64, None, None, None, None) == NULL         # nothing to write
+    assert f(P(A1), None, 0, 1, 60, None, P(A2), P(A3), None) == SHAPE
+    assert f(P(A1), P(A4), 2, 1, 64, P(A4), P(A2), P(A3), None) == ALIAS
+    assert f(P(A1), None, 0, 1, 64, None, P(A2), P(A3), None) == DEVICE
+
+
+def test_device_queries_without_gpu():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    assert _L().bitlinear_num_sms() == 0
+    assert _L().bitlinear_device_status(None) == DEVICE
+
+
+def test_binding_type_checks():
+    import torch
+    with pytest.raises(TypeError):
+        bl.quant_act(torch.zeros(2, 64, dtype=torch.float16))
+    with pytest.raises((TypeError, ValueError)):
+        bl.pack(torch.zeros(2, 64, dtype=torch.int8))       # CPU tensor

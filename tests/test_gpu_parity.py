@@ -1,0 +1,233 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integers (ternary codes, packed words, int8 activations, int32 accumulators)
+must match bit for bit; the absmean scale beta and the per-token gamma too
+(both are binary32 values that decide integer codes, computed in the same
+precision on both sides).  Float outputs must lie within 1e-6 relative error
+of the oracle's binary64 rescale; bf16 outputs must be one of the bf16
+roundings of a value within that tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import ternary_weight_linear_forward_b200 as bl
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-6
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    d = torch.device("cuda:0")
+    torch.cuda.set_device(d)
+    return d
+
+
+@pytest.fixture(autouse=True)
+def _status_clean(dev):
+    yield
+    bl.device_status()
+
+
+def T(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def gpu_prep(W, dev):
+    W_t, beta = bl.quantize_weights(T(W, dev))
+    return W_t, beta, bl.pack(W_t)
+
+
+def assert_f32_close(y_gpu, y64):
+    y = y_gpu.astype(np.float64)
+    nz = y64 != 0
+    assert np.all(y[~nz] == 0)
+    if nz.any():
+        rel = np.abs(y[nz] - y64[nz]) / np.abs(y64[nz])
+        assert rel.max() <= REL_TOL, f"max rel err {rel.max():.3g}"
+
+
+def assert_bf16_ok(y_bits, y64):
+    lo = oracle.to_bf16((y64 * (1 - REL_TOL)).astype(np.float32))
+    hi = oracle.to_bf16((y64 * (1 + REL_TOL)).astype(np.float32))
+    ok = (y_bits == lo) | (y_bits == hi)
+    assert ok.all(), f"{(~ok).sum()} bf16 outputs outside tolerance"
+
+
+# --------------------------------------------------------------------------
+# weight preparation
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,seed", [(1, 16, 0), (7, 48, 1), (300, 1024, 2), (1024, 1024, 3),
+                                      (149, 4096, 4), (4096, 11008, 1002), (11008, 4096, 1012)])
+def test_quantize_and_pack_bit_exact(dev, N, K, seed):
+    W = workloads.latent_weights(seed, N, K)
+    W_t, beta, W_p = gpu_prep(W, dev)
+    oW_t, obeta = oracle.quantize_weights(W)
+    assert beta.item() == float(obeta)
+    np.testing.assert_array_equal(W_t.cpu().numpy(), oW_t)
+    np.testing.assert_array_equal(W_p.cpu().numpy().view(np.uint32), oracle.pack(oW_t))
+
+
+def test_quantize_special_matrices(dev):
+    z = np.zeros((8, 32), np.float32)
+    W_t, beta, W_p = gpu_prep(z, dev)
+    assert beta.item() == 0.0 and not W_t.any()
+    assert np.all(W_p.cpu().numpy().view(np.uint32) == 0x55555555)
+    # mean |W| = 1 exactly and eps = 0: q = W, so +-0.5 ties go to 0, +-1.5 clips to +-1
+    W = np.array([[0.5, -0.5, 1.5, -1.5] * 4] * 3, np.float32)
+    W_t, beta = bl.quantize_weights(T(W, dev), eps=0.0)
+    assert beta.item() == 1.0
+    np.testing.assert_array_equal(W_t.cpu().numpy(), oracle.ternarize(W, 1.0, 0.0))
+    np.testing.assert_array_equal(W_t.cpu().numpy()[0, :4], [0, 0, 1, -1])
+    # wide dynamic range (no element below 2^-38 of the max, so the sum is exact)
+    g = np.random.default_rng(5)
+    W = (g.standard_normal((64, 256)) * np.exp(g.uniform(-20, 20, (64, 256)))).astype(np.float32)
+    W_t, beta, _ = gpu_prep(W, dev)
+    oW_t, obeta = oracle.quantize_weights(W)
+    assert beta.item() == float(obeta)
+    np.testing.assert_array_equal(W_t.cpu().numpy(), oW_t)
+
+
+def test_pack_of_arbitrary_trits(dev):
+    g = np.random.default_rng(6)
+    W_t = g.integers(-1, 2, size=(333, 16 * 37)).astype(np.int8)
+    W_p = bl.pack(T(W_t, dev))
+    np.testing.assert_array_equal(W_p.cpu().numpy().view(np.uint32), oracle.pack(W_t))
+
+
+# --------------------------------------------------------------------------
+# activation quantiser
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,dtype", [(1, 16, "f32"), (1, 4096, "bf16"), (1, 11008, "bf16"), (5, 1024, "f32"),
+                                       (64, 4096, "f32"), (2048, 4096, "f32"), (3, 2560, "bf16")])
+def test_quant_act_bit_exact(dev, M, K, dtype):
+    x = workloads.activations(100 + M, M, K, outliers=True)
+    if dtype == "bf16":
+        bits = workloads.bf16_bits(x)
+        xt = T(bits.view(np.int16), dev).view(torch.bfloat16)
+        x = workloads.bf16_to_f32(bits)
+    else:
+        xt = T(x, dev)
+    x_q, gamma = bl.quant_act(xt)
+    ox_q, og = oracle.quant_act(x)
+    np.testing.assert_array_equal(x_q.cpu().numpy(), ox_q)
+    np.testing.assert_array_equal(gamma.cpu().numpy(), og)
+
+
+def test_quant_act_edge_rows(dev):
+    x = np.zeros((4, 64), np.float32)
+    x[1, 5] = 3e-6                       # below the gamma floor
+    x[2, :4] = [1, -2, 0.5, 4]           # the hand-worked token: -63.5 -> -64
+    x[3, :4] = [127, 62.5, -0.5, 1.5]    # ties to even: 62, 0, 2
+    x_q, gamma = bl.quant_act(T(x, dev))
+    ox_q, og = oracle.quant_act(x)
+    np.testing.assert_array_equal(x_q.cpu().numpy(), ox_q)
+    np.testing.assert_array_equal(gamma.cpu().numpy(), og)
+    np.testing.assert_array_equal(x_q.cpu().numpy()[3, :4], [127, 62, 0, 2])
+
+
+# --------------------------------------------------------------------------
+# forward: accumulators bit-exact, outputs within tolerance
+# --------------------------------------------------------------------------
+
+def run_case(dev, M, K, N, seed, x_dtype="f32", y_dtype="f32", outliers=False):
+    W = workloads.latent_weights(seed, N, K)
+    x = workloads.activations(seed + 7, M, K, outliers)
+    if x_dtype == "bf16":
+        bits = workloads.bf16_bits(x)
+        xt = T(bits.view(np.int16), dev).view(torch.bfloat16)
+        x = workloads.bf16_to_f32(bits)
+    else:
+        xt = T(x, dev)
+    W_t, beta, W_p = gpu_prep(W, dev)
+    oW_t, obeta = oracle.quantize_weights(W)
+    x_q, gamma = bl.quant_act(xt)
+    acc = bl.forward_acc(x_q, W_p)
+    y = bl.forward(x_q, gamma, W_p, beta, out_dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32)
+    ref = oracle.forward(x, oW_t, obeta)
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref["acc"])
+    if y_dtype == "bf16":
+        assert_bf16_ok(y.cpu().view(torch.int16).numpy().view(np.uint16), ref["y64"])
+    else:
+        yv = y.cpu().numpy()
+        assert_f32_close(yv, ref["y64"])
+        np.testing.assert_array_equal(yv, ref["y"])      # same binary32 op order: identical
+    return ref
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 16, 33, 64])
+@pytest.mark.parametrize("K,N", [(64, 5), (1024, 148), (1024, 149), (2560, 1000), (6912, 300)])
+def test_gemv_parity_sweep(dev, M, K, N):
+    run_case(dev, M, K, N, seed=10 * M + K % 97 + N)
+
+
+@pytest.mark.parametrize("K", [64, 128, 1024, 1088, 2048, 2560, 4096, 6912, 11008, 16384, 16448, 32768])
+def test_gemv_m1_all_team_shapes(dev, K):
+    run_case(dev, 1, K, 333, seed=K)
+
+
+@pytest.mark.parametrize("N", [1, 2, 147, 148, 149, 296, 5000])
+def test_gemv_row_partition_tails(dev, N):
+    run_case(dev, 1, 4096, N, seed=N)
+    run_case(dev, 5, 1024, N, seed=N + 1)
+
+
+def test_gemv_bf16_output(dev):
+    run_case(dev, 1, 4096, 2000, 21, y_dtype="bf16")
+    run_case(dev, 9, 2560, 700, 22, y_dtype="bf16")
+
+
+def test_gemv_extreme_values(dev):
+    # every activation at +-127 and every weight +1: |acc| = 127 K at the int32 bound of the kernel
+    K, N = 11008, 64
+    x_q = torch.full((1, K), 127, dtype=torch.int8, device=dev)
+    x_q[0, 1::2] = -127
+    W_t = np.ones((N, K), np.int8)
+    W_t[1::2] = -1
+    W_t[2] = 0
+    W_p = bl.pack(T(W_t, dev))
+    acc = bl.forward_acc(x_q, W_p).cpu().numpy()
+    np.testing.assert_array_equal(acc, oracle.ternary_acc(x_q.cpu().numpy(), W_t))
+    x_q.fill_(127)
+    acc = bl.forward_acc(x_q, W_p).cpu().numpy()
+    assert acc[0, 0] == 127 * K and acc[0, 1] == -127 * K and acc[0, 2] == 0
+
+
+# --------------------------------------------------------------------------
+# the workloads at full size
+# --------------------------------------------------------------------------
+
+def test_workload_single_layer_m1_k1024(dev):
+    s = workloads.W1.shapes[0]
+    run_case(dev, s.M, s.K, s.N, s.w_seed)
+
+
+@pytest.mark.parametrize("shape", workloads.W2.shapes, ids=lambda s: s.name)
+def test_workload_decode_m1_bf16(dev, shape):
+    # the bench's workload, same weights, activations and launch path
+    W = shape.weights()
+    bits = shape.inputs_bf16_bits()
+    x = workloads.bf16_to_f32(bits)
+    W_t, beta, W_p = gpu_prep(W, dev)
+    oW_t, obeta = oracle.quantize_weights(W)
+    x_q, gamma = bl.quant_act(T(bits.view(np.int16), dev).view(torch.bfloat16))
+    y = bl.forward(x_q, gamma, W_p, beta)
+    ref = oracle.forward(x, oW_t, obeta)
+    np.testing.assert_array_equal(x_q.cpu().numpy(), ref["x_q"])
+    np.testing.assert_array_equal(bl.forward_acc(x_q, W_p).cpu().numpy(), ref["acc"])
+    assert_f32_close(y.cpu().numpy(), ref["y64"])
+    zero_frac = float((W_t == 0).float().mean())
+    assert abs(zero_frac - 0.3101) < 2e-3
+
+
+@pytest.mark.parametrize("shape", workloads.W3.shapes, ids=lambda s: s.name)
+def test_workload_small_batch(dev, shape):
+    run_case(dev, shape.M, shape.K, shape.N, shape.w_seed)
