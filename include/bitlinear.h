@@ -148,6 +148,24 @@ bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, in
                             const uint32_t* W_p, const float* beta, int64_t N,
                             void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace bitlinear_forward_fp needs for this shape (may be 0). */
+size_t bitlinear_forward_fp_workspace(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Quantise + forward in one call, the shape of the forward function sketched
+ * in [BNC] "Implementierungshinweise" (quantise the input, ternary matmul,
+ * scale): bitlinear_quant_act(x) followed by bitlinear_forward, with results
+ * bit-identical to those two calls.  For M <= 4 tokens with
+ * (M rounded up to 1, 2 or 4) * K <= 65536 the quantiser runs in the GEMV
+ * prologue (one kernel, workspace 0); otherwise x_q and gamma are staged in
+ * the workspace and the two kernels run back to back.
+ *   x  [M, K] float32 (BL_F32) or bfloat16 (BL_BF16) in; other arguments as
+ *   for bitlinear_forward.  K % 64 == 0, K <= BL_MAX_K.
+ */
+bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* W_p,
+                               const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /*
  * Inspection variant of bitlinear_forward: writes the int32 accumulators
  * acc[M, N] = sum_k W_t[n, k] * x_q[m, k] instead of y (same kernels, same

@@ -34,6 +34,8 @@ SIGNATURES = {
     "bitlinear_quant_act": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
     "bitlinear_forward_workspace": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_fp_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_forward_fp": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_device_status": (_I, [_P]),
@@ -168,6 +170,31 @@ def forward(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: tor
     return out
 
 
+def forward_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype=torch.float32, out=None,
+               ws=None, stream=None) -> torch.Tensor:
+    """quant_act + forward in one call (one kernel for M <= 4); bit-identical to the two calls."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, 2, "x")
+    _need(W_p, torch.int32, 2, "W_p")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x.shape
+    N = W_p.shape[0]
+    if W_p.shape[1] * 16 != K:
+        raise ValueError("W_p must be [N, K/16]")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = int(lib().bitlinear_forward_fp_workspace(M, N, K))
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x.device)
+    xdt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_forward_fp",
+           lib().bitlinear_forward_fp(_ptr(x), xdt, M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt, _ptr(ws),
+                                      0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
 def forward_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
     """int32 accumulators acc[m, n] = sum_k W_t[n, k] x_q[m, k] (same kernels as forward)."""
     _need(x_q, torch.int8, 2, "x_q")
@@ -237,8 +264,7 @@ class BitLinear:
         return cls(pack(W_t), beta)
 
     def __call__(self, x: torch.Tensor, out_dtype=torch.float32, out=None) -> torch.Tensor:
-        x_q, gamma = quant_act(x)
-        return forward(x_q, gamma, self.W_p, self.beta, out_dtype=out_dtype, out=out)
+        return forward_fp(x, self.W_p, self.beta, out_dtype=out_dtype, out=out)
 
 
 class DecoderBlock:

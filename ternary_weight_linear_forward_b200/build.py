@@ -65,7 +65,7 @@ def build(force: bool = False, verbose: bool = False, extra: list | None = None)
     with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(compile_one, _sources()))
     tmp = LIB + ".tmp"
-    cmd = [nv, *ARCH, "-shared", "-rdc=true", *objs, "-o", tmp, "-lcuda"]
+    cmd = [nv, *ARCH, "-shared", "-rdc=true", *objs, "-o", tmp,]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n" + r.stderr)

@@ -216,6 +216,47 @@ bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, in
     return run_forward(x_q, gamma, M, K, W_p, beta, N, y, y_dtype == BL_F32 ? Y_F32 : Y_BF16, ws, ws_bytes, stream);
 }
 
+static size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+size_t bitlinear_forward_fp_workspace(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || K < 1) return 0;
+    if (gemv_fused_quant_ok(M, K)) return 0;
+    return round256((size_t)M * K) + round256((size_t)M * 4) + bitlinear_forward_workspace(M, N, K);
+}
+
+bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* W_p,
+                               const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                               void* stream) {
+    if (!x || !W_p || !beta || !y) return BL_ERR_NULL;
+    if ((x_dtype != BL_F32 && x_dtype != BL_BF16) || (y_dtype != BL_F32 && y_dtype != BL_BF16)) return BL_ERR_DTYPE;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    if (!aligned16(x) || !aligned16(W_p) || !aligned16(beta) || !aligned16(y)) return BL_ERR_ALIGN;
+    const size_t ye = y_dtype == BL_F32 ? 4 : 2;
+    const size_t ybytes = (size_t)M * N * ye, xb = (size_t)M * K * (x_dtype == BL_BF16 ? 2 : 4);
+    if (overlap(y, ybytes, x, xb) || overlap(y, ybytes, W_p, (size_t)N * (K / 16) * 4) || overlap(y, ybytes, beta, 4))
+        return BL_ERR_ALIAS;
+    const size_t need = bitlinear_forward_fp_workspace(M, N, K);
+    if (need && (!ws || ws_bytes < need)) return BL_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return BL_ERR_ALIGN;
+    if (need && (overlap(ws, need, x, xb) || overlap(ws, need, y, ybytes))) return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
+    if (!need)
+        return from_cuda(launch_gemv_fused(x, x_dtype == BL_BF16, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev,
+                                           as_stream(stream)));
+    int8_t* x_q = reinterpret_cast<int8_t*>(ws);
+    float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
+    char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * 4);
+    cudaError_t e = launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream));
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    return run_forward(x_q, gamma, M, K, W_p, beta, N, y, mode, fws, ws_bytes - (fws - reinterpret_cast<char*>(ws)),
+                       stream);
+}
+
 bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,
                                 int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
     bl_status s = check_forward(x_q, nullptr, M, K, W_p, nullptr, N, acc, 4);

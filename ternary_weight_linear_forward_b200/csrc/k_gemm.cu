@@ -1,8 +1,393 @@
 // k_gemm.cu -- prefill BitLinear forward (M > 64) on tcgen05 int8 tensor cores.
+//
+// unite.ai "Microsofts Inference Framework bringt 1-Bit grosse Sprachmodelle
+// auf lokale Geraete", eq. 3 "BitLinear-Betrieb": y = W_f x_hat (beta gamma /
+// Q_b).  With many tokens the ternary contraction is a dense int8 GEMM, so it
+// runs on the 5th-generation tensor cores:
+//
+//   D[m, n] = sum_k x_q[m, k] * c[n, k]      (c = w + 1 in {0, 1, 2}, s8 x s8 -> s32)
+//   acc     = D[m, n] - rowsum_m             (rowsum_m = sum_k x_q[m, k])
+//   y       = (float)acc * ((beta * gamma_m) / 127)
+//
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles, K in blocks of
+// 128 bytes.  Warp roles:
+//   warp 0      TMA producer: x_q tile (128 x 128 B, 128-byte swizzle) and the
+//               packed weight tile (256 rows x 8 words) per K-block, no multicast;
+//   warp 1      TMEM allocation and the single-thread tcgen05.mma issuer
+//               (4 MMAs of K = 32 per K-block), tcgen05.commit to free stages;
+//   warps 2-5   unpack: packed word -> four registers of codes (w >> 2s) &
+//               0x03030303, i.e. 16 consecutive-k bytes, stored as one 16-byte
+//               chunk into the 128-byte-swizzled K-major operand layout;
+//   warps 6-9   epilogue: tcgen05.ld of the int32 accumulators (32 TMEM lanes
+//               per warp), rowsum correction, rescale, bf16/fp32 store.
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap
+// the main loop of tile t + 1.  Every mbarrier wait is bounded.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace bl {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;  // bytes of K per stage
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;           // 16 KiB
+constexpr int BC_BYTES = BN * BK;          // 32 KiB unpacked codes
+constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words
+constexpr int STAGE_BYTES = A_BYTES + BC_BYTES + BP_BYTES;
+constexpr int HDR_BYTES = 1024;
+constexpr int GEMM_SMEM = 1024 /* alignment slack */ + HDR_BYTES + STAGES * STAGE_BYTES;
+constexpr int GEMM_THREADS = 320;
+constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators
+
+struct GemmHdr {
+    uint64_t full[STAGES];      // TMA bytes landed
+    uint64_t unpacked[STAGES];  // codes written by the 128 unpack threads
+    uint64_t empty[STAGES];     // MMAs reading the stage finished
+    uint64_t tfull[2];          // accumulator complete
+    uint64_t tempty[2];         // accumulator drained by the 128 epilogue threads
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(GemmHdr) <= HDR_BYTES, "gemm header too large");
+
+struct GemmParams {
+    const float* gamma;
+    const float* beta;
+    const int* rowsum;
+    void* y;
+    int M, N, K, mode;
+    int tiles_m, tiles_n, num_kb;
+};
+
+// -------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle
+// layout (8-row atoms of 1024 bytes stacked at a 1024-byte stride).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
+    d |= (uint64_t)1u << 16;                  // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024u >> 4) << 32;        // stride byte offset: next 8-row atom
+    d |= (uint64_t)1u << 46;                  // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                  // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor of kind::i8: s32 accumulator, s8 A and B, both
+// K-major, M = 128, N = 256.
+constexpr uint32_t IDESC = (2u << 4)                       // D format s32
+                           | (1u << 7)                     // A signed 8-bit
+                           | (1u << 10)                    // B signed 8-bit
+                           | ((uint32_t)(BN >> 3) << 17)   // N / 8
+                           | ((uint32_t)(BM >> 4) << 24);  // M / 16
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: lane i gets row (lane base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ bool aborted(GemmHdr& h) { return *(volatile int*)&h.abort_flag != 0; }
+
+__device__ __forceinline__ bool wait_or_abort(GemmHdr& h, uint64_t* bar, uint32_t parity) {
+    if (aborted(h)) return false;
+    if (!mbar_wait(bar, parity)) {
+        h.abort_flag = 1;
+        return false;
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------- kernels
+
+__global__ void __launch_bounds__(256) rowsum_kernel(const int8_t* __restrict__ x_q, int M, int K,
+                                                     int* __restrict__ rowsum) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= M) return;
+    const int4* p = reinterpret_cast<const int4*>(x_q + (long long)row * K);
+    int s = 0;
+    for (int g = lane; g < K / 16; g += 32) {
+        int4 v = __ldg(p + g);
+        s += bytesum_s8(v.x) + bytesum_s8(v.y) + bytesum_s8(v.z) + bytesum_s8(v.w);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) rowsum[row] = s;
+}
+
+__device__ __forceinline__ void store_chunk(const GemmParams& p, int m, int n0, const int (&v)[32], int rs, float f,
+                                            bool vec_ok) {
+    const long long o = (long long)m * p.N + n0;
+    const bool full = n0 + 32 <= p.N;
+    if (p.mode == Y_ACC) {
+        int* y = reinterpret_cast<int*>(p.y) + o;
+        if (full && vec_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<int4*>(y + j) = make_int4(v[j] - rs, v[j + 1] - rs, v[j + 2] - rs, v[j + 3] - rs);
+        } else {
+            for (int j = 0; j < 32 && n0 + j < p.N; ++j) y[j] = v[j] - rs;
+        }
+    } else if (p.mode == Y_F32) {
+        float* y = reinterpret_cast<float*>(p.y) + o;
+        float t[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) t[j] = __fmul_rn((float)(v[j] - rs), f);
+        if (full && vec_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(y + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
+        } else {
+            for (int j = 0; j < 32 && n0 + j < p.N; ++j) y[j] = t[j];
+        }
+    } else {
+        uint16_t* y = reinterpret_cast<uint16_t*>(p.y) + o;
+        uint32_t h[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t lo = f32_to_bf16_rn(__fmul_rn((float)(v[2 * j] - rs), f));
+            const uint32_t hi = f32_to_bf16_rn(__fmul_rn((float)(v[2 * j + 1] - rs), f));
+            h[j] = lo | (hi << 16);
+        }
+        if (full && vec_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) *reinterpret_cast<uint4*>(y + 2 * j) = make_uint4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+        } else {
+            for (int j = 0; j < 32 && n0 + j < p.N; ++j) y[j] = (uint16_t)(h[j >> 1] >> ((j & 1) * 16));
+        }
+    }
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                const GemmParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* base =
+        smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-byte aligned for the swizzle
+    GemmHdr& h = *reinterpret_cast<GemmHdr*>(base);
+    unsigned char* stages = base + HDR_BYTES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&h.full[s], 1);
+            mbar_init(&h.unpacked[s], 128);
+            mbar_init(&h.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&h.tfull[b], 1);
+            mbar_init(&h.tempty[b], 128);
+        }
+        h.abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) tmem_alloc(&h.tmem_base, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = h.tmem_base;
+    pdl_launch_dependents();
+    pdl_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!wait_or_abort(h, &h.empty[s], ph ^ 1)) goto done;
+                    unsigned char* st = stages + (size_t)s * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&h.full[s], A_BYTES + BP_BYTES);
+                    tma_load_2d(st, &tmap_a, kb * BK, mb * BM, &h.full[s]);
+                    tma_load_2d(st + A_BYTES + BC_BYTES, &tmap_b, kb * (BK / 16), nb * BN, &h.full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0, acc_it = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++acc_it) {
+                const int b = acc_it & 1;
+                const uint32_t aph = (acc_it >> 1) & 1;
+                if (!wait_or_abort(h, &h.tempty[b], aph ^ 1)) goto done;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!wait_or_abort(h, &h.full[s], ph)) goto done;
+                    if (!wait_or_abort(h, &h.unpacked[s], ph)) goto done;
+                    tc_fence_after();
+                    unsigned char* st = stages + (size_t)s * STAGE_BYTES;
+                    const uint64_t adesc = sw128_desc(smem_u32(st));
+                    const uint64_t bdesc = sw128_desc(smem_u32(st + A_BYTES));
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)  // K = 32 bytes per MMA: advance 32 B = 2 in addr >> 4
+                        mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, (kb | k) != 0);
+                    mma_commit(&h.empty[s]);
+                }
+                mma_commit(&h.tfull[b]);
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ unpack
+        const int ut = threadIdx.x - 64;  // 0..127
+        int it = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!wait_or_abort(h, &h.full[s], ph)) goto done;
+                unsigned char* st = stages + (size_t)s * STAGE_BYTES;
+                const uint32_t* bp = reinterpret_cast<const uint32_t*>(st + A_BYTES + BC_BYTES);
+                const uint32_t bc = smem_u32(st + A_BYTES);
+#pragma unroll 4
+                for (int i = 0; i < BN * (BK / 16) / 128; ++i) {
+                    const int w = ut + 128 * i;
+                    const int n = w >> 3, j = w & 7;
+                    const uint32_t word = bp[w];
+                    const uint32_t t0 = word & 0x03030303u;
+                    const uint32_t t1 = (word >> 2) & 0x03030303u;
+                    const uint32_t t2 = (word >> 4) & 0x03030303u;
+                    const uint32_t t3 = (word >> 6) & 0x03030303u;
+                    const uint32_t dst = bc + (uint32_t)(n * BK + ((j ^ (n & 7)) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(t0), "r"(t1), "r"(t2),
+                                 "r"(t3)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&h.unpacked[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lanes 32q .. 32q + 31
+        const bool vec_ok = p.mode == Y_BF16 ? (p.N % 8 == 0) : (p.N % 4 == 0);
+        const float beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
+        int acc_it = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++acc_it) {
+            const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+            const int b = acc_it & 1;
+            const uint32_t aph = (acc_it >> 1) & 1;
+            // tcgen05.ld is warp-collective: the whole warp proceeds or leaves together
+            if (!__all_sync(0xffffffffu, wait_or_abort(h, &h.tfull[b], aph))) goto done;
+            tc_fence_after();
+            const int m = mb * BM + q * 32 + lane;
+            int rs = 0;
+            float f = 0.0f;
+            if (m < p.M) {
+                rs = __ldg(p.rowsum + m);
+                if (p.mode != Y_ACC) f = __fdiv_rn(__fmul_rn(beta, __ldg(p.gamma + m)), 127.0f);
+            }
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                int v[32];
+                tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                const int n0 = nb * BN + c * 32;
+                if (m < p.M && n0 < p.N) store_chunk(p, m, n0, v, rs, f, vec_ok);
+            }
+            tc_fence_before();
+            mbar_arrive(&h.tempty[b]);
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------- host
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
 
 size_t gemm_ws_bytes(long long M, long long N, long long K) {
     (void)N;
@@ -10,9 +395,53 @@ size_t gemm_ws_bytes(long long M, long long N, long long K) {
     return (size_t)((M * 4 + 255) / 256 * 256);
 }
 
-cudaError_t launch_gemm(const int8_t*, const float*, int, int, const uint32_t*, const float*, int, void*, YMode, void*,
-                        const DevInfo&, cudaStream_t) {
-    return cudaErrorNotSupported;
+cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    if (dev.max_smem_optin < GEMM_SMEM) return cudaErrorNotSupported;
+    CUtensorMap ta, tb;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {BK, BM};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(x_q), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t box[2] = {BK / 16, BN};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(W_p), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    int* rowsum = reinterpret_cast<int*>(ws);
+    cudaError_t e = launch_pdl(rowsum_kernel, dim3((M + 7) / 8), dim3(256), 0, st, x_q, M, K, rowsum);
+    if (e != cudaSuccess) return e;
+
+    GemmParams p;
+    p.gamma = gamma;
+    p.beta = beta;
+    p.rowsum = rowsum;
+    p.y = y;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.mode = mode;
+    p.tiles_m = (M + BM - 1) / BM;
+    p.tiles_n = (N + BN - 1) / BN;
+    p.num_kb = (K + BK - 1) / BK;
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = std::max(1, std::min(tiles, dev.num_sms));
+    e = ensure_smem_optin(reinterpret_cast<const void*>(gemm_kernel), GEMM_SMEM);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(gemm_kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
 }
 
 }  // namespace bl

@@ -10,19 +10,24 @@
 //   * one CTA per SM owns a contiguous slab of output rows, i.e. one
 //     contiguous byte range of W_p; a producer warp streams it into a
 //     shared-memory ring with 1-D bulk copies (cp.async.bulk, evict-first L2
-//     hint), issuing every chunk that fits at kernel start so the whole
-//     GPU's share of HBM requests is in flight from the first microsecond;
-//     per-chunk mbarriers let compute start as soon as the first chunk lands;
-//   * consumer "teams" of LPR lanes each take one row at a time; a lane
-//     covers UPL 16-byte groups (64 trits each) of the row;
-//   * the weight stream is requested before griddepcontrol.wait, so under
-//     programmatic dependent launch it overlaps the activation quantiser;
+//     hint), issuing every chunk that fits as soon as the CTA starts, so the
+//     GPU's whole share of HBM requests is in flight from the first
+//     microsecond and the stream overlaps the previous kernel's tail under
+//     programmatic dependent launch;
 //   * the contraction uses codes c = w + 1: sum_k c_k x_k - sum_k x_k =
 //     sum_k w_k x_k.  A packed word holds the codes of k = 16j+4s+b at bits
 //     8b+2s; masking with 0x03030303 << 2s (no shift) leaves 4^s * c in the
 //     four bytes, so one LOP3 and one dp4a.u32.s32 per 4 trits accumulate
 //     4^s * sum(c x) exactly in int32 (|partial| <= 4064 K < 2^31);
-//   * team sums by warp shuffles; one lane writes y = (acc - rowsum) * f.
+//   * M <= 4 ("small" kernel): the activations live in shared memory (with an
+//     XOR swizzle of the 16-byte chunks that makes the per-lane reads
+//     bank-conflict free); a team of LPR lanes works on R rows at once so
+//     every lane keeps 4 * R * MT independent dp4a chains in flight, and the
+//     R * MT team sums are finished by one batched transpose-reduction of
+//     warp shuffles.  The quantiser can run in the prologue (fused forward),
+//     so a decode layer is a single kernel;
+//   * 4 < M <= 64 ("mt" kernel): one warp per row, activations read through
+//     L1 from global memory, MT tokens per pass.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -30,24 +35,33 @@ namespace bl {
 
 namespace {
 
-constexpr int GEMV_CWARPS = 8;                      // consumer warps
-constexpr int GEMV_THREADS = (GEMV_CWARPS + 1) * 32;  // + 1 producer warp
 constexpr int GEMV_MAX_STAGES = 32;
-constexpr int GEMV_HDR = 2048;                      // barriers + per-token tables
+constexpr int GEMV_HDR = 2048;  // barriers + per-token tables + reduction scratch
 constexpr int GEMV_MAX_M = 64;
-constexpr int GEMV_RING_BYTES = 200 * 1024;
+constexpr int GEMV_MAX_CWARPS = 11;                           // small kernel: <= 384 threads and
+constexpr int GEMV_MAX_THREADS = (GEMV_MAX_CWARPS + 1) * 32;  // <= 85 registers: two CTAs fit an SM
+constexpr int GEMV_CO_RESIDENT = 2;                           // a kernel and its PDL successor
+constexpr int GEMV_MT_CWARPS = 8;  // consumer warps of the mt kernel
 constexpr int GEMV_CHUNK_TARGET = 8192;
+constexpr int GEMV_XQ_SMEM_MAX = 64 * 1024;
+constexpr int GEMV_SMALL_MAX_M = 4;
+
+enum XMode : int { X_QUANTISED = 0, X_F32 = 1, X_BF16 = 2 };
 
 struct GemvParams {
+    const void* x;  // fp32/bf16 activations when the quantiser is fused
     const int8_t* x_q;
     const float* gamma;
     const uint32_t* W_p;
     const float* beta;
     void* y;
-    int M, K, N, mode;
-    int rpc;           // packed rows per chunk
+    int M, K, N, mode, x_mode;
+    int rpc;           // packed rows per chunk (a power of two)
+    int rpc_shift;     // log2(rpc)
+    int reuse;         // 0: every chunk has its own ring slot (slot = chunk, parity 0)
     int stages;        // ring depth
-    int stage_stride;  // bytes per ring slot (multiple of 128)
+    int stage_stride;  // bytes per ring slot (rpc rows, a multiple of 16)
+    int xq_bytes;      // shared-memory bytes reserved for x_q (small kernel)
 };
 
 struct Shared {
@@ -56,6 +70,8 @@ struct Shared {
     int abort_flag;
     int rowsum[GEMV_MAX_M];
     float fscale[GEMV_MAX_M];
+    unsigned red_u[GEMV_MAX_CWARPS][GEMV_SMALL_MAX_M];
+    int red_i[GEMV_MAX_CWARPS][GEMV_SMALL_MAX_M];
 };
 static_assert(sizeof(Shared) <= GEMV_HDR, "header too large");
 
@@ -86,14 +102,22 @@ __device__ __forceinline__ int combine4(int a0, int a1, int a2, int a3) {
     return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);  // each a_s is a multiple of 4^s
 }
 
-// Producer: stream this CTA's rows [r0, r0 + nrows) of W_p into the ring.
-__device__ __forceinline__ void produce(const GemvParams& p, Shared& sh, unsigned char* ring, int r0, int nrows) {
+// Ring slot and phase parity of chunk c.  Without reuse the whole slab fits
+// (slot = c, first phase); otherwise slots cycle through the ring.
+__device__ __forceinline__ int chunk_slot(const GemvParams& p, int c) { return p.reuse ? c % p.stages : c; }
+__device__ __forceinline__ uint32_t chunk_parity(const GemvParams& p, int c) {
+    return p.reuse ? (uint32_t)((c / p.stages) & 1) : 0u;
+}
+
+// Producer: stream chunks [c0, c1) of this CTA's rows [r0, r0 + nrows) of W_p
+// into the ring (a chunk is rpc rows; chunk c goes to slot c % stages).
+__device__ __forceinline__ void produce(const GemvParams& p, Shared& sh, unsigned char* ring, int r0, int nrows,
+                                        int c0, int c1) {
     const int RB = p.K / 4;
-    const int nchunks = (nrows + p.rpc - 1) / p.rpc;
     const uint64_t pol = policy_evict_first();
     const unsigned char* src = reinterpret_cast<const unsigned char*>(p.W_p) + (long long)r0 * RB;
-    for (int c = 0; c < nchunks; ++c) {
-        const int st = c % p.stages;
+    for (int c = c0; c < c1; ++c) {
+        const int st = chunk_slot(p, c);
         if (c >= p.stages) {
             if (!mbar_wait(&sh.empty[st], ((c / p.stages) - 1) & 1)) {
                 sh.abort_flag = 1;
@@ -109,17 +133,23 @@ __device__ __forceinline__ void produce(const GemvParams& p, Shared& sh, unsigne
 
 // Wait for the chunk holding slab row i; false once the CTA has aborted.
 __device__ __forceinline__ bool wait_row(const GemvParams& p, Shared& sh, int i) {
-    const int c = i / p.rpc;
+    const int c = i >> p.rpc_shift;
     if (*(volatile int*)&sh.abort_flag) return false;
-    if (!mbar_wait(&sh.full[c % p.stages], (c / p.stages) & 1)) {
+    if (!mbar_wait(&sh.full[chunk_slot(p, c)], chunk_parity(p, c))) {
         sh.abort_flag = 1;
         return false;
     }
     return true;
 }
 
-__device__ __forceinline__ void release_row(const GemvParams& p, Shared& sh, int i, int nchunks) {
-    if (nchunks > p.stages) mbar_arrive(&sh.empty[(i / p.rpc) % p.stages]);
+__device__ __forceinline__ void release_row(const GemvParams& p, Shared& sh, int i) {
+    if (p.reuse) mbar_arrive(&sh.empty[chunk_slot(p, i >> p.rpc_shift)]);
+}
+
+__device__ __forceinline__ const uint4* row_ptr(const GemvParams& p, const unsigned char* ring, int i) {
+    const int c = i >> p.rpc_shift;
+    return reinterpret_cast<const uint4*>(ring + (size_t)chunk_slot(p, c) * p.stage_stride +
+                                          (size_t)(i & (p.rpc - 1)) * (p.K / 4));
 }
 
 __device__ __forceinline__ void cta_rows(const GemvParams& p, int& r0, int& nrows) {
@@ -141,95 +171,285 @@ __device__ __forceinline__ void init_barriers(const GemvParams& p, Shared& sh) {
     __syncthreads();
 }
 
-// ---------------------------------------------------------------- M == 1
+__device__ __forceinline__ void consumer_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
 
-template <int LPR, int UPL>
-__global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_m1_kernel(const GemvParams p) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    Shared& sh = *reinterpret_cast<Shared*>(smem);
-    unsigned char* ring = smem + GEMV_HDR;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int r0, nrows;
-    cta_rows(p, r0, nrows);
-    init_barriers(p, sh);
-    pdl_launch_dependents();
-    if (warp == GEMV_CWARPS) {
-        if (lane == 0) produce(p, sh, ring, r0, nrows);
-        return;
-    }
-    pdl_wait();
+// 16-byte chunk c of a token's x_q row is stored at slot c ^ ((c >> 3) & 3):
+// lane l of a team reads chunks 4l + q, which this maps to distinct bank groups.
+__device__ __forceinline__ int xq_slot(int c) { return c ^ ((c >> 3) & 3); }
 
-    constexpr int T = GEMV_CWARPS * 32 / LPR;  // teams per CTA
-    const int team = threadIdx.x / LPR;
-    const int tl = lane % LPR;
-    const int K4 = p.K / 64;                   // 16-byte groups per row
-    const int RB = p.K / 4;
-    const int nchunks = (nrows + p.rpc - 1) / p.rpc;
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+    return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
+           ((uint32_t)(d & 0xFF) << 24);
+}
 
-    int xr[UPL][16];
-    int rs = 0;
+// same rounding as the standalone quantiser: rint(x * s), clamp to [-127, 127]
+__device__ __forceinline__ int q8(float v, float s) {
+    int r = __float2int_rn(__fmul_rn(v, s));
+    return min(max(r, -127), 127);
+}
+
+template <int MODE>  // X_F32 or X_BF16
+__device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
+    if (MODE == X_BF16) {
+        const uint4* pp = reinterpret_cast<const uint4*>(row) + 2 * g;
+        uint4 a = __ldg(pp), b = __ldg(pp + 1);
+        uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int u = 0; u < UPL; ++u) {
-        const int idx = tl + u * LPR;
-        if (idx < K4) {
-            const int4* px = reinterpret_cast<const int4*>(p.x_q) + 4 * idx;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                int4 v = __ldg(px + q);
-                xr[u][4 * q + 0] = v.x;
-                xr[u][4 * q + 1] = v.y;
-                xr[u][4 * q + 2] = v.z;
-                xr[u][4 * q + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) xr[u][q] = 0;
+        for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
+    } else {
+        const float4* pp = reinterpret_cast<const float4*>(row) + 4 * g;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) rs += bytesum_s8(xr[u][q]);
-    }
-#pragma unroll
-    for (int off = LPR / 2; off; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
-    // beta and gamma are absent (NULL) when only the accumulators are wanted
-    const float f = p.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(__ldg(p.beta), __ldg(p.gamma)), 127.0f);
-
-    // Warp-uniform trip count: every lane runs every shuffle.
-    const int iters = (nrows + T - 1) / T;
-    for (int it = 0; it < iters; ++it) {
-        const int i = it * T + team;
-        const bool valid = i < nrows;
-        bool ok = valid && wait_row(p, sh, i);
-        int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-        if (ok) {
-            const int c = i / p.rpc;
-            const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)(c % p.stages) * p.stage_stride +
-                                                                (size_t)(i - c * p.rpc) * RB);
-#pragma unroll
-            for (int u = 0; u < UPL; ++u) {
-                const int idx = tl + u * LPR;
-                if (idx < K4) {
-                    const uint4 w = wrow[idx];
-                    word_dot(w.x, xr[u][0], xr[u][1], xr[u][2], xr[u][3], a0, a1, a2, a3);
-                    word_dot(w.y, xr[u][4], xr[u][5], xr[u][6], xr[u][7], a0, a1, a2, a3);
-                    word_dot(w.z, xr[u][8], xr[u][9], xr[u][10], xr[u][11], a0, a1, a2, a3);
-                    word_dot(w.w, xr[u][12], xr[u][13], xr[u][14], xr[u][15], a0, a1, a2, a3);
-                }
-            }
-        }
-        int acc = combine4(a0, a1, a2, a3);
-#pragma unroll
-        for (int off = LPR / 2; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (ok && tl == 0) {
-            release_row(p, sh, i, nchunks);
-            store_y(p, 0, r0 + i, acc - rs, f);
+        for (int i = 0; i < 4; ++i) {
+            float4 f = __ldg(pp + i);
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
         }
     }
 }
 
-// ------------------------------------------------------------ 1 < M <= 64
+// Fill the shared x_q rows (tokens 0..MT-1; tokens >= M are zero), rowsum[]
+// and fscale[].  Runs on the consumer threads only.
+template <int MT, int XM>
+__device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& sh, int4* xsm, int ctid, int cthreads,
+                                                  int cwarps) {
+    const int G = p.K / 16;  // 16-byte chunks per token
+    const int lane = ctid & 31, warp = ctid >> 5;
+    float s[MT];
+    float gam[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) s[m] = gam[m] = 0.0f;
+    if (XM != X_QUANTISED) {
+        // pass 1: per-token absmax over the row (exact, order-free)
+        unsigned amax[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) amax[m] = 0u;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (m < p.M) {
+                const char* xr = reinterpret_cast<const char*>(p.x) + (long long)m * p.K * (XM == X_BF16 ? 2 : 4);
+                for (int g = ctid; g < G; g += cthreads) {
+                    float v[16];
+                    load16<XM>(xr, g, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) amax[m] = max(amax[m], __float_as_uint(fabsf(v[i])));
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            unsigned a = __reduce_max_sync(0xffffffffu, amax[m]);
+            if (lane == 0) sh.red_u[warp][m] = a;
+        }
+        consumer_sync(cthreads);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            unsigned a = 0u;
+            for (int w = 0; w < cwarps; ++w) a = max(a, sh.red_u[w][m]);
+            gam[m] = fmaxf(__uint_as_float(a), 1e-5f);
+            s[m] = __fdiv_rn(127.0f, gam[m]);
+        }
+    }
+    // pass 2: write x_q chunks into their swizzled slots, accumulate row sums
+    int rs[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) rs[m] = 0;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        int4* dst = xsm + (size_t)m * G;
+        for (int g = ctid; g < G; g += cthreads) {
+            int4 q = make_int4(0, 0, 0, 0);
+            if (m < p.M) {
+                if (XM == X_QUANTISED) {
+                    q = __ldg(reinterpret_cast<const int4*>(p.x_q + (long long)m * p.K) + g);
+                } else {
+                    const char* xr =
+                        reinterpret_cast<const char*>(p.x) + (long long)m * p.K * (XM == X_BF16 ? 2 : 4);
+                    float v[16];
+                    load16<XM>(xr, g, v);
+                    q.x = (int)pack4(q8(v[0], s[m]), q8(v[1], s[m]), q8(v[2], s[m]), q8(v[3], s[m]));
+                    q.y = (int)pack4(q8(v[4], s[m]), q8(v[5], s[m]), q8(v[6], s[m]), q8(v[7], s[m]));
+                    q.z = (int)pack4(q8(v[8], s[m]), q8(v[9], s[m]), q8(v[10], s[m]), q8(v[11], s[m]));
+                    q.w = (int)pack4(q8(v[12], s[m]), q8(v[13], s[m]), q8(v[14], s[m]), q8(v[15], s[m]));
+                }
+                rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
+            }
+            dst[xq_slot(g)] = q;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        int v = rs[m];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) sh.red_i[warp][m] = v;
+    }
+    consumer_sync(cthreads);
+    if (ctid < MT) {
+        const int m = ctid;
+        int t = 0;
+        for (int w = 0; w < cwarps; ++w) t += sh.red_i[w][m];
+        sh.rowsum[m] = t;
+        float f = 0.0f;
+        if (p.mode != Y_ACC && m < p.M) {
+            const float g = XM == X_QUANTISED ? __ldg(p.gamma + m) : gam[m];
+            f = __fdiv_rn(__fmul_rn(__ldg(p.beta), g), 127.0f);
+        }
+        sh.fscale[m] = f;
+    }
+    consumer_sync(cthreads);
+}
+
+// Batched reduction of V = 1, 2 or 4 values over the LPR lanes of a team.
+// Lane tl ends up with the full sum of value `which`.
+template <int LPR, int V>
+__device__ __forceinline__ int team_reduce(const int (&v)[V], int tl, int& which) {
+    if constexpr (V == 1) {
+        int k = v[0];
+#pragma unroll
+        for (int o = LPR / 2; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+        which = 0;
+        return k;
+    } else if constexpr (V == 2) {
+        constexpr int h1 = LPR / 2;
+        const bool hi = (tl & h1) != 0;
+        int k = hi ? v[1] : v[0];
+        k += __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], h1);
+#pragma unroll
+        for (int o = LPR / 4; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+        which = hi ? 1 : 0;
+        return k;
+    } else {
+        constexpr int h1 = LPR / 2, h2 = LPR / 4;
+        const bool hi = (tl & h1) != 0;
+        int k0 = hi ? v[2] : v[0];
+        int k1 = hi ? v[3] : v[1];
+        k0 += __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[2], h1);
+        k1 += __shfl_xor_sync(0xffffffffu, hi ? v[1] : v[3], h1);
+        const bool hi2 = (tl & h2) != 0;
+        int k = hi2 ? k1 : k0;
+        k += __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, h2);
+#pragma unroll
+        for (int o = LPR / 8; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+        which = (hi ? 2 : 0) + (hi2 ? 1 : 0);
+        return k;
+    }
+}
+
+// ---------------------------------------------------------------- M <= 4
+
+template <int LPR, int MT, int R, int XM>
+__global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small_kernel(const GemvParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    Shared& sh = *reinterpret_cast<Shared*>(smem);
+    int4* xsm = reinterpret_cast<int4*>(smem + GEMV_HDR);
+    unsigned char* ring = smem + GEMV_HDR + p.xq_bytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cwarps = blockDim.x / 32 - 1;  // warp 0 produces, warps 1.. consume
+    const int cthreads = cwarps * 32;
+    int r0, nrows;
+    cta_rows(p, r0, nrows);
+    const int nchunks = (nrows + p.rpc - 1) / p.rpc;
+    // Thread 0 sets up the barriers and puts the slab's bulk copies in flight
+    // before anyone else runs, so the HBM stream starts as early as possible.
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], p.rpc);
+        }
+        sh.abort_flag = 0;
+        fence_mbar_init();
+        produce(p, sh, ring, r0, nrows, 0, min(nchunks, p.stages));
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    if (warp == 0) {
+        if (lane == 0 && nchunks > p.stages) produce(p, sh, ring, r0, nrows, p.stages, nchunks);
+        return;
+    }
+    pdl_wait();
+    const int ctid = threadIdx.x - 32;
+    stage_activations<MT, XM>(p, sh, xsm, ctid, cthreads, cwarps);
+
+    constexpr int V = R * MT;
+    const int T = cthreads / LPR;  // teams
+    const int team = ctid / LPR;
+    const int tl = ctid % LPR;
+    const int K4 = p.K / 64;  // 16-byte groups of packed weights per row
+    const int G = p.K / 16;   // 16-byte chunks of x_q per token
+    const int iters = (nrows + T * R - 1) / (T * R);  // warp-uniform trip count
+
+    for (int it = 0; it < iters; ++it) {
+        const int b = (it * T + team) * R;
+        const int nvalid = max(0, min(R, nrows - b));
+        bool ok = nvalid > 0;
+        for (int r = 0; r < nvalid; ++r) ok = ok && wait_row(p, sh, b + r);
+        // row offsets once per team-iteration (missing rows alias row b)
+        uint32_t ro[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            ro[r] = (uint32_t)(reinterpret_cast<const unsigned char*>(row_ptr(p, ring, b + (r < nvalid ? r : 0))) - ring);
+        int a[R][MT][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) a[r][m][0] = a[r][m][1] = a[r][m][2] = a[r][m][3] = 0;
+        if (ok && tl < K4) {
+            // software pipeline: the next group's weights load while this one is used
+            uint4 wn[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * tl);
+            for (int idx = tl; idx < K4; idx += LPR) {
+                uint4 w[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r) w[r] = wn[r];
+                const int nxt = idx + LPR < K4 ? idx + LPR : idx;
+#pragma unroll
+                for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * nxt);
+                const int key = (idx >> 1) & 3;  // swizzle of chunks 4 idx .. 4 idx + 3
+                const int4* xb = xsm + 4 * idx;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const int4 xv = xb[m * G + (q ^ key)];
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            const uint32_t wq = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+                            word_dot(wq, xv.x, xv.y, xv.z, xv.w, a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
+                        }
+                    }
+                }
+            }
+        }
+        int vals[V];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) vals[r * MT + m] = combine4(a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
+        int which;
+        const int tot = team_reduce<LPR, V>(vals, tl, which);
+        // lane tl = which * (LPR / V) is the first lane that owns value `which`
+        if (ok && tl == which * (LPR / V)) {
+            const int r = which / MT, m = which % MT;
+            if (r < nvalid) {
+                if (m == 0) release_row(p, sh, b + r);
+                if (m < p.M) store_y(p, m, r0 + b + r, tot - sh.rowsum[m], sh.fscale[m]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ 4 < M <= 64
 
 template <int MT>
-__global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_mt_kernel(const GemvParams p) {
+__global__ void __launch_bounds__((GEMV_MT_CWARPS + 1) * 32, 1) gemv_mt_kernel(const GemvParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     Shared& sh = *reinterpret_cast<Shared*>(smem);
     unsigned char* ring = smem + GEMV_HDR;
@@ -238,17 +458,16 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_mt_kernel(const GemvPara
     cta_rows(p, r0, nrows);
     init_barriers(p, sh);
     pdl_launch_dependents();
-    if (warp == GEMV_CWARPS) {
-        if (lane == 0) produce(p, sh, ring, r0, nrows);
+    if (warp == GEMV_MT_CWARPS) {
+        if (lane == 0) produce(p, sh, ring, r0, nrows, 0, (nrows + p.rpc - 1) / p.rpc);
         return;
     }
     pdl_wait();
 
     const int K4 = p.K / 64;
-    const int RB = p.K / 4;
     const int nchunks = (nrows + p.rpc - 1) / p.rpc;
     // per-token row sums of x_q and rescale factors
-    for (int m = warp; m < p.M; m += GEMV_CWARPS) {
+    for (int m = warp; m < p.M; m += GEMV_MT_CWARPS) {
         const int4* px = reinterpret_cast<const int4*>(p.x_q + (long long)m * p.K);
         int s = 0;
         for (int g = lane; g < p.K / 16; g += 32) {
@@ -259,17 +478,16 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_mt_kernel(const GemvPara
         for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) {
             sh.rowsum[m] = s;
+            // beta and gamma are absent (NULL) when only the accumulators are wanted
             sh.fscale[m] = p.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(__ldg(p.beta), __ldg(p.gamma + m)), 127.0f);
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(GEMV_CWARPS * 32) : "memory");
+    consumer_sync(GEMV_MT_CWARPS * 32);
 
-    for (int i = warp; i < nrows; i += GEMV_CWARPS) {
+    for (int i = warp; i < nrows; i += GEMV_MT_CWARPS) {
         // every lane waits the same barrier; the decision is made warp-uniform
         if (!__all_sync(0xffffffffu, wait_row(p, sh, i))) break;
-        const int c = i / p.rpc;
-        const uint4* wrow = reinterpret_cast<const uint4*>(ring + (size_t)(c % p.stages) * p.stage_stride +
-                                                            (size_t)(i - c * p.rpc) * RB);
+        const uint4* wrow = row_ptr(p, ring, i);
         for (int m0 = 0; m0 < p.M; m0 += MT) {
             int a[MT][4];
 #pragma unroll
@@ -298,41 +516,113 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_mt_kernel(const GemvPara
             }
         }
         __syncwarp();
-        if (lane == 0) release_row(p, sh, i, nchunks);
+        if (lane == 0) release_row(p, sh, i);
     }
 }
 
 // ------------------------------------------------------------------- host
 
-template <typename K>
-cudaError_t launch_with_smem(K kernel, int grid, size_t smem, cudaStream_t st, const GemvParams& p) {
+template <typename KernelT>
+cudaError_t launch_with_smem(KernelT kernel, int grid, int threads, size_t smem, cudaStream_t st,
+                             const GemvParams& p) {
     cudaError_t e = ensure_smem_optin(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kernel, dim3(grid), dim3(GEMV_THREADS), smem, st, p);
+    return launch_pdl(kernel, dim3(grid), dim3(threads), smem, st, p);
 }
 
-using M1Kernel = void (*)(const GemvParams);
+using GemvKernel = void (*)(const GemvParams);
 
-template <int LPR>
-M1Kernel m1_kernel_for(int upl) {
-    switch (upl) {
-        case 1: return gemv_m1_kernel<LPR, 1>;
-        case 2: return gemv_m1_kernel<LPR, 2>;
-        case 3: return gemv_m1_kernel<LPR, 3>;
-        case 4: return gemv_m1_kernel<LPR, 4>;
-        case 5: return gemv_m1_kernel<LPR, 5>;
-        case 6: return gemv_m1_kernel<LPR, 6>;
-        case 7: return gemv_m1_kernel<LPR, 7>;
-        case 8: return gemv_m1_kernel<LPR, 8>;
+template <int LPR, int XM>
+GemvKernel small_kernel_for(int mt, int r) {
+    if (mt == 1 && r == 1) return gemv_small_kernel<LPR, 1, 1, XM>;
+    if (mt == 1 && r == 2) return gemv_small_kernel<LPR, 1, 2, XM>;
+    if (mt == 1 && r == 4) return gemv_small_kernel<LPR, 1, 4, XM>;
+    if (mt == 2 && r == 1) return gemv_small_kernel<LPR, 2, 1, XM>;
+    if (mt == 2 && r == 2) return gemv_small_kernel<LPR, 2, 2, XM>;
+    return gemv_small_kernel<LPR, 4, 1, XM>;
+}
+
+template <int XM>
+GemvKernel small_kernel_for(int lpr, int mt, int r) {
+    if (lpr == 32) return small_kernel_for<32, XM>(mt, r);
+    if (lpr == 16) return small_kernel_for<16, XM>(mt, r);
+    return small_kernel_for<8, XM>(mt, r);
+}
+
+// Ring geometry for a CTA slab of `rows_per_cta` rows and `ring_bytes` of
+// space: chunks of a power-of-two number of rows (about 8 KiB), one slot per
+// chunk when the slab fits, otherwise a ring of as many slots as fit.
+void ring_geometry(GemvParams& p, int rows_per_cta, int ring_bytes) {
+    const int RB = p.K / 4;
+    const int cap = std::max(1, std::min(rows_per_cta, GEMV_CHUNK_TARGET / RB));
+    p.rpc_shift = 0;
+    while ((2 << p.rpc_shift) <= cap) ++p.rpc_shift;
+    p.rpc = 1 << p.rpc_shift;
+    p.stage_stride = p.rpc * RB;  // multiple of 16 (K % 64 == 0); >= one row (<= 64 KiB)
+    const int nchunks = (rows_per_cta + p.rpc - 1) / p.rpc;
+    const int fit = std::max(1, std::min(ring_bytes / p.stage_stride, GEMV_MAX_STAGES));
+    p.reuse = nchunks > fit;
+    p.stages = p.reuse ? fit : nchunks;
+}
+
+int small_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+
+cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st) {
+    const int M = p.M, K = p.K, N = p.N;
+    const int grid = std::max(1, std::min(N, dev.num_sms));
+    const int rows_per_cta = (N + grid - 1) / grid;
+    const int max_dyn = dev.max_smem_optin;
+    const int K4 = K / 64;
+
+    const int mt = small_mt(M);
+    if (M <= GEMV_SMALL_MAX_M && mt * K <= GEMV_XQ_SMEM_MAX) {
+        // Choose lanes-per-row (team size) and rows-per-team-iteration so that
+        // every row of the CTA fits in one team-iteration when possible, with
+        // the fewest idle lanes; then size the CTA to the teams it needs.
+        int lpr = 32, r = 1;
+        double best = -1.0;
+        for (int cand_r : {4, 2, 1}) {
+            if (cand_r * mt > 4) continue;
+            for (int l : {32, 16, 8}) {
+                const int upl = (K4 + l - 1) / l;
+                const double lane_eff = (double)K4 / (l * upl);
+                const int teams_cap = GEMV_MAX_CWARPS * 32 / l;
+                const int iters = (rows_per_cta + teams_cap * cand_r - 1) / (teams_cap * cand_r);
+                const double score = lane_eff / iters + 0.01 * cand_r;  // prefer one pass, then ILP
+                if (score > best + 1e-9) {
+                    best = score;
+                    lpr = l;
+                    r = cand_r;
+                }
+            }
+        }
+        const int teams = (rows_per_cta + r - 1) / r;
+        const int cwarps = std::max(1, std::min(GEMV_MAX_CWARPS, (teams * lpr + 31) / 32));
+        p.xq_bytes = (mt * K + 127) / 128 * 128;
+        // leave room for the next launch's CTA on the same SM
+        const int budget = (max_dyn - 1024) / GEMV_CO_RESIDENT;
+        const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * (K / 4));
+        ring_geometry(p, rows_per_cta, ring_bytes);
+        const size_t smem = GEMV_HDR + p.xq_bytes + (size_t)p.stages * p.stage_stride;
+        GemvKernel k = p.x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED>(lpr, mt, r)
+                       : p.x_mode == X_F32     ? small_kernel_for<X_F32>(lpr, mt, r)
+                                               : small_kernel_for<X_BF16>(lpr, mt, r);
+        return launch_with_smem(k, grid, (cwarps + 1) * 32, smem, st, p);
     }
-    return nullptr;
+    if (p.x_mode != X_QUANTISED) return cudaErrorInvalidValue;  // callers quantise first
+    p.xq_bytes = 0;
+    ring_geometry(p, rows_per_cta, max_dyn - GEMV_HDR);
+    const size_t smem = GEMV_HDR + (size_t)p.stages * p.stage_stride;
+    const int threads = (GEMV_MT_CWARPS + 1) * 32;
+    if (M <= 1) return launch_with_smem(gemv_mt_kernel<1>, grid, threads, smem, st, p);
+    if (M <= 2) return launch_with_smem(gemv_mt_kernel<2>, grid, threads, smem, st, p);
+    if (M <= 4) return launch_with_smem(gemv_mt_kernel<4>, grid, threads, smem, st, p);
+    return launch_with_smem(gemv_mt_kernel<8>, grid, threads, smem, st, p);
 }
 
-}  // namespace
-
-cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
-                        int N, void* y, YMode mode, const DevInfo& dev, cudaStream_t st) {
-    GemvParams p;
+GemvParams make_params(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
+                       int N, void* y, YMode mode) {
+    GemvParams p = {};
     p.x_q = x_q;
     p.gamma = gamma;
     p.W_p = W_p;
@@ -342,40 +632,28 @@ cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, con
     p.K = K;
     p.N = N;
     p.mode = mode;
-    const int RB = K / 4;
-    const int grid = std::max(1, std::min(N, dev.num_sms));
-    const int rows_per_cta = (N + grid - 1) / grid;
-    p.rpc = std::max(1, std::min(rows_per_cta, GEMV_CHUNK_TARGET / RB));
-    p.stage_stride = ((p.rpc * RB) + 127) / 128 * 128;
-    const int nchunks = (rows_per_cta + p.rpc - 1) / p.rpc;
-    const int max_ring = std::min(GEMV_RING_BYTES, dev.max_smem_optin - GEMV_HDR);
-    p.stages = std::max(1, std::min({max_ring / p.stage_stride, GEMV_MAX_STAGES, nchunks}));
-    const size_t smem = GEMV_HDR + (size_t)p.stages * p.stage_stride;
+    p.x_mode = X_QUANTISED;
+    return p;
+}
 
-    const int K4 = K / 64;
-    if (M == 1 && K4 <= 8 * 32) {
-        // pick lanes-per-row and groups-per-lane to cover K4 with least idle lanes
-        int best_lpr = 32, best_upl = (K4 + 31) / 32;
-        double best_eff = -1.0;
-        for (int lpr : {32, 16, 8}) {
-            const int upl = (K4 + lpr - 1) / lpr;
-            if (upl > 8) continue;
-            const double eff = (double)K4 / (lpr * upl);
-            if (eff > best_eff + 1e-9) {
-                best_eff = eff;
-                best_lpr = lpr;
-                best_upl = upl;
-            }
-        }
-        M1Kernel k = best_lpr == 32 ? m1_kernel_for<32>(best_upl)
-                     : best_lpr == 16 ? m1_kernel_for<16>(best_upl)
-                                      : m1_kernel_for<8>(best_upl);
-        return launch_with_smem(k, grid, smem, st, p);
-    }
-    if (M <= 1) return launch_with_smem(gemv_mt_kernel<1>, grid, smem, st, p);
-    if (M <= 2) return launch_with_smem(gemv_mt_kernel<2>, grid, smem, st, p);
-    if (M <= 4) return launch_with_smem(gemv_mt_kernel<4>, grid, smem, st, p);
-    return launch_with_smem(gemv_mt_kernel<8>, grid, smem, st, p);
+}  // namespace
+
+cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
+                        int N, void* y, YMode mode, const DevInfo& dev, cudaStream_t st) {
+    GemvParams p = make_params(x_q, gamma, M, K, W_p, beta, N, y, mode);
+    return launch_gemv_impl(p, dev, st);
+}
+
+bool gemv_fused_quant_ok(long long M, long long K) {
+    return M <= GEMV_SMALL_MAX_M && small_mt((int)M) * K <= GEMV_XQ_SMEM_MAX;
+}
+
+cudaError_t launch_gemv_fused(const void* x, bool bf16, int M, int K, const uint32_t* W_p, const float* beta, int N,
+                              void* y, YMode mode, const DevInfo& dev, cudaStream_t st) {
+    GemvParams p = make_params(nullptr, nullptr, M, K, W_p, beta, N, y, mode);
+    p.x = x;
+    p.x_mode = bf16 ? X_BF16 : X_F32;
+    return launch_gemv_impl(p, dev, st);
 }
 
 }  // namespace bl

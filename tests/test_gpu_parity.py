@@ -231,3 +231,99 @@ def test_workload_decode_m1_bf16(dev, shape):
 @pytest.mark.parametrize("shape", workloads.W3.shapes, ids=lambda s: s.name)
 def test_workload_small_batch(dev, shape):
     run_case(dev, shape.M, shape.K, shape.N, shape.w_seed)
+
+
+# --------------------------------------------------------------------------
+# fused quantise + forward: bit-identical to quant_act followed by forward
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 17])
+@pytest.mark.parametrize("K,N,x_dtype", [(1024, 300, "bf16"), (4096, 1111, "f32"), (16384, 150, "bf16"),
+                                         (6912, 149, "f32")])
+def test_forward_fp_matches_two_calls_and_oracle(dev, M, K, N, x_dtype):
+    W = workloads.latent_weights(M + K + N, N, K)
+    x = workloads.activations(M * 3 + K, M, K, outliers=True)
+    if x_dtype == "bf16":
+        bits = workloads.bf16_bits(x)
+        xt = T(bits.view(np.int16), dev).view(torch.bfloat16)
+        x = workloads.bf16_to_f32(bits)
+    else:
+        xt = T(x, dev)
+    W_t, beta, W_p = gpu_prep(W, dev)
+    y_fused = bl.forward_fp(xt, W_p, beta)
+    x_q, gamma = bl.quant_act(xt)
+    y_two = bl.forward(x_q, gamma, W_p, beta)
+    np.testing.assert_array_equal(y_fused.cpu().numpy(), y_two.cpu().numpy())
+    oW_t, obeta = oracle.quantize_weights(W)
+    ref = oracle.forward(x, oW_t, obeta)
+    assert_f32_close(y_fused.cpu().numpy(), ref["y64"])
+    yb = bl.forward_fp(xt, W_p, beta, out_dtype=torch.bfloat16)
+    assert_bf16_ok(yb.cpu().view(torch.int16).numpy().view(np.uint16), ref["y64"])
+
+
+def test_forward_fp_zero_and_tiny_tokens(dev):
+    K, N = 1024, 64
+    W = workloads.latent_weights(3, N, K)
+    x = np.zeros((3, K), np.float32)
+    x[1, 7] = 2e-6                                  # gamma floor
+    x[2] = workloads.activations(4, 1, K)[0]
+    W_t, beta, W_p = gpu_prep(W, dev)
+    y = bl.forward_fp(T(x, dev), W_p, beta).cpu().numpy()
+    oW_t, obeta = oracle.quantize_weights(W)
+    ref = oracle.forward(x, oW_t, obeta)
+    assert np.all(y[0] == 0)
+    assert_f32_close(y, ref["y64"])
+
+
+# --------------------------------------------------------------------------
+# prefill GEMM (M > 64, tcgen05): accumulators bit-exact, tails in M, N, K
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,N", [(128, 128, 256), (65, 64, 5), (200, 1088, 300), (129, 4096, 257),
+                                   (511, 1024, 512), (512, 2048, 256), (513, 640, 1000), (300, 6912, 64),
+                                   (2047, 256, 130), (2049, 512, 260)])
+def test_gemm_parity_tails(dev, M, K, N):
+    run_case(dev, M, K, N, seed=M + 3 * K + N)
+
+
+@pytest.mark.parametrize("y_dtype", ["f32", "bf16"])
+def test_gemm_output_dtypes(dev, y_dtype):
+    run_case(dev, 300, 2048, 777, 31, y_dtype=y_dtype, outliers=True)
+
+
+def test_gemm_matches_gemv_on_same_inputs(dev):
+    # the dispatch boundary: rows computed by the GEMM equal those of the GEMV
+    K, N = 4096, 1000
+    W = workloads.latent_weights(41, N, K)
+    x = workloads.activations(42, 130, K, outliers=True)
+    W_t, beta, W_p = gpu_prep(W, dev)
+    x_q, gamma = bl.quant_act(T(x, dev))
+    y_gemm = bl.forward(x_q, gamma, W_p, beta).cpu().numpy()
+    for lo in (0, 64, 66):
+        # slices are cloned: the ABI requires 16-byte aligned pointers
+        y_gemv = bl.forward(x_q[lo:lo + 64].clone(), gamma[lo:lo + 64].clone(), W_p, beta).cpu().numpy()
+        np.testing.assert_array_equal(y_gemm[lo:lo + 64], y_gemv)
+
+
+def _sampled_rows_check(dev, shape, n_rows=48):
+    W = shape.weights()
+    x = shape.inputs()
+    W_t, beta, W_p = gpu_prep(W, dev)
+    x_q, gamma = bl.quant_act(T(x, dev))
+    acc = bl.forward_acc(x_q, W_p).cpu().numpy()
+    y = bl.forward(x_q, gamma, W_p, beta, out_dtype=torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    oW_t, obeta = oracle.quantize_weights(W)
+    assert beta.item() == float(obeta)
+    rows = np.random.default_rng(shape.M + shape.N).choice(shape.M, n_rows, replace=False)
+    rows[:2] = [0, shape.M - 1]
+    ref = oracle.forward(x[rows], oW_t, obeta)     # per-token quantiser: a row subset is exact
+    np.testing.assert_array_equal(x_q.cpu().numpy()[rows], ref["x_q"])
+    np.testing.assert_array_equal(acc[rows], ref["acc"])
+    assert_bf16_ok(y[rows], ref["y64"])
+
+
+@pytest.mark.parametrize("shape", workloads.W4.shapes, ids=lambda s: s.name)
+def test_workload_prefill_sampled_rows(dev, shape):
+    # full-size prefill (M = 2048) in the launch configuration the benchmark
+    # times; the oracle checks a sample of whole output rows
+    _sampled_rows_check(dev, shape)
