@@ -1,0 +1,439 @@
+"""Benchmark of the BitLinear W1.58A8 decode hot path on B200.
+
+One step = one pass of the decode hot path over one synthetic token batch of
+the FFN up/down decode workload (M = 1, bf16 activations with 1% x20 outlier
+channels):
+    quantise x_up  [1, 4096]  + ternary GEMV with W_up   [11008, 4096]
+    quantise x_dn  [1, 11008] + ternary GEMV with W_down [4096, 11008]
+each through the fused C-ABI call bitlinear_forward_fp (one kernel per
+projection).  Weights are prepared once (absmean ternarisation + 2-bit
+packing, outside the timed region) and rotate over enough copies that every
+step reads its weights from HBM (working set > L2).
+
+Printed metric: algorithmic GB/s (packed weights + activations + outputs per
+step / step time), whole job over all ranks, plus the roofline of the GEMV
+against the measured HBM copy bandwidth, the CPU oracle timed on the host,
+an end-to-end figure through the public API with host buffers, the prefill
+GEMM (M = 2048) in int8 TOPS against the int8 tensor peak, and SM clocks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "BitLinear W1.58A8 GEMV GB/s (frac of HBM peak); prefill GEMM int8 TOPS vs peak"
+WORKLOAD = workloads.W2
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : bf16 tensor ratio
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_decode_m1_traffic.json")
+
+
+def step_bytes() -> int:
+    return sum(s.algorithmic_bytes for s in WORKLOAD.shapes)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAK_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("k_gemv.cu", "common.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "ternary_weight_linear_forward_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current GEMV source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampler (reads only)."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([v.strip() for v in out.split(",")])
+            except (OSError, subprocess.SubprocessError):
+                return
+            self._stop.wait(0.05)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for s in self.samples for n, v in zip(names, s[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_step_fn(row_frac: float = 1.0):
+    """One oracle step over the workload; with row_frac < 1 only the first
+    row_frac of each weight matrix's output rows (a bounded sample).
+    Returns (step function, algorithmic bytes per step)."""
+    import oracle
+    prepared, nbytes = [], 0
+    for s in WORKLOAD.shapes:
+        rows = max(1, int(round(s.N * row_frac)))
+        W_t, beta = oracle.quantize_weights(s.weights())
+        prepared.append((s.inputs(), np.ascontiguousarray(W_t[:rows]), beta))
+        xb = 2 if s.x_dtype == "bf16" else 4
+        nbytes += rows * (s.K // 16) * 4 + s.M * s.K * xb + s.M * rows * 4
+
+    def step():
+        for x, W_t, beta in prepared:
+            r = oracle.forward(x, W_t, beta)
+            _ = r["y"]
+    return step, nbytes
+
+
+def run_cpu_oracle(budget_s: float, max_steps: int | None = None, step=None):
+    """Time the oracle, as it stands, on one host core: steps until max_steps
+    or until budget_s has elapsed."""
+    if step is None:
+        step, _ = cpu_oracle_step_fn()
+    step()  # warm caches, page in
+    n, t0 = 0, time.perf_counter()
+    while True:
+        step()
+        n += 1
+        el = time.perf_counter() - t0
+        if (max_steps and n >= max_steps) or el >= budget_s:
+            break
+    return n, el
+
+
+REF_ROW_FRAC = 1.0 / 8.0
+
+
+def reference_arm(args):
+    """The reference arm is the CPU oracle (there is no other implementation):
+    W untimed warm-up steps, then exactly K timed steps, each over the first
+    1/8 of every weight matrix's output rows."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    fn, nbytes = cpu_oracle_step_fn(REF_ROW_FRAC)
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    el = time.perf_counter() - t0
+    v = nbytes * args.steps / el / 1e9
+    sample = (f"each step: quantiser on the full activations + ternary GEMV over the first 1/8 of the output "
+              f"rows of both projections ({nbytes} algorithmic bytes per step)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8xt2->i32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD.name, "shapes": [s.name for s in WORKLOAD.shapes], "row_fraction": REF_ROW_FRAC},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import ternary_weight_linear_forward_b200 as bl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    L2 = props.L2_cache_size
+
+    # ---- offline weight preparation (not timed) ----
+    shapes = WORKLOAD.shapes
+    packed_bytes = sum(s.packed_bytes for s in shapes)
+    copies = max(2, int(4 * L2 // packed_bytes) + 1)       # working set >= 4x L2
+    layers = []
+    for s in shapes:
+        W = torch.from_numpy(s.weights()).to(dev)
+        W_t, beta = bl.quantize_weights(W)
+        W_p = bl.pack(W_t)
+        del W, W_t
+        xb = torch.from_numpy(s.inputs_bf16_bits().view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((s.M, s.N), dtype=torch.float32, device=dev)
+        layers.append({"shape": s, "W_p": [W_p] + [W_p.clone() for _ in range(copies - 1)], "beta": beta,
+                       "x": xb, "y": y})
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, which=None):
+        for j, L in enumerate(layers):
+            if which is None or which == j:
+                bl.forward_fp(L["x"], L["W_p"][i % copies], L["beta"], out=L["y"], stream=stream)
+
+    def capture(n, start, which=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    step(start + i, which)
+        return g
+
+    # graphs of at most CHUNK steps; the timed region replays exactly K steps
+    CHUNK = 256
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize()
+
+    def graphs_for(n, which=None):
+        gs, done = [], 0
+        while done < n:
+            k = min(CHUNK, n - done)
+            gs.append(capture(k, done, which))
+            done += k
+        return gs
+
+    warm = graphs_for(args.warmup)
+    timed = graphs_for(args.steps)
+
+    def run(gs):
+        for g in gs:
+            g.replay()
+
+    def timed_run(gs):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            run(gs)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            run(warm)
+        torch.cuda.synchronize()
+        t_step = timed_run(timed)
+    clocks = clk.summary()
+    t_max = t_step
+    if world > 1:
+        t = torch.tensor([t_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    ms_per_step = t_max / args.steps * 1e3
+    value = world * step_bytes() * args.steps / t_max / 1e9
+
+    # ---- roofline of the GEMV: each projection alone, same launch path ----
+    peaks, peak_kind = load_peaks()
+    per_shape = {}
+    launch_bytes, launch_time = 0.0, 0.0
+    for j, L in enumerate(layers):
+        n = max(64, min(args.steps, 1024))
+        gw = graphs_for(32, which=j)
+        with torch.cuda.stream(stream):
+            run(gw)
+        gs = graphs_for(n, which=j)
+        t = timed_run(gs)
+        s = L["shape"]
+        per_shape[s.name] = {"us_per_launch": t / n * 1e6, "GB/s": s.algorithmic_bytes * n / t / 1e9,
+                             "bytes_per_launch": s.algorithmic_bytes}
+        launch_bytes += s.algorithmic_bytes * n
+        launch_time += t
+        del gs, gw
+    achieved = launch_bytes / launch_time / 1e9
+    traffic = recorded_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                "kernel": "gemv_small_kernel (fused absmax int8 quantiser + ternary GEMV)",
+                "per_shape": per_shape}
+
+    # ---- end to end through the public API with pinned host buffers ----
+    host_x = [L["x"].cpu().pin_memory() for L in layers]
+    host_y = [torch.empty_like(L["y"], device="cpu").pin_memory() for L in layers]
+    dev_x = [torch.empty_like(L["x"]) for L in layers]
+    h2d = sum(h.numel() * h.element_size() for h in host_x)
+    d2h = sum(h.numel() * h.element_size() for h in host_y)
+    n_e2e = max(16, min(args.steps, 2000))
+
+    def e2e_step(i):
+        with torch.cuda.stream(stream):
+            for j, L in enumerate(layers):
+                dev_x[j].copy_(host_x[j], non_blocking=True)
+                bl.forward_fp(dev_x[j], L["W_p"][i % copies], L["beta"], out=L["y"], stream=stream)
+                host_y[j].copy_(L["y"], non_blocking=True)
+    for i in range(4):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_e2e):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([t_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_e2e = float(t.item())
+    e2e = {"value": world * step_bytes() * n_e2e / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": n_e2e,
+           "path": "pinned H2D copy + bitlinear_forward_fp per projection + D2H copy, one stream, no graph"}
+
+    # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
+    prefill = None
+    if not args.no_prefill:
+        prefill = {}
+        int8_peak_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
+        for s in workloads.W4.shapes:
+            W = torch.from_numpy(s.weights()).to(dev)
+            W_t, beta = bl.quantize_weights(W)
+            W_p = bl.pack(W_t)
+            del W, W_t
+            x = torch.from_numpy(s.inputs()).to(dev)
+            x_q, gamma = bl.quant_act(x)
+            y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.forward_workspace(s.M, s.N, s.K), dtype=torch.uint8, device=dev)
+            reps = 20
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    bl.forward(x_q, gamma, W_p, beta, out=y, ws=ws, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(reps):
+                        bl.forward(x_q, gamma, W_p, beta, out=y, ws=ws, stream=stream)
+            g.replay()
+            t = timed_run([g])
+            tops = s.ops * reps / t / 1e12
+            prefill[s.name] = {"us_per_call": t / reps * 1e6, "TOPS": tops,
+                               "frac_of_int8_peak": tops / int8_peak_burst,
+                               "frac_of_nominal_4500": tops / 4500.0}
+            del g, W_p, x, x_q, y, ws
+        prefill["int8_peak_TOPS"] = int8_peak_burst
+        prefill["int8_peak_source"] = (f"{peak_kind} bf16_tflops {peaks['bf16_tflops']} x nominal int8/bf16 ratio "
+                                       f"{INT8_OVER_BF16}")
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        fn, _ = cpu_oracle_step_fn()
+        n, el = run_cpu_oracle(float(os.environ.get("BENCH_CPU_BUDGET_S", "12")), step=fn)
+        cpu = {"value": step_bytes() * n / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} full steps of the workload (both projections), about "
+                         f"{float(os.environ.get('BENCH_CPU_BUDGET_S', '12')):.0f} s of one host core"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8xt2->i32", "data": "synthetic",
+            "config": {"workload": WORKLOAD.name, "shapes": [s.name for s in shapes],
+                       "x_dtype": "bf16", "y_dtype": "f32", "outlier_channels": "1% x20",
+                       "l2": f"inputs larger than L2: weights rotate over {copies} copies "
+                             f"({copies * packed_bytes / 1e6:.0f} MB vs L2 {L2 / 1e6:.0f} MB)",
+                       "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": len(shapes) * args.steps, "clocks": clocks, "prefill": prefill,
+            "device": props.name,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -36,10 +36,11 @@ namespace bl {
 namespace {
 
 constexpr int GEMV_MAX_STAGES = 32;
-constexpr int GEMV_HDR = 2048;  // barriers + per-token tables + reduction scratch
+constexpr int GEMV_HDR = 4096;  // barriers + per-token tables + reduction scratch
 constexpr int GEMV_MAX_M = 64;
-constexpr int GEMV_MAX_CWARPS = 11;                           // small kernel: <= 384 threads and
-constexpr int GEMV_MAX_THREADS = (GEMV_MAX_CWARPS + 1) * 32;  // <= 85 registers: two CTAs fit an SM
+constexpr int GEMV_MAX_CWARPS = 13;                           // small kernel: <= 448 threads and
+constexpr int GEMV_MAX_THREADS = (GEMV_MAX_CWARPS + 1) * 32;  // <= 73 registers: two CTAs fit an SM
+constexpr int GEMV_KS_MAX_ROWS = 64;                          // rows per CTA when K is split
 constexpr int GEMV_CO_RESIDENT = 2;                           // a kernel and its PDL successor
 constexpr int GEMV_MT_CWARPS = 8;  // consumer warps of the mt kernel
 constexpr int GEMV_CHUNK_TARGET = 8192;
@@ -62,6 +63,9 @@ struct GemvParams {
     int stages;        // ring depth
     int stage_stride;  // bytes per ring slot (rpc rows, a multiple of 16)
     int xq_bytes;      // shared-memory bytes reserved for x_q (small kernel)
+    int ks;            // K slices per row (small kernel): 1, 2 or 4
+    int slice4;        // 16-byte weight groups per slice
+    int wave;          // mt kernel: rows in flight per wave
 };
 
 struct Shared {
@@ -72,6 +76,7 @@ struct Shared {
     float fscale[GEMV_MAX_M];
     unsigned red_u[GEMV_MAX_CWARPS][GEMV_SMALL_MAX_M];
     int red_i[GEMV_MAX_CWARPS][GEMV_SMALL_MAX_M];
+    int part[GEMV_KS_MAX_ROWS][GEMV_SMALL_MAX_M];  // K-slice partial sums
 };
 static_assert(sizeof(Shared) <= GEMV_HDR, "header too large");
 
@@ -256,6 +261,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
             s[m] = __fdiv_rn(127.0f, gam[m]);
         }
     }
+    for (int i = ctid; i < GEMV_KS_MAX_ROWS * GEMV_SMALL_MAX_M; i += cthreads) (&sh.part[0][0])[i] = 0;
     // pass 2: write x_q chunks into their swizzled slots, accumulate row sums
     int rs[MT];
 #pragma unroll
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&sh.full[s], 1);
-            mbar_init(&sh.empty[s], p.rpc);
+            mbar_init(&sh.empty[s], p.rpc * p.ks);  // every K slice of every row releases once
         }
         sh.abort_flag = 0;
         fence_mbar_init();
@@ -383,33 +389,41 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small
     const int tl = ctid % LPR;
     const int K4 = p.K / 64;  // 16-byte groups of packed weights per row
     const int G = p.K / 16;   // 16-byte chunks of x_q per token
-    const int iters = (nrows + T * R - 1) / (T * R);  // warp-uniform trip count
+    const int KS = p.ks;
+    // work item = (group of R rows, K slice); warp-uniform trip count
+    const int items = (nrows + R - 1) / R * KS;
+    const int iters = (items + T - 1) / T;
 
     for (int it = 0; it < iters; ++it) {
-        const int b = (it * T + team) * R;
-        const int nvalid = max(0, min(R, nrows - b));
+        const int item = it * T + team;
+        const int b = (item / KS) * R;
+        const int sl = item % KS;
+        const int k_lo = sl * p.slice4, k_hi = min(K4, k_lo + p.slice4);
+        const int nvalid = item < items ? max(0, min(R, nrows - b)) : 0;
         bool ok = nvalid > 0;
         for (int r = 0; r < nvalid; ++r) ok = ok && wait_row(p, sh, b + r);
         // row offsets once per team-iteration (missing rows alias row b)
         uint32_t ro[R];
 #pragma unroll
         for (int r = 0; r < R; ++r)
-            ro[r] = (uint32_t)(reinterpret_cast<const unsigned char*>(row_ptr(p, ring, b + (r < nvalid ? r : 0))) - ring);
+            ro[r] = ok ? (uint32_t)(reinterpret_cast<const unsigned char*>(row_ptr(p, ring, b + (r < nvalid ? r : 0))) -
+                                    ring)
+                       : 0u;
         int a[R][MT][4];
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
             for (int m = 0; m < MT; ++m) a[r][m][0] = a[r][m][1] = a[r][m][2] = a[r][m][3] = 0;
-        if (ok && tl < K4) {
+        if (ok && k_lo + tl < k_hi) {
             // software pipeline: the next group's weights load while this one is used
             uint4 wn[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * tl);
-            for (int idx = tl; idx < K4; idx += LPR) {
+            for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * (k_lo + tl));
+            for (int idx = k_lo + tl; idx < k_hi; idx += LPR) {
                 uint4 w[R];
 #pragma unroll
                 for (int r = 0; r < R; ++r) w[r] = wn[r];
-                const int nxt = idx + LPR < K4 ? idx + LPR : idx;
+                const int nxt = idx + LPR < k_hi ? idx + LPR : idx;
 #pragma unroll
                 for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * nxt);
                 const int key = (idx >> 1) & 3;  // swizzle of chunks 4 idx .. 4 idx + 3
@@ -440,8 +454,24 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small
             const int r = which / MT, m = which % MT;
             if (r < nvalid) {
                 if (m == 0) release_row(p, sh, b + r);
-                if (m < p.M) store_y(p, m, r0 + b + r, tot - sh.rowsum[m], sh.fscale[m]);
+                if (KS == 1) {
+                    if (m < p.M) store_y(p, m, r0 + b + r, tot - sh.rowsum[m], sh.fscale[m]);
+                } else {
+                    atomicAdd(&sh.part[b + r][m], tot);
+                }
             }
+        }
+        // With a recycled ring, the rows of one iteration fit strictly inside
+        // the ring (host-side sizing) and no team starts the next iteration
+        // before all have finished this one: a parity wait then never meets a
+        // slot two loads behind the one it asks for.
+        if (p.reuse) consumer_sync(cthreads);
+    }
+    if (KS > 1) {  // all slices of every row are in: finish the rows
+        consumer_sync(cthreads);
+        for (int i = ctid; i < nrows * MT; i += cthreads) {
+            const int r = i / MT, m = i % MT;
+            if (m < p.M) store_y(p, m, r0 + r, sh.part[r][m] - sh.rowsum[m], sh.fscale[m]);
         }
     }
 }
@@ -484,39 +514,48 @@ __global__ void __launch_bounds__((GEMV_MT_CWARPS + 1) * 32, 1) gemv_mt_kernel(c
     }
     consumer_sync(GEMV_MT_CWARPS * 32);
 
-    for (int i = warp; i < nrows; i += GEMV_MT_CWARPS) {
+    // rows go out in waves of p.wave (<= consumer warps); with a recycled ring a
+    // wave fits strictly inside it and waves are separated by a barrier
+    for (int base = 0; base < nrows; base += p.wave) {
+        const int i = base + warp;
+        const bool mine = warp < p.wave && i < nrows;
         // every lane waits the same barrier; the decision is made warp-uniform
-        if (!__all_sync(0xffffffffu, wait_row(p, sh, i))) break;
-        const uint4* wrow = row_ptr(p, ring, i);
-        for (int m0 = 0; m0 < p.M; m0 += MT) {
-            int a[MT][4];
+        const bool ok = __all_sync(0xffffffffu, mine && wait_row(p, sh, i));
+        if (ok) {
+            const uint4* wrow = row_ptr(p, ring, i);
+            for (int m0 = 0; m0 < p.M; m0 += MT) {
+                int a[MT][4];
 #pragma unroll
-            for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0;
-            for (int idx = lane; idx < K4; idx += 32) {
-                const uint4 w = wrow[idx];
-                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0;
+                for (int idx = lane; idx < K4; idx += 32) {
+                    const uint4 w = wrow[idx];
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m0 + m < p.M) {
-                        const int4* px = reinterpret_cast<const int4*>(p.x_q + (long long)(m0 + m) * p.K) + 4 * idx;
+                    for (int m = 0; m < MT; ++m) {
+                        if (m0 + m < p.M) {
+                            const int4* px =
+                                reinterpret_cast<const int4*>(p.x_q + (long long)(m0 + m) * p.K) + 4 * idx;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int4 xv = __ldg(px + q);
-                            word_dot(wv[q], xv.x, xv.y, xv.z, xv.w, a[m][0], a[m][1], a[m][2], a[m][3]);
+                            for (int q = 0; q < 4; ++q) {
+                                const int4 xv = __ldg(px + q);
+                                word_dot(wv[q], xv.x, xv.y, xv.z, xv.w, a[m][0], a[m][1], a[m][2], a[m][3]);
+                            }
                         }
                     }
                 }
-            }
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                int acc = combine4(a[m][0], a[m][1], a[m][2], a[m][3]);
+                for (int m = 0; m < MT; ++m) {
+                    int acc = combine4(a[m][0], a[m][1], a[m][2], a[m][3]);
 #pragma unroll
-                for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == 0 && m0 + m < p.M) store_y(p, m0 + m, r0 + i, acc - sh.rowsum[m0 + m], sh.fscale[m0 + m]);
+                    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    if (lane == 0 && m0 + m < p.M)
+                        store_y(p, m0 + m, r0 + i, acc - sh.rowsum[m0 + m], sh.fscale[m0 + m]);
+                }
             }
+            __syncwarp();
+            if (lane == 0) release_row(p, sh, i);
         }
-        __syncwarp();
-        if (lane == 0) release_row(p, sh, i);
+        if (p.reuse) consumer_sync(GEMV_MT_CWARPS * 32);
     }
 }
 
@@ -576,33 +615,51 @@ cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st)
 
     const int mt = small_mt(M);
     if (M <= GEMV_SMALL_MAX_M && mt * K <= GEMV_XQ_SMEM_MAX) {
-        // Choose lanes-per-row (team size) and rows-per-team-iteration so that
-        // every row of the CTA fits in one team-iteration when possible, with
-        // the fewest idle lanes; then size the CTA to the teams it needs.
-        int lpr = 32, r = 1;
-        double best = -1.0;
-        for (int cand_r : {4, 2, 1}) {
-            if (cand_r * mt > 4) continue;
-            for (int l : {32, 16, 8}) {
-                const int upl = (K4 + l - 1) / l;
-                const double lane_eff = (double)K4 / (l * upl);
-                const int teams_cap = GEMV_MAX_CWARPS * 32 / l;
-                const int iters = (rows_per_cta + teams_cap * cand_r - 1) / (teams_cap * cand_r);
-                const double score = lane_eff / iters + 0.01 * cand_r;  // prefer one pass, then ILP
-                if (score > best + 1e-9) {
-                    best = score;
-                    lpr = l;
-                    r = cand_r;
-                }
+        // Launch shape (measured on B200 over lanes-per-row x rows-per-team x
+        // K-slices x warps for the 4096x11008 and 11008x4096 decode shapes):
+        // about ten consumer warps, two rows per team (one when M > 2), and the
+        // widest team for which every row of the CTA still fits one pass.
+        const int cw_target = 10;
+        int r = std::max(1, 2 / mt);
+        const int teams_needed = (rows_per_cta + r - 1) / r;
+        int lpr = 8;
+        for (int l : {32, 16, 8}) {
+            if (teams_needed * l <= cw_target * 32) {
+                lpr = l;
+                break;
             }
         }
-        const int teams = (rows_per_cta + r - 1) / r;
-        const int cwarps = std::max(1, std::min(GEMV_MAX_CWARPS, (teams * lpr + 31) / 32));
+        int ks = 1;
+        if (rows_per_cta <= GEMV_KS_MAX_ROWS && lpr == 32 && (cw_target * 32 / lpr) * r >= 2 * rows_per_cta)
+            ks = 2;  // few rows: split K so every warp has work
+        p.ks = ks;
+        p.slice4 = (K4 + ks - 1) / ks;
+        const int items = (rows_per_cta + r - 1) / r * ks;
+        int cwarps = std::max(1, std::min(cw_target, (items * lpr + 31) / 32));
         p.xq_bytes = (mt * K + 127) / 128 * 128;
         // leave room for the next launch's CTA on the same SM
         const int budget = (max_dyn - 1024) / GEMV_CO_RESIDENT;
         const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * (K / 4));
         ring_geometry(p, rows_per_cta, ring_bytes);
+        if (p.reuse) {
+            // one team per warp, and the rows of one iteration (ceil(teams / ks) * r)
+            // within (stages - 1) * rpc so that they never wrap onto a slot twice
+            const int window = std::max(1, (p.stages - 1) * p.rpc);
+            if (lpr != 32) {
+                lpr = 32;
+                p.slice4 = (K4 + ks - 1) / ks;
+            }
+            r = std::min(r, window);
+            while (r > 1 && (r & (r - 1))) --r;  // keep r in {1, 2, 4}
+            const int teams_max = std::max(1, window / r * ks);
+            cwarps = std::max(1, std::min(cwarps, teams_max));
+            // teams per iteration a multiple (or divisor) of ks: iterations then
+            // start on row-group boundaries
+            if (cwarps >= ks)
+                cwarps = cwarps / ks * ks;
+            else
+                while (ks % cwarps) --cwarps;
+        }
         const size_t smem = GEMV_HDR + p.xq_bytes + (size_t)p.stages * p.stage_stride;
         GemvKernel k = p.x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED>(lpr, mt, r)
                        : p.x_mode == X_F32     ? small_kernel_for<X_F32>(lpr, mt, r)
@@ -612,6 +669,7 @@ cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st)
     if (p.x_mode != X_QUANTISED) return cudaErrorInvalidValue;  // callers quantise first
     p.xq_bytes = 0;
     ring_geometry(p, rows_per_cta, max_dyn - GEMV_HDR);
+    p.wave = p.reuse ? std::max(1, std::min(GEMV_MT_CWARPS, (p.stages - 1) * p.rpc)) : GEMV_MT_CWARPS;
     const size_t smem = GEMV_HDR + (size_t)p.stages * p.stage_stride;
     const int threads = (GEMV_MT_CWARPS + 1) * 32;
     if (M <= 1) return launch_with_smem(gemv_mt_kernel<1>, grid, threads, smem, st, p);

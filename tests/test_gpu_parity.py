@@ -180,6 +180,12 @@ def test_gemv_row_partition_tails(dev, N):
     run_case(dev, 5, 1024, N, seed=N + 1)
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 32768, 5000), (3, 16384, 9000), (2, 65536, 700)])
+def test_gemv_ring_reuse(dev, M, K, N):
+    # slabs larger than the shared-memory ring: chunks recycle ring slots
+    run_case(dev, M, K, N, seed=K + N)
+
+
 def test_gemv_bf16_output(dev):
     run_case(dev, 1, 4096, 2000, 21, y_dtype="bf16")
     run_case(dev, 9, 2560, 700, 22, y_dtype="bf16")
