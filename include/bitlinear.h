@@ -175,6 +175,33 @@ bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K,
                                 const uint32_t* W_p, int64_t N, int32_t* acc,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* Rows the built-in scratch of bitlinear_forward_noalloc holds (64 KiB of int32). */
+#define BL_NOALLOC_MAX_M 16384
+
+/*
+ * bitlinear_forward for callers that cannot allocate device memory -- a C
+ * runtime with a fixed arena and no device allocator to hand the library,
+ * or code being recorded into a stream capture where an allocation is not
+ * allowed.  The pages have no counterpart: this is a library convenience.
+ * Same arguments, kernels, dispatch and results as bitlinear_forward, without
+ * ws/ws_bytes: the M int32 row sums the prefill path (M > 64) needs live in a
+ * static device array of the library (BL_NOALLOC_MAX_M entries, held by every
+ * device that loads the library until exit); the decode path (M <= 64) needs
+ * no scratch.
+ *   - M > BL_NOALLOC_MAX_M returns BL_ERR_WORKSPACE (scratch too small), with
+ *     nothing launched.
+ *   - The first call on a device looks up the array's device address and
+ *     checks the device (no allocation); make that first call before any
+ *     stream capture on that device.
+ *   - Every call on a device shares the array and overwrites the rows it
+ *     uses before reading them; calls that overlap on the GPU (for example on
+ *     two streams) race on it and must be serialised by the caller.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
+                                    const uint32_t* W_p, const float* beta, int64_t N,
+                                    void* y, int y_dtype, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Decoder-block glue                                                        */
 /* ------------------------------------------------------------------------ */

@@ -37,6 +37,7 @@ SIGNATURES = {
     "bitlinear_forward_fp_workspace": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward_fp": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_device_status": (_I, [_P]),
     "bitlinear_num_sms": (_I, []),
@@ -192,6 +193,30 @@ def forward_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype
     _check("bitlinear_forward_fp",
            lib().bitlinear_forward_fp(_ptr(x), xdt, M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt, _ptr(ws),
                                       0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_noalloc(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,
+                    out_dtype=torch.float32, out=None, stream=None) -> torch.Tensor:
+    """forward() for callers that cannot allocate device memory: the library
+    keeps the prefill scratch in a static device array (M <= 16384; the first
+    call on a device should come before any stream capture; concurrent calls
+    on one device race on the shared scratch).  Only ``out`` is allocated
+    here, and only when it is not given."""
+    _need(x_q, torch.int8, 2, "x_q")
+    _need(W_p, torch.int32, 2, "W_p")
+    _need(gamma, torch.float32, 1, "gamma")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x_q.shape
+    N = W_p.shape[0]
+    if W_p.shape[1] * 16 != K:
+        raise ValueError("W_p must be [N, K/16]")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    _check("bitlinear_forward_noalloc",
+           lib().bitlinear_forward_noalloc(_ptr(x_q), _ptr(gamma), M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                           _stream(stream)))
     return out
 
 
