@@ -405,6 +405,33 @@ def main():
         prefill["int8_peak_source"] = (f"{peak_kind} bf16_tflops {peaks['bf16_tflops']} x nominal int8/bf16 ratio "
                                        f"{INT8_OVER_BF16}")
 
+    # ---- decoder block at batch-1 decode (hidden 2560, intermediate 6912) ----
+    block = None
+    if not args.no_prefill:
+        bw = {p: torch.from_numpy(w).to(dev) for p, w in workloads.block_weights().items()}
+        nblk = max(2, int(1.2 * L2 // sum(w.numel() // 4 for w in bw.values())) + 1)   # >= 1.2x L2 of weights
+        blocks = [bl.DecoderBlock.from_float(bw) for _ in range(nblk)]
+        del bw
+        bx = torch.from_numpy(workloads.block_input()).to(dev)
+        wbytes = sum(L.W_p.numel() * 4 for L in blocks[0].layers.values())
+        with torch.cuda.stream(stream):
+            for b_ in blocks:
+                b_(bx)
+        torch.cuda.synchronize()
+        reps = 8 * nblk
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(reps):
+                    blocks[i % nblk](bx)
+        g.replay()
+        t = timed_run([g])
+        us = t / reps * 1e6
+        block = {"us_per_block": us, "weight_bytes": wbytes, "GB/s": wbytes / (t / reps) / 1e9,
+                 "frac_of_hbm": wbytes / (t / reps) / 1e9 / peaks["hbm_gbs"], "kernels_per_block": 12,
+                 "copies": nblk}
+        del g, blocks
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -425,7 +452,7 @@ def main():
                              f"({copies * packed_bytes / 1e6:.0f} MB vs L2 {L2 / 1e6:.0f} MB)",
                        "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": len(shapes) * args.steps, "clocks": clocks, "prefill": prefill,
+            "gpu_launches": len(shapes) * args.steps, "clocks": clocks, "prefill": prefill, "block": block,
             "device": props.name,
         }
         print(json.dumps(line), flush=True)
