@@ -43,7 +43,11 @@ constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words
 constexpr int STAGE_BYTES = A_BYTES + BC_BYTES + BP_BYTES;
 constexpr int HDR_BYTES = 1024;
 constexpr int GEMM_SMEM = 1024 /* alignment slack */ + HDR_BYTES + STAGES * STAGE_BYTES;
-constexpr int GEMM_THREADS = 320;
+constexpr int UNPACK_WARPS = 8;
+constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
+constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;               // epilogue warps EPI_WARP0 .. +3
+constexpr int GEMM_THREADS = (EPI_WARP0 + 4) * 32;
+constexpr int WORDS_PER_THREAD = BN * (BK / 16) / UNPACK_THREADS;  // packed words per K-block
 constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators
 
 struct GemmHdr {
@@ -233,7 +237,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&h.full[s], 1);
-            mbar_init(&h.unpacked[s], 128);
+            mbar_init(&h.unpacked[s], UNPACK_THREADS);
             mbar_init(&h.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -297,9 +301,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 mma_commit(&h.tfull[b]);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < EPI_WARP0) {
         // ------------------------------------------------ unpack
-        const int ut = threadIdx.x - 64;  // 0..127
+        const int ut = threadIdx.x - 64;  // 0 .. UNPACK_THREADS - 1
+        // word w = ut + UNPACK_THREADS * i of the packed tile is row n = w / 8,
+        // word j = w % 8: its 16 codes go to 16-byte chunk j ^ (n % 8) of row n
+        uint32_t dst_off[WORDS_PER_THREAD];
+#pragma unroll
+        for (int i = 0; i < WORDS_PER_THREAD; ++i) {
+            const int w = ut + UNPACK_THREADS * i;
+            const int n = w >> 3, j = w & 7;
+            dst_off[i] = (uint32_t)(n * BK + ((j ^ (n & 7)) << 4));
+        }
         int it = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
@@ -309,18 +322,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 unsigned char* st = stages + (size_t)s * STAGE_BYTES;
                 const uint32_t* bp = reinterpret_cast<const uint32_t*>(st + A_BYTES + BC_BYTES);
                 const uint32_t bc = smem_u32(st + A_BYTES);
-#pragma unroll 4
-                for (int i = 0; i < BN * (BK / 16) / 128; ++i) {
-                    const int w = ut + 128 * i;
-                    const int n = w >> 3, j = w & 7;
-                    const uint32_t word = bp[w];
-                    const uint32_t t0 = word & 0x03030303u;
-                    const uint32_t t1 = (word >> 2) & 0x03030303u;
-                    const uint32_t t2 = (word >> 4) & 0x03030303u;
-                    const uint32_t t3 = (word >> 6) & 0x03030303u;
-                    const uint32_t dst = bc + (uint32_t)(n * BK + ((j ^ (n & 7)) << 4));
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(t0), "r"(t1), "r"(t2),
-                                 "r"(t3)
+                uint32_t word[WORDS_PER_THREAD];
+#pragma unroll
+                for (int i = 0; i < WORDS_PER_THREAD; ++i) word[i] = bp[ut + UNPACK_THREADS * i];
+#pragma unroll
+                for (int i = 0; i < WORDS_PER_THREAD; ++i) {
+                    const uint32_t t0 = word[i] & 0x03030303u;
+                    const uint32_t t1 = (word[i] >> 2) & 0x03030303u;
+                    const uint32_t t2 = (word[i] >> 4) & 0x03030303u;
+                    const uint32_t t3 = (word[i] >> 6) & 0x03030303u;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(bc + dst_off[i]), "r"(t0), "r"(t1),
+                                 "r"(t2), "r"(t3)
                                  : "memory");
                 }
                 fence_proxy_async_smem();
