@@ -59,7 +59,7 @@ enum {
     BL_ERR_ALIAS = 9       /* an output overlaps an input */
 };
 
-enum { BL_F32 = 0, BL_BF16 = 1 };
+enum { BL_F32 = 0, BL_BF16 = 1, BL_I8 = 2 /* already-quantised x_q with per-token gamma */ };
 
 /* Largest K accepted (keeps every int32 partial of the contraction exact). */
 #define BL_MAX_K 262144
@@ -165,6 +165,34 @@ size_t bitlinear_forward_fp_workspace(int64_t M, int64_t N, int64_t K);
 bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* W_p,
                                const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
                                void* stream);
+
+/* One problem of a bitlinear_forward_fp_batch call. */
+typedef struct {
+    const void* x;          /* [M, K] activations (x_dtype of the call), in */
+    const float* gamma;     /* [M] per-token scale when x_dtype is BL_I8 (x is x_q), else unused */
+    const uint32_t* W_p;    /* [N, K/16] packed weights (bitlinear_pack layout), in */
+    const float* beta;      /* [1] absmean scale of W_p, in */
+    void* y;                /* [M, N] output (y_dtype of the call), out */
+    int64_t K, N;
+} bl_problem;
+
+/* Most problems one bitlinear_forward_fp_batch call takes. */
+#define BL_BATCH_MAX 8
+
+/*
+ * Several independent decode projections in one launch: bitlinear_forward_fp
+ * on each problem (same results, bit for bit), or bitlinear_forward when
+ * x_dtype is BL_I8 (x holds x_q and gamma the per-token scales), e.g. the q / k / v
+ * projections of one token, gate and up, or projections of different layers
+ * whose inputs are ready.  The problems share M (<= 4), x_dtype and y_dtype;
+ * each needs (M rounded up to 1, 2 or 4) * K <= 65536, K % 64 == 0.  Every SM
+ * runs one CTA per problem, so their HBM streams and fixed latencies overlap.
+ * Outputs must not overlap any input or each other.
+ *   problems: host array of `count` descriptors (1 <= count <= BL_BATCH_MAX),
+ *             read during the call only.
+ */
+bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int64_t M, int x_dtype, int y_dtype,
+                                     void* stream);
 
 /*
  * Inspection variant of bitlinear_forward: writes the int32 accumulators

@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
 
-BL_F32, BL_BF16 = 0, 1
+BL_F32, BL_BF16, BL_I8 = 0, 1, 2
 COMBINE = {"none": 0, "add": 1, "silu_mul": 2}
 EPS_W = 1e-5
 
@@ -36,6 +36,7 @@ SIGNATURES = {
     "bitlinear_forward": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_forward_fp_workspace": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward_fp": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_fp_batch": (_I, [_P, _I, _I64, _I, _I, _P]),
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
@@ -196,6 +197,54 @@ def forward_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype
     return out
 
 
+class _Problem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("W_p", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("y", ctypes.c_void_p),
+                ("K", ctypes.c_int64), ("N", ctypes.c_int64)]
+
+
+def forward_fp_batch(problems, out_dtype=torch.float32, stream=None):
+    """Several independent decode projections in one launch.
+
+    ``problems``: list of dicts with keys ``x`` ([M, K] fp32/bf16, or int8 x_q
+    together with ``gamma`` [M]), ``W_p``, ``beta`` and optionally ``out``.
+    All share M (<= 4) and the x dtype.  Returns the list of outputs."""
+    if not 1 <= len(problems) <= 8:
+        raise ValueError("1 to 8 problems")
+    arr = (_Problem * len(problems))()
+    outs = []
+    x0 = problems[0]["x"]
+    quantised = x0.dtype == torch.int8
+    for i, pr in enumerate(problems):
+        x, W_p, beta = pr["x"], pr["W_p"], pr["beta"]
+        if x.dtype != x0.dtype or x.shape[0] != x0.shape[0]:
+            raise ValueError("problems must share M and the x dtype")
+        _need(x, x.dtype, 2, "x")
+        _need(W_p, torch.int32, 2, "W_p")
+        _need(beta, torch.float32, 1, "beta")
+        gamma = pr.get("gamma")
+        if quantised:
+            _need(gamma, torch.float32, 1, "gamma")
+        M, K = x.shape
+        N = W_p.shape[0]
+        if W_p.shape[1] * 16 != K:
+            raise ValueError("W_p must be [N, K/16]")
+        out = pr.get("out")
+        if out is None:
+            out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+        outs.append(out)
+        arr[i] = _Problem(x.data_ptr(), gamma.data_ptr() if quantised else None, W_p.data_ptr(), beta.data_ptr(),
+                          out.data_ptr(), K, N)
+    if any(o.dtype != outs[0].dtype for o in outs):
+        raise ValueError("outputs must share a dtype")
+    ydt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[outs[0].dtype]
+    xdt = BL_I8 if quantised else BL_BF16 if x0.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_forward_fp_batch",
+           lib().bitlinear_forward_fp_batch(ctypes.cast(arr, ctypes.c_void_p), len(problems), x0.shape[0], xdt, ydt,
+                                            _stream(stream)))
+    return outs
+
+
 def forward_noalloc(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,
                     out_dtype=torch.float32, out=None, stream=None) -> torch.Tensor:
     """forward() for callers that cannot allocate device memory: the library
@@ -329,13 +378,13 @@ class DecoderBlock:
         xh = (b["xq_h"], b["g_h"])
         xf = (b["xq_f"], b["g_f"])
         quant_act_rms(x, out=xh)
-        for p in ("q", "k", "v"):
-            forward(*xh, L[p].W_p, L[p].beta, out=b[p])
+        forward_fp_batch([{"x": xh[0], "gamma": xh[1], "W_p": L[p].W_p, "beta": L[p].beta, "out": b[p]}
+                          for p in ("q", "k", "v")])
         quant_act_rms(b["v"], out=xh)                     # attention over one token = v
         forward(*xh, L["o"].W_p, L["o"].beta, out=b["o"])
         quant_act_rms(x, b["o"], "add", h=b["h1"], out=xh)
-        forward(*xh, L["gate"].W_p, L["gate"].beta, out=b["gate"])
-        forward(*xh, L["up"].W_p, L["up"].beta, out=b["up"])
+        forward_fp_batch([{"x": xh[0], "gamma": xh[1], "W_p": L[p].W_p, "beta": L[p].beta, "out": b[p]}
+                          for p in ("gate", "up")])
         quant_act_rms(b["gate"], b["up"], "silu_mul", h=b["u"] if keep_u else None, out=xf)
         forward(*xf, L["down"].W_p, L["down"].beta, out=b["down"])
         quant_act_rms(b["h1"], b["down"], "add", h=b["out"], quantize=False)

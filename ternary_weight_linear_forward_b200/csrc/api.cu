@@ -257,6 +257,44 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
                        stream);
 }
 
+bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int64_t M, int x_dtype, int y_dtype,
+                                     void* stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BL_BATCH_MAX || count > gemv_group_max()) return BL_ERR_SHAPE;
+    if ((x_dtype != BL_F32 && x_dtype != BL_BF16 && x_dtype != BL_I8) || (y_dtype != BL_F32 && y_dtype != BL_BF16))
+        return BL_ERR_DTYPE;
+    if (M < 1 || !gemv_fused_quant_ok(M, 64)) return BL_ERR_SHAPE;
+    const size_t xe = x_dtype == BL_BF16 ? 2 : x_dtype == BL_I8 ? 1 : 4, ye = y_dtype == BL_F32 ? 4 : 2;
+    GemvProblem probs[BL_BATCH_MAX];
+    for (int i = 0; i < count; ++i) {
+        const bl_problem& q = problems[i];
+        if (!q.x || !q.W_p || !q.beta || !q.y || (x_dtype == BL_I8 && !q.gamma)) return BL_ERR_NULL;
+        bl_status s = check_nk(q.N, q.K, 64);
+        if (s) return s;
+        if (!gemv_fused_quant_ok(M, q.K)) return BL_ERR_SHAPE;
+        if (!aligned16(q.x) || !aligned16(q.W_p) || !aligned16(q.beta) || !aligned16(q.y) ||
+            (x_dtype == BL_I8 && !aligned16(q.gamma)))
+            return BL_ERR_ALIGN;
+        probs[i] = {q.x, x_dtype == BL_I8 ? q.gamma : nullptr, q.W_p, q.beta, q.y, (int)q.K, (int)q.N};
+    }
+    for (int i = 0; i < count; ++i) {  // no output overlaps any input or another output
+        const bl_problem& a = problems[i];
+        const size_t yb = (size_t)M * a.N * ye;
+        for (int j = 0; j < count; ++j) {
+            const bl_problem& b = problems[j];
+            if (overlap(a.y, yb, b.x, (size_t)M * b.K * xe) || overlap(a.y, yb, b.W_p, (size_t)b.N * (b.K / 16) * 4) ||
+                (x_dtype == BL_I8 && overlap(a.y, yb, b.gamma, (size_t)M * 4)) ||
+                overlap(a.y, yb, b.beta, 4) || (i != j && overlap(a.y, yb, b.y, (size_t)M * b.N * ye)))
+                return BL_ERR_ALIAS;
+        }
+    }
+    DevInfo dev;
+    bl_status s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype,
+                                             y_dtype == BL_F32 ? Y_F32 : Y_BF16, dev, as_stream(stream)));
+}
+
 bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,
                                 int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
     bl_status s = check_forward(x_q, nullptr, M, K, W_p, nullptr, N, acc, 4);

@@ -157,10 +157,10 @@ __device__ __forceinline__ const uint4* row_ptr(const GemvParams& p, const unsig
                                           (size_t)(i & (p.rpc - 1)) * (p.K / 4));
 }
 
-__device__ __forceinline__ void cta_rows(const GemvParams& p, int& r0, int& nrows) {
+__device__ __forceinline__ void cta_rows(const GemvParams& p, int cta, int ncta, int& r0, int& nrows) {
     const long long N = p.N;
-    r0 = (int)((N * blockIdx.x) / gridDim.x);
-    const int r1 = (int)((N * (blockIdx.x + 1)) / gridDim.x);
+    r0 = (int)((N * cta) / ncta);
+    const int r1 = (int)((N * (cta + 1)) / ncta);
     nrows = r1 - r0;
 }
 
@@ -350,9 +350,9 @@ __device__ __forceinline__ int team_reduce(const int (&v)[V], int tl, int& which
 
 // ---------------------------------------------------------------- M <= 4
 
+// One CTA's share (CTA `cta` of `ncta` working on problem p) of the M <= 4 forward.
 template <int LPR, int MT, int R, int XM>
-__global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small_kernel(const GemvParams p) {
-    extern __shared__ __align__(128) unsigned char smem[];
+__device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, int ncta, unsigned char* smem) {
     Shared& sh = *reinterpret_cast<Shared*>(smem);
     int4* xsm = reinterpret_cast<int4*>(smem + GEMV_HDR);
     unsigned char* ring = smem + GEMV_HDR + p.xq_bytes;
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small
     const int cwarps = blockDim.x / 32 - 1;  // warp 0 produces, warps 1.. consume
     const int cthreads = cwarps * 32;
     int r0, nrows;
-    cta_rows(p, r0, nrows);
+    cta_rows(p, cta, ncta, r0, nrows);
     const int nchunks = (nrows + p.rpc - 1) / p.rpc;
     // Thread 0 sets up the barriers and puts the slab's bulk copies in flight
     // before anyone else runs, so the HBM stream starts as early as possible.
@@ -476,6 +476,38 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small
     }
 }
 
+template <int LPR, int MT, int R, int XM>
+__global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small_kernel(const GemvParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    gemv_small_body<LPR, MT, R, XM>(p, blockIdx.x, gridDim.x, smem);
+}
+
+// Several independent problems (same M, same x / y formats) in one launch:
+// CTAs [cta0[i], cta0[i+1]) work on problem i.  Each problem keeps its own
+// launch shape (lanes per row); the block size is the largest of them.
+constexpr int GEMV_GROUP_MAX = 8;
+
+struct GroupParams {
+    GemvParams prob[GEMV_GROUP_MAX];
+    int lpr[GEMV_GROUP_MAX];
+    int cta0[GEMV_GROUP_MAX + 1];
+    int count;
+};
+
+template <int MT, int R, int XM>
+__global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_group_kernel(const __grid_constant__ GroupParams g) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    int i = 0;
+    while (i + 1 < g.count && (int)blockIdx.x >= g.cta0[i + 1]) ++i;
+    const int cta = blockIdx.x - g.cta0[i], ncta = g.cta0[i + 1] - g.cta0[i];
+    if (g.lpr[i] == 32)
+        gemv_small_body<32, MT, R, XM>(g.prob[i], cta, ncta, smem);
+    else if (g.lpr[i] == 16)
+        gemv_small_body<16, MT, R, XM>(g.prob[i], cta, ncta, smem);
+    else
+        gemv_small_body<8, MT, R, XM>(g.prob[i], cta, ncta, smem);
+}
+
 // ------------------------------------------------------------ 4 < M <= 64
 
 template <int MT>
@@ -485,7 +517,7 @@ __global__ void __launch_bounds__((GEMV_MT_CWARPS + 1) * 32, 1) gemv_mt_kernel(c
     unsigned char* ring = smem + GEMV_HDR;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int r0, nrows;
-    cta_rows(p, r0, nrows);
+    cta_rows(p, blockIdx.x, gridDim.x, r0, nrows);
     init_barriers(p, sh);
     pdl_launch_dependents();
     if (warp == GEMV_MT_CWARPS) {
@@ -570,6 +602,7 @@ cudaError_t launch_with_smem(KernelT kernel, int grid, int threads, size_t smem,
 }
 
 using GemvKernel = void (*)(const GemvParams);
+using GroupKernel = void (*)(const GroupParams);
 
 template <int LPR, int XM>
 GemvKernel small_kernel_for(int mt, int r) {
@@ -606,69 +639,87 @@ void ring_geometry(GemvParams& p, int rows_per_cta, int ring_bytes) {
 
 int small_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
 
-cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st) {
-    const int M = p.M, K = p.K, N = p.N;
+struct SmallShape {
+    int lpr, r, cwarps, grid;
+    size_t smem;
+};
+
+// Launch shape and ring geometry of the small kernel for problem p when
+// `co_resident` CTAs share an SM (sets the ring fields of p).
+SmallShape configure_small(GemvParams& p, const DevInfo& dev, int co_resident) {
+    const int K = p.K, N = p.N;
     const int grid = std::max(1, std::min(N, dev.num_sms));
     const int rows_per_cta = (N + grid - 1) / grid;
-    const int max_dyn = dev.max_smem_optin;
     const int K4 = K / 64;
+    const int mt = small_mt(p.M);
+    // Launch shape (measured on B200 over lanes-per-row x rows-per-team x
+    // K-slices x warps for the 4096x11008 and 11008x4096 decode shapes):
+    // about ten consumer warps, two rows per team (one when M > 2), and the
+    // widest team for which every row of the CTA still fits one pass.
+    const int cw_target = 10;
+    int r = std::max(1, 2 / mt);
+    const int teams_needed = (rows_per_cta + r - 1) / r;
+    int lpr = 8;
+    for (int l : {32, 16, 8}) {
+        if (teams_needed * l <= cw_target * 32) {
+            lpr = l;
+            break;
+        }
+    }
+    int ks = 1;
+    if (rows_per_cta <= GEMV_KS_MAX_ROWS && lpr == 32 && (cw_target * 32 / lpr) * r >= 2 * rows_per_cta)
+        ks = 2;  // few rows: split K so every warp has work
+    p.ks = ks;
+    p.slice4 = (K4 + ks - 1) / ks;
+    const int items = (rows_per_cta + r - 1) / r * ks;
+    int cwarps = std::max(1, std::min(cw_target, (items * lpr + 31) / 32));
+    p.xq_bytes = (mt * K + 127) / 128 * 128;
+    // leave room for the other CTAs on the same SM
+    const int budget = (dev.max_smem_optin - 1024) / co_resident;
+    const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * (K / 4));
+    ring_geometry(p, rows_per_cta, ring_bytes);
+    if (p.reuse) {
+        // one team per warp, and the rows of one iteration (ceil(teams / ks) * r)
+        // within (stages - 1) * rpc so that they never wrap onto a slot twice
+        const int window = std::max(1, (p.stages - 1) * p.rpc);
+        lpr = 32;
+        r = std::min(r, window);
+        while (r > 1 && (r & (r - 1))) --r;  // keep r in {1, 2, 4}
+        const int teams_max = std::max(1, window / r * ks);
+        cwarps = std::max(1, std::min(cwarps, teams_max));
+        // teams per iteration a multiple (or divisor) of ks: iterations then
+        // start on row-group boundaries
+        if (cwarps >= ks)
+            cwarps = cwarps / ks * ks;
+        else
+            while (ks % cwarps) --cwarps;
+    }
+    SmallShape sh;
+    sh.lpr = lpr;
+    sh.r = r;
+    sh.cwarps = cwarps;
+    sh.grid = grid;
+    sh.smem = GEMV_HDR + p.xq_bytes + (size_t)p.stages * p.stage_stride;
+    return sh;
+}
 
-    const int mt = small_mt(M);
-    if (M <= GEMV_SMALL_MAX_M && mt * K <= GEMV_XQ_SMEM_MAX) {
-        // Launch shape (measured on B200 over lanes-per-row x rows-per-team x
-        // K-slices x warps for the 4096x11008 and 11008x4096 decode shapes):
-        // about ten consumer warps, two rows per team (one when M > 2), and the
-        // widest team for which every row of the CTA still fits one pass.
-        const int cw_target = 10;
-        int r = std::max(1, 2 / mt);
-        const int teams_needed = (rows_per_cta + r - 1) / r;
-        int lpr = 8;
-        for (int l : {32, 16, 8}) {
-            if (teams_needed * l <= cw_target * 32) {
-                lpr = l;
-                break;
-            }
-        }
-        int ks = 1;
-        if (rows_per_cta <= GEMV_KS_MAX_ROWS && lpr == 32 && (cw_target * 32 / lpr) * r >= 2 * rows_per_cta)
-            ks = 2;  // few rows: split K so every warp has work
-        p.ks = ks;
-        p.slice4 = (K4 + ks - 1) / ks;
-        const int items = (rows_per_cta + r - 1) / r * ks;
-        int cwarps = std::max(1, std::min(cw_target, (items * lpr + 31) / 32));
-        p.xq_bytes = (mt * K + 127) / 128 * 128;
-        // leave room for the next launch's CTA on the same SM
-        const int budget = (max_dyn - 1024) / GEMV_CO_RESIDENT;
-        const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * (K / 4));
-        ring_geometry(p, rows_per_cta, ring_bytes);
-        if (p.reuse) {
-            // one team per warp, and the rows of one iteration (ceil(teams / ks) * r)
-            // within (stages - 1) * rpc so that they never wrap onto a slot twice
-            const int window = std::max(1, (p.stages - 1) * p.rpc);
-            if (lpr != 32) {
-                lpr = 32;
-                p.slice4 = (K4 + ks - 1) / ks;
-            }
-            r = std::min(r, window);
-            while (r > 1 && (r & (r - 1))) --r;  // keep r in {1, 2, 4}
-            const int teams_max = std::max(1, window / r * ks);
-            cwarps = std::max(1, std::min(cwarps, teams_max));
-            // teams per iteration a multiple (or divisor) of ks: iterations then
-            // start on row-group boundaries
-            if (cwarps >= ks)
-                cwarps = cwarps / ks * ks;
-            else
-                while (ks % cwarps) --cwarps;
-        }
-        const size_t smem = GEMV_HDR + p.xq_bytes + (size_t)p.stages * p.stage_stride;
-        GemvKernel k = p.x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED>(lpr, mt, r)
-                       : p.x_mode == X_F32     ? small_kernel_for<X_F32>(lpr, mt, r)
-                                               : small_kernel_for<X_BF16>(lpr, mt, r);
-        return launch_with_smem(k, grid, (cwarps + 1) * 32, smem, st, p);
+bool small_ok(int M, int K) { return M <= GEMV_SMALL_MAX_M && small_mt(M) * K <= GEMV_XQ_SMEM_MAX; }
+
+cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st) {
+    const int M = p.M, N = p.N;
+    if (small_ok(M, p.K)) {
+        const SmallShape sh = configure_small(p, dev, GEMV_CO_RESIDENT);
+        const int mt = small_mt(M);
+        GemvKernel k = p.x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED>(sh.lpr, mt, sh.r)
+                       : p.x_mode == X_F32     ? small_kernel_for<X_F32>(sh.lpr, mt, sh.r)
+                                               : small_kernel_for<X_BF16>(sh.lpr, mt, sh.r);
+        return launch_with_smem(k, sh.grid, (sh.cwarps + 1) * 32, sh.smem, st, p);
     }
     if (p.x_mode != X_QUANTISED) return cudaErrorInvalidValue;  // callers quantise first
+    const int grid = std::max(1, std::min(N, dev.num_sms));
+    const int rows_per_cta = (N + grid - 1) / grid;
     p.xq_bytes = 0;
-    ring_geometry(p, rows_per_cta, max_dyn - GEMV_HDR);
+    ring_geometry(p, rows_per_cta, dev.max_smem_optin - GEMV_HDR);
     p.wave = p.reuse ? std::max(1, std::min(GEMV_MT_CWARPS, (p.stages - 1) * p.rpc)) : GEMV_MT_CWARPS;
     const size_t smem = GEMV_HDR + (size_t)p.stages * p.stage_stride;
     const int threads = (GEMV_MT_CWARPS + 1) * 32;
@@ -676,6 +727,13 @@ cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st)
     if (M <= 2) return launch_with_smem(gemv_mt_kernel<2>, grid, threads, smem, st, p);
     if (M <= 4) return launch_with_smem(gemv_mt_kernel<4>, grid, threads, smem, st, p);
     return launch_with_smem(gemv_mt_kernel<8>, grid, threads, smem, st, p);
+}
+
+template <int XM>
+GroupKernel group_kernel_for(int mt) {
+    if (mt == 1) return gemv_group_kernel<1, 2, XM>;
+    if (mt == 2) return gemv_group_kernel<2, 1, XM>;
+    return gemv_group_kernel<4, 1, XM>;
 }
 
 GemvParams make_params(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
@@ -704,6 +762,48 @@ cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, con
 
 bool gemv_fused_quant_ok(long long M, long long K) {
     return M <= GEMV_SMALL_MAX_M && small_mt((int)M) * K <= GEMV_XQ_SMEM_MAX;
+}
+
+int gemv_group_max() { return GEMV_GROUP_MAX; }
+
+cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
+                                    const DevInfo& dev, cudaStream_t st) {
+    // x_dtype: 0 fp32, 1 bf16 (quantiser fused), 2 int8 x_q with gamma
+    const int xm = x_dtype == 2 ? X_QUANTISED : x_dtype == 1 ? X_BF16 : X_F32;
+    if (count < 1 || count > GEMV_GROUP_MAX) return cudaErrorInvalidValue;
+    GroupParams g = {};
+    g.count = count;
+    int threads = 32;
+    size_t smem = 0;
+    int cta = 0;
+    for (int i = 0; i < count; ++i) {
+        const GemvProblem& q = probs[i];
+        if (!small_ok(M, q.K)) return cudaErrorInvalidValue;
+        GemvParams p = make_params(nullptr, nullptr, M, q.K, q.W_p, q.beta, q.N, q.y, mode);
+        if (xm == X_QUANTISED) {
+            p.x_q = static_cast<const int8_t*>(q.x);
+            p.gamma = q.gamma;
+        } else {
+            p.x = q.x;
+        }
+        p.x_mode = xm;
+        // the problems of the group share each SM (one CTA each)
+        const SmallShape sh = configure_small(p, dev, count);
+        g.prob[i] = p;
+        g.lpr[i] = sh.lpr;
+        g.cta0[i] = cta;
+        cta += sh.grid;
+        threads = std::max(threads, (sh.cwarps + 1) * 32);
+        smem = std::max(smem, sh.smem);
+    }
+    g.cta0[count] = cta;
+    const int mt = small_mt(M);
+    GroupKernel k = xm == X_QUANTISED ? group_kernel_for<X_QUANTISED>(mt)
+                    : xm == X_BF16    ? group_kernel_for<X_BF16>(mt)
+                                      : group_kernel_for<X_F32>(mt);
+    cudaError_t e = ensure_smem_optin(reinterpret_cast<const void*>(k), smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k, dim3(cta), dim3(threads), smem, st, g);
 }
 
 cudaError_t launch_gemv_fused(const void* x, bool bf16, int M, int K, const uint32_t* W_p, const float* beta, int N,

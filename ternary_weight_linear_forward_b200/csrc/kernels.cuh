@@ -41,6 +41,18 @@ bool gemv_fused_quant_ok(long long M, long long K);
 cudaError_t launch_gemv_fused(const void* x, bool bf16, int M, int K, const uint32_t* W_p, const float* beta, int N,
                               void* y, YMode mode, const DevInfo& dev, cudaStream_t st);
 
+struct GemvProblem {
+    const void* x;
+    const float* gamma;  // x is x_q when non-null
+    const uint32_t* W_p;
+    const float* beta;
+    void* y;
+    int K, N;
+};
+int gemv_group_max();
+cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
+                                    const DevInfo& dev, cudaStream_t st);
+
 // k_gemm.cu  (M > 64, tcgen05 int8 tensor cores)
 size_t gemm_ws_bytes(long long M, long long N, long long K);
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,

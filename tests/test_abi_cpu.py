@@ -140,3 +140,29 @@ def test_binding_type_checks():
         bl.quant_act(torch.zeros(2, 64, dtype=torch.float16))
     with pytest.raises((TypeError, ValueError)):
         bl.pack(torch.zeros(2, 64, dtype=torch.int8))       # CPU tensor
+
+
+class _Prob(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("W_p", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("y", ctypes.c_void_p), ("K", ctypes.c_int64), ("N", ctypes.c_int64)]
+
+
+def test_forward_fp_batch_validation():
+    f = _L().bitlinear_forward_fp_batch
+    arr = (_Prob * 9)()
+    for i in range(9):
+        arr[i] = _Prob(A1, None, A2, A3, A4 + i * 0x100000, 1024, 64)
+    pa = ctypes.cast(arr, ctypes.c_void_p)
+    assert f(None, 1, 1, 0, 0, None) == NULL
+    assert f(pa, 0, 1, 0, 0, None) == SHAPE
+    assert f(pa, 9, 1, 0, 0, None) == SHAPE
+    assert f(pa, 2, 5, 0, 0, None) == SHAPE           # M > 4
+    assert f(pa, 2, 1, 3, 0, None) == DTYPE
+    assert f(pa, 2, 1, 2, 0, None) == NULL            # int8 x needs gamma
+    arr[1].y = A4                                      # two outputs overlap
+    assert f(pa, 2, 1, 0, 0, None) == ALIAS
+    arr[1].y = A4 + 0x100000
+    arr[1].K = 1000
+    assert f(pa, 2, 1, 0, 0, None) == SHAPE
+    arr[1].K = 1024
+    assert f(pa, 2, 1, 0, 0, None) == DEVICE

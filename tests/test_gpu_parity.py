@@ -333,3 +333,60 @@ def test_workload_prefill_sampled_rows(dev, shape):
     # full-size prefill (M = 2048) in the launch configuration the benchmark
     # times; the oracle checks a sample of whole output rows
     _sampled_rows_check(dev, shape)
+
+
+# --------------------------------------------------------------------------
+# batched independent projections in one launch
+# --------------------------------------------------------------------------
+
+def _prep_batch(dev, shapes, M, x_dtype, seed):
+    probs, refs = [], []
+    for i, (K, N) in enumerate(shapes):
+        W = workloads.latent_weights(seed + i, N, K)
+        x = workloads.activations(seed + 50 + i, M, K, outliers=True)
+        if x_dtype == "bf16":
+            bits = workloads.bf16_bits(x)
+            xt = T(bits.view(np.int16), dev).view(torch.bfloat16)
+            x = workloads.bf16_to_f32(bits)
+        else:
+            xt = T(x, dev)
+        W_t, beta, W_p = gpu_prep(W, dev)
+        probs.append({"x": xt, "W_p": W_p, "beta": beta})
+        oW_t, obeta = oracle.quantize_weights(W)
+        refs.append(oracle.forward(x, oW_t, obeta))
+    return probs, refs
+
+
+@pytest.mark.parametrize("M,x_dtype,shapes", [
+    (1, "bf16", [(4096, 11008), (11008, 4096)]),
+    (1, "f32", [(2560, 2560), (2560, 2560), (2560, 2560)]),
+    (2, "f32", [(1024, 300), (6912, 149), (64, 5)]),
+    (4, "bf16", [(4096, 1000), (2560, 777)]),
+    (1, "f32", [(1024, 1024)]),
+    (3, "f32", [(128, 7), (256, 9), (512, 11), (1024, 13), (2048, 17), (4096, 19), (8192, 23), (16384, 29)]),
+])
+def test_forward_fp_batch_matches_single_calls(dev, M, x_dtype, shapes):
+    probs, refs = _prep_batch(dev, shapes, M, x_dtype, seed=M * 100 + len(shapes))
+    outs = bl.forward_fp_batch(probs)
+    for pr, out, ref in zip(probs, outs, refs):
+        single = bl.forward_fp(pr["x"], pr["W_p"], pr["beta"])
+        np.testing.assert_array_equal(out.cpu().numpy(), single.cpu().numpy())
+        assert_f32_close(out.cpu().numpy(), ref["y64"])
+    # bf16 outputs
+    outs = bl.forward_fp_batch(probs, out_dtype=torch.bfloat16)
+    for out, ref in zip(outs, refs):
+        assert_bf16_ok(out.cpu().view(torch.int16).numpy().view(np.uint16), ref["y64"])
+
+
+def test_forward_fp_batch_quantised_inputs(dev):
+    # q / k / v style: one x_q shared by three projections
+    K = 2560
+    x = workloads.activations(77, 1, K)
+    x_q, gamma = bl.quant_act(T(x, dev))
+    probs = []
+    for i, N in enumerate((2560, 2560, 1280)):
+        W_t, beta, W_p = gpu_prep(workloads.latent_weights(80 + i, N, K), dev)
+        probs.append({"x": x_q, "gamma": gamma, "W_p": W_p, "beta": beta})
+    outs = bl.forward_fp_batch(probs)
+    for pr, out in zip(probs, outs):
+        np.testing.assert_array_equal(out.cpu().numpy(), bl.forward(x_q, gamma, pr["W_p"], pr["beta"]).cpu().numpy())
