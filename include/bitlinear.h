@@ -140,9 +140,9 @@ size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K);
  *         layout), beta [1] float32 -- all inputs
  *   y     [M, N] float32 or bfloat16 out
  *   ws    >= bitlinear_forward_workspace(M, N, K) bytes (may be NULL when that is 0)
- * K % 64 == 0, K <= BL_MAX_K.  M <= 64 runs the decode GEMV (CUDA cores);
- * larger M runs the prefill GEMM (tcgen05 int8 tensor cores).  Both give
- * identical results.
+ * K % 64 == 0, K <= BL_MAX_K.  M <= 64 runs a decode kernel (see
+ * bitlinear_set_decode_engine); larger M runs the prefill GEMM (tcgen05 int8
+ * tensor cores).  All give identical results.
  */
 bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
                             const uint32_t* W_p, const float* beta, int64_t N,
@@ -258,6 +258,34 @@ enum { BL_COMBINE_NONE = 0, BL_COMBINE_ADD = 1, BL_COMBINE_SILU_MUL = 2 };
  */
 bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, int64_t M, int64_t K,
                                   float* h, int8_t* x_q, float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode engine                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Engines for the decode forward (M <= 64 tokens). */
+enum {
+    BL_ENGINE_AUTO = 0,          /* the library picks per shape (default): CUDA cores for
+                                    M <= 4, tensor cores for 5 <= M <= 16 where they fit */
+    BL_ENGINE_CUDA_CORES = 1,    /* add / sub / skip as masked byte dot products on CUDA cores */
+    BL_ENGINE_TENSOR_CORES = 2   /* codes expanded to bytes, contraction on tcgen05 (M <= 16) */
+};
+
+/*
+ * Selects the decode engine of every later forward call in this process
+ * (bitlinear_forward, _fp, _fp_batch, _acc, _noalloc with M <= 64).  Both
+ * engines compute the same integers and the same floats, bit for bit; the
+ * choice only changes speed.  Shapes the tensor-core engine does not take
+ * (M > 16, or x_hat of all tokens larger than its shared-memory budget) run on
+ * CUDA cores whatever the setting.  Not a feature of the pages: an
+ * implementation switch, used by tests to check both engines.  Returns
+ * BL_ERR_SHAPE for an unknown engine.  Takes effect for calls made after it
+ * returns; not synchronised with calls made concurrently from other threads.
+ */
+bl_status bitlinear_set_decode_engine(int engine);
+
+/* The engine last set (BL_ENGINE_AUTO initially). */
+int bitlinear_get_decode_engine(void);
 
 /* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */

@@ -9,6 +9,7 @@ if the shared library is missing or no sm_100 device is present, calls fail.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -40,6 +41,8 @@ SIGNATURES = {
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_set_decode_engine": (_I, [_I]),
+    "bitlinear_get_decode_engine": (_I, []),
     "bitlinear_device_status": (_I, [_P]),
     "bitlinear_num_sms": (_I, []),
 }
@@ -310,6 +313,32 @@ def quant_act_rms(a: torch.Tensor, b: torch.Tensor | None = None, combine: str =
            lib().bitlinear_quant_act_rms(_ptr(a), _ptr(b), COMBINE[combine], M, K, _ptr(h), _ptr(x_q),
                                          _ptr(gamma), _stream(stream)))
     return h, x_q, gamma
+
+
+ENGINES = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
+
+
+def set_decode_engine(name: str):
+    """Engine of later decode calls (M <= 64): 'auto', 'cuda_cores' or 'tensor_cores'."""
+    if name not in ENGINES:
+        raise ValueError(f"unknown decode engine {name!r}")
+    _check("bitlinear_set_decode_engine", lib().bitlinear_set_decode_engine(ENGINES[name]))
+
+
+def get_decode_engine() -> str:
+    v = int(lib().bitlinear_get_decode_engine())
+    return {i: n for n, i in ENGINES.items()}[v]
+
+
+@contextlib.contextmanager
+def decode_engine(name: str):
+    """Run the enclosed calls with the given decode engine, then restore the previous one."""
+    prev = get_decode_engine()
+    set_decode_engine(name)
+    try:
+        yield
+    finally:
+        set_decode_engine(prev)
 
 
 def device_status(stream=None):

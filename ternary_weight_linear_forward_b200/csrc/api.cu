@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" boundary of libbitlinear: host-side validation,
 // device checks and dispatch.  Every entry point is declared, with its
 // defining passage, in include/bitlinear.h.
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -82,6 +83,23 @@ bl_status check_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_
 
 constexpr int GEMV_MAX_M = 64;
 
+std::atomic<int> g_engine{BL_ENGINE_AUTO};
+
+// Tensor-core decode for this problem set?  Automatic choice (measured on
+// B200): a kind::i8 MMA costs the same ~186 cycles for any N <= 256, so with
+// few tokens dp4a on CUDA cores streams weights faster (M <= 4); beyond that
+// the CUDA-core engine's multi-token kernel is the slower one.
+constexpr int AUTO_TC_MIN_M = 5;
+
+bool use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
+    const int engine = g_engine.load(std::memory_order_relaxed);
+    if (engine == BL_ENGINE_CUDA_CORES || M > decode_tc_max_m()) return false;
+    if (engine == BL_ENGINE_AUTO && M < AUTO_TC_MIN_M) return false;
+    for (int i = 0; i < count; ++i)
+        if (!decode_tc_supported(M, probs[i].K, probs[i].N, count, dev)) return false;
+    return true;
+}
+
 bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
                       const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes, void* stream) {
     const size_t need = bitlinear_forward_workspace(M, N, K);
@@ -91,7 +109,10 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
     bl_status s = current_device(dev);
     if (s) return s;
     cudaError_t e;
-    if (M <= GEMV_MAX_M)
+    const GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
+    if (M <= GEMV_MAX_M && use_tc((int)M, &prob, 1, dev))
+        e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
+    else if (M <= GEMV_MAX_M)
         e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
@@ -99,6 +120,10 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
 }
 
 }  // namespace
+
+bool decode_use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
+    return use_tc(M, probs, count, dev);
+}
 
 cudaError_t ensure_smem_optin(const void* kernel, size_t bytes) {
     static std::mutex mu;
@@ -245,6 +270,9 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
     s = current_device(dev);
     if (s) return s;
     const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
+    const GemvProblem prob = {x, nullptr, W_p, beta, y, (int)K, (int)N};
+    if (M <= GEMV_MAX_M && use_tc((int)M, &prob, 1, dev))  // quantiser fused, workspace unused
+        return from_cuda(launch_decode_tc(&prob, 1, (int)M, x_dtype, mode, dev, as_stream(stream)));
     if (!need)
         return from_cuda(launch_gemv_fused(x, x_dtype == BL_BF16, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev,
                                            as_stream(stream)));
@@ -291,8 +319,10 @@ bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int6
     DevInfo dev;
     bl_status s = current_device(dev);
     if (s) return s;
-    return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype,
-                                             y_dtype == BL_F32 ? Y_F32 : Y_BF16, dev, as_stream(stream)));
+    const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
+    if (use_tc((int)M, probs, count, dev))
+        return from_cuda(launch_decode_tc(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
+    return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
 }
 
 bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,
@@ -344,6 +374,15 @@ bl_status bitlinear_device_status(void* stream) {
     }
     return BL_OK;
 }
+
+bl_status bitlinear_set_decode_engine(int engine) {
+    if (engine != BL_ENGINE_AUTO && engine != BL_ENGINE_CUDA_CORES && engine != BL_ENGINE_TENSOR_CORES)
+        return BL_ERR_SHAPE;
+    g_engine.store(engine, std::memory_order_relaxed);
+    return BL_OK;
+}
+
+int bitlinear_get_decode_engine(void) { return g_engine.load(std::memory_order_relaxed); }
 
 int bitlinear_num_sms(void) {
     DevInfo dev;

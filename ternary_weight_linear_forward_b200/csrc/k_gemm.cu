@@ -305,11 +305,9 @@ done:
 
 // ------------------------------------------------------------------- host
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-EncodeTiled encode_fn() {
+EncodeTiled tensor_map_encoder() {
     static EncodeTiled fn = nullptr;
     static std::once_flag once;
     std::call_once(once, []() {
@@ -322,8 +320,6 @@ EncodeTiled encode_fn() {
     return fn;
 }
 
-}  // namespace
-
 size_t gemm_ws_bytes(long long M, long long N, long long K) {
     (void)N;
     (void)K;
@@ -332,7 +328,7 @@ size_t gemm_ws_bytes(long long M, long long N, long long K) {
 
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
                         int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st) {
-    EncodeTiled enc = encode_fn();
+    EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     if (dev.max_smem_optin < GEMM_SMEM) return cudaErrorNotSupported;
     CUtensorMap ta, tb;

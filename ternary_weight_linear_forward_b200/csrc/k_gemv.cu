@@ -28,6 +28,7 @@
 //     so a decode layer is a single kernel;
 //   * 4 < M <= 64 ("mt" kernel): one warp per row, activations read through
 //     L1 from global memory, MT tokens per pass.
+#include "act_inl.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -46,8 +47,6 @@ constexpr int GEMV_MT_CWARPS = 8;  // consumer warps of the mt kernel
 constexpr int GEMV_CHUNK_TARGET = 8192;
 constexpr int GEMV_XQ_SMEM_MAX = 64 * 1024;
 constexpr int GEMV_SMALL_MAX_M = 4;
-
-enum XMode : int { X_QUANTISED = 0, X_F32 = 1, X_BF16 = 2 };
 
 struct GemvParams {
     const void* x;  // fp32/bf16 activations when the quantiser is fused
@@ -183,41 +182,6 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 // 16-byte chunk c of a token's x_q row is stored at slot c ^ ((c >> 3) & 3):
 // lane l of a team reads chunks 4l + q, which this maps to distinct bank groups.
 __device__ __forceinline__ int xq_slot(int c) { return c ^ ((c >> 3) & 3); }
-
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-    return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
-           ((uint32_t)(d & 0xFF) << 24);
-}
-
-// same rounding as the standalone quantiser: rint(x * s), clamp to [-127, 127]
-__device__ __forceinline__ int q8(float v, float s) {
-    int r = __float2int_rn(__fmul_rn(v, s));
-    return min(max(r, -127), 127);
-}
-
-template <int MODE>  // X_F32 or X_BF16
-__device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
-    if (MODE == X_BF16) {
-        const uint4* pp = reinterpret_cast<const uint4*>(row) + 2 * g;
-        uint4 a = __ldg(pp), b = __ldg(pp + 1);
-        uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            v[2 * i] = __uint_as_float(w[i] << 16);
-            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-    } else {
-        const float4* pp = reinterpret_cast<const float4*>(row) + 4 * g;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float4 f = __ldg(pp + i);
-            v[4 * i] = f.x;
-            v[4 * i + 1] = f.y;
-            v[4 * i + 2] = f.z;
-            v[4 * i + 3] = f.w;
-        }
-    }
-}
 
 // Fill the shared x_q rows (tokens 0..MT-1; tokens >= M are zero), rowsum[]
 // and fscale[].  Runs on the consumer threads only.

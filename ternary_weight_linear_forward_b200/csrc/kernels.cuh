@@ -53,6 +53,14 @@ int gemv_group_max();
 cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
                                     const DevInfo& dev, cudaStream_t st);
 
+// k_decode_tc.cu  (M <= 16, tcgen05 int8 tensor cores)
+int decode_tc_max_m();
+bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev);
+cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode, const DevInfo& dev,
+                             cudaStream_t st);
+// api.cu: the process-wide engine choice applied to a decode problem set
+bool decode_use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev);
+
 // k_gemm.cu  (M > 64, tcgen05 int8 tensor cores)
 size_t gemm_ws_bytes(long long M, long long N, long long K);
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,

@@ -97,7 +97,10 @@ extern "C" bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* g
     const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (M <= NOALLOC_GEMV_MAX_M)
+    const GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
+    if (M <= NOALLOC_GEMV_MAX_M && decode_use_tc((int)M, &prob, 1, d->info))
+        e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, d->info, st);
+    else if (M <= NOALLOC_GEMV_MAX_M)
         e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->info, st);
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->scratch, d->info, st);

@@ -134,6 +134,19 @@ def test_device_queries_without_gpu():
     assert _L().bitlinear_device_status(None) == DEVICE
 
 
+def test_decode_engine_switch():
+    L_ = _L()
+    assert L_.bitlinear_get_decode_engine() == 0           # BL_ENGINE_AUTO initially
+    assert L_.bitlinear_set_decode_engine(3) == SHAPE
+    assert L_.bitlinear_set_decode_engine(-1) == SHAPE
+    for name in ("cuda_cores", "tensor_cores", "auto"):
+        with bl.decode_engine(name):
+            assert bl.get_decode_engine() == name
+    assert bl.get_decode_engine() == "auto"
+    with pytest.raises(ValueError):
+        bl.set_decode_engine("fpga")
+
+
 def test_binding_type_checks():
     import torch
     with pytest.raises(TypeError):

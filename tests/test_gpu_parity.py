@@ -163,10 +163,13 @@ def run_case(dev, M, K, N, seed, x_dtype="f32", y_dtype="f32", outliers=False):
     return ref
 
 
+@pytest.mark.parametrize("engine", ["cuda_cores", "tensor_cores"])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 16, 33, 64])
 @pytest.mark.parametrize("K,N", [(64, 5), (1024, 148), (1024, 149), (2560, 1000), (6912, 300)])
-def test_gemv_parity_sweep(dev, M, K, N):
-    run_case(dev, M, K, N, seed=10 * M + K % 97 + N)
+def test_gemv_parity_sweep(dev, M, K, N, engine):
+    # shapes the tensor-core engine does not take run on CUDA cores
+    with bl.decode_engine(engine):
+        run_case(dev, M, K, N, seed=10 * M + K % 97 + N)
 
 
 @pytest.mark.parametrize("K", [64, 128, 1024, 1088, 2048, 2560, 4096, 6912, 11008, 16384, 16448, 32768])
