@@ -140,9 +140,18 @@ size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K);
  *         layout), beta [1] float32 -- all inputs
  *   y     [M, N] float32 or bfloat16 out
  *   ws    >= bitlinear_forward_workspace(M, N, K) bytes (may be NULL when that is 0)
- * K % 64 == 0, K <= BL_MAX_K.  M <= 64 runs a decode kernel (see
- * bitlinear_set_decode_engine); larger M runs the prefill GEMM (tcgen05 int8
- * tensor cores).  All give identical results.
+ * K % 64 == 0, K <= BL_MAX_K.  By default M <= 4 runs the decode GEMV on
+ * CUDA cores, 5 <= M <= 16 a decode kernel on the tcgen05 int8 tensor cores
+ * (where x_hat fits its shared memory) and larger M the GEMM on the tensor
+ * cores (bitlinear_set_decode_engine selects other kernels for M <= 64).  All
+ * give identical results.
+ *
+ * The forward kernels begin streaming W_p and read beta before the kernel
+ * queued ahead of them on the stream has finished (programmatic dependent
+ * launch); x_q and gamma are read only after it finished.  W_p and beta must
+ * therefore not be written by a kernel that is still running when the
+ * forward is launched: kernels without programmatic dependent launch, this
+ * library's own included, always finish first.
  */
 bl_status bitlinear_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
                             const uint32_t* W_p, const float* beta, int64_t N,
@@ -212,10 +221,10 @@ bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K,
  * or code being recorded into a stream capture where an allocation is not
  * allowed.  The pages have no counterpart: this is a library convenience.
  * Same arguments, kernels, dispatch and results as bitlinear_forward, without
- * ws/ws_bytes: the M int32 row sums the prefill path (M > 64) needs live in a
+ * ws/ws_bytes: the M int32 row sums the GEMM path (M > 4) needs live in a
  * static device array of the library (BL_NOALLOC_MAX_M entries, held by every
- * device that loads the library until exit); the decode path (M <= 64) needs
- * no scratch.
+ * device that loads the library until exit); the CUDA-core and swap-AB
+ * decode kernels need no scratch.
  *   - M > BL_NOALLOC_MAX_M returns BL_ERR_WORKSPACE (scratch too small), with
  *     nothing launched.
  *   - The first call on a device looks up the array's device address and
@@ -265,19 +274,19 @@ bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, i
 
 /* Engines for the decode forward (M <= 64 tokens). */
 enum {
-    BL_ENGINE_AUTO = 0,          /* the library picks per shape (default): CUDA cores for
-                                    M <= 4, tensor cores for 5 <= M <= 16 where they fit */
-    BL_ENGINE_CUDA_CORES = 1,    /* add / sub / skip as masked byte dot products on CUDA cores */
-    BL_ENGINE_TENSOR_CORES = 2   /* codes expanded to bytes, contraction on tcgen05 (M <= 16) */
+    BL_ENGINE_AUTO = 0,          /* the library picks per shape (default): the CUDA-core GEMV
+                                    for M <= 4, the swap-AB decode kernel for 5 <= M <= 16
+                                    where it fits, the tcgen05 GEMM otherwise */
+    BL_ENGINE_CUDA_CORES = 1,    /* M <= 64 on CUDA cores (masked byte dot products) */
+    BL_ENGINE_TENSOR_CORES = 2   /* M <= 16 on the swap-AB tcgen05 decode kernel where it
+                                    fits (weight rows on the MMA's 128 lanes), else as AUTO */
 };
 
 /*
  * Selects the decode engine of every later forward call in this process
- * (bitlinear_forward, _fp, _fp_batch, _acc, _noalloc with M <= 64).  Both
- * engines compute the same integers and the same floats, bit for bit; the
- * choice only changes speed.  Shapes the tensor-core engine does not take
- * (M > 16, or x_hat of all tokens larger than its shared-memory budget) run on
- * CUDA cores whatever the setting.  Not a feature of the pages: an
+ * (bitlinear_forward, _fp, _fp_batch, _acc, _noalloc with M <= 64).  All
+ * kernels compute the same integers and the same floats, bit for bit; the
+ * choice only changes speed.  Not a feature of the pages: an
  * implementation switch, used by tests to check both engines.  Returns
  * BL_ERR_SHAPE for an unknown engine.  Takes effect for calls made after it
  * returns; not synchronised with calls made concurrently from other threads.

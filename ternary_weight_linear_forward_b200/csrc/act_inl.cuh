@@ -26,27 +26,74 @@ __device__ __forceinline__ int q8(float v, float s) {
     return min(max(r, -127), 127);
 }
 
-template <int MODE>  // X_F32 or X_BF16
-__device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
-    if (MODE == X_BF16) {
-        const uint4* pp = reinterpret_cast<const uint4*>(row) + 2 * g;
-        uint4 a = __ldg(pp), b = __ldg(pp + 1);
-        uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+// One 16-element chunk of an activation row in its storage format:
+// 4 x 16 bytes of fp32, 2 x 16 bytes of bf16 or 16 int8 codes.
+template <int XM>
+struct XChunk {
+    uint4 u[XM == X_F32 ? 4 : (XM == X_BF16 ? 2 : 1)];
+};
+
+// chunk g of `row` (read-only path)
+template <int XM>
+__device__ __forceinline__ void ld_chunk(const void* row, int g, XChunk<XM>& c) {
+    constexpr int n = XM == X_F32 ? 4 : (XM == X_BF16 ? 2 : 1);
+    const uint4* pp = reinterpret_cast<const uint4*>(row) + n * g;
+#pragma unroll
+    for (int i = 0; i < n; ++i) c.u[i] = __ldg(pp + i);
+}
+
+// the chunk's 16 values as binary32 (X_F32 or X_BF16)
+template <int XM>
+__device__ __forceinline__ void cvt_chunk(const XChunk<XM>& c, float (&v)[16]) {
+    if constexpr (XM == X_BF16) {
+        const uint32_t w[8] = {c.u[0].x, c.u[0].y, c.u[0].z, c.u[0].w, c.u[1].x, c.u[1].y, c.u[1].z, c.u[1].w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             v[2 * i] = __uint_as_float(w[i] << 16);
             v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
     } else {
-        const float4* pp = reinterpret_cast<const float4*>(row) + 4 * g;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float4 f = __ldg(pp + i);
-            v[4 * i] = f.x;
-            v[4 * i + 1] = f.y;
-            v[4 * i + 2] = f.z;
-            v[4 * i + 3] = f.w;
+            v[4 * i] = __uint_as_float(c.u[i].x);
+            v[4 * i + 1] = __uint_as_float(c.u[i].y);
+            v[4 * i + 2] = __uint_as_float(c.u[i].z);
+            v[4 * i + 3] = __uint_as_float(c.u[i].w);
         }
+    }
+}
+
+template <int MODE>  // X_F32 or X_BF16
+__device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
+    XChunk<MODE> c;
+    ld_chunk<MODE>(row, g, c);
+    cvt_chunk<MODE>(c, v);
+}
+
+// max |v| over the chunk, as the bit pattern of a non-negative float
+template <int XM>
+__device__ __forceinline__ unsigned chunk_absmax(const XChunk<XM>& c, unsigned a) {
+    float v[16];
+    cvt_chunk<XM>(c, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = max(a, __float_as_uint(fabsf(v[i])));
+    return a;
+}
+
+// the chunk's 16 int8 codes (quantised with scale s unless already int8)
+template <int XM>
+__device__ __forceinline__ int4 chunk_codes(const XChunk<XM>& c, float s) {
+    if constexpr (XM == X_QUANTISED) {
+        return make_int4((int)c.u[0].x, (int)c.u[0].y, (int)c.u[0].z, (int)c.u[0].w);
+    } else {
+        float v[16];
+        cvt_chunk<XM>(c, v);
+        int4 q;
+        q.x = (int)pack4(q8(v[0], s), q8(v[1], s), q8(v[2], s), q8(v[3], s));
+        q.y = (int)pack4(q8(v[4], s), q8(v[5], s), q8(v[6], s), q8(v[7], s));
+        q.z = (int)pack4(q8(v[8], s), q8(v[9], s), q8(v[10], s), q8(v[11], s));
+        q.w = (int)pack4(q8(v[12], s), q8(v[13], s), q8(v[14], s), q8(v[15], s));
+        return q;
     }
 }
 

@@ -85,19 +85,26 @@ constexpr int GEMV_MAX_M = 64;
 
 std::atomic<int> g_engine{BL_ENGINE_AUTO};
 
-// Tensor-core decode for this problem set?  Automatic choice (measured on
-// B200): a kind::i8 MMA costs the same ~186 cycles for any N <= 256, so with
-// few tokens dp4a on CUDA cores streams weights faster (M <= 4); beyond that
-// the CUDA-core engine's multi-token kernel is the slower one.
-constexpr int AUTO_TC_MIN_M = 5;
+// Which kernel runs a problem set of M tokens.  Measured on B200 (4096 x 4096
+// and 4096 x 11008, x_q given): a kind::i8 tcgen05 MMA costs about the same
+// ~186 cycles for any N <= 256, so with few tokens dp4a on CUDA cores streams
+// the weights fastest (M <= 4); for 5 <= M <= 16 the swap-AB decode kernel
+// (7.8-22 us) beats the GEMM (~21 us, one 128-row tile and a row-sum launch)
+// and the CUDA cores (17-105 us); beyond that the GEMM wins (M = 64: 23-26 us
+// against 193-482 us on CUDA cores).
+constexpr int AUTO_CUDA_MAX_M = 4;
 
-bool use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
+DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
+    if (M > GEMV_MAX_M) return PATH_GEMM;
     const int engine = g_engine.load(std::memory_order_relaxed);
-    if (engine == BL_ENGINE_CUDA_CORES || M > decode_tc_max_m()) return false;
-    if (engine == BL_ENGINE_AUTO && M < AUTO_TC_MIN_M) return false;
-    for (int i = 0; i < count; ++i)
-        if (!decode_tc_supported(M, probs[i].K, probs[i].N, count, dev)) return false;
-    return true;
+    if (engine == BL_ENGINE_CUDA_CORES) return PATH_CUDA;
+    const bool tc_first = engine == BL_ENGINE_TENSOR_CORES || M > AUTO_CUDA_MAX_M;
+    if (tc_first && M <= decode_tc_max_m()) {
+        bool ok = true;
+        for (int i = 0; i < count; ++i) ok = ok && decode_tc_supported(M, probs[i].K, probs[i].N, count, dev);
+        if (ok) return PATH_TC;
+    }
+    return M <= AUTO_CUDA_MAX_M ? PATH_CUDA : PATH_GEMM;
 }
 
 bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
@@ -110,9 +117,10 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
     if (s) return s;
     cudaError_t e;
     const GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
-    if (M <= GEMV_MAX_M && use_tc((int)M, &prob, 1, dev))
+    const DecodePath path = pick_path((int)M, &prob, 1, dev);
+    if (path == PATH_TC)
         e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
-    else if (M <= GEMV_MAX_M)
+    else if (path == PATH_CUDA)
         e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
@@ -121,8 +129,8 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
 
 }  // namespace
 
-bool decode_use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
-    return use_tc(M, probs, count, dev);
+DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
+    return pick_path(M, probs, count, dev);
 }
 
 cudaError_t ensure_smem_optin(const void* kernel, size_t bytes) {
@@ -223,7 +231,7 @@ bl_status bitlinear_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, 
 }
 
 size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K) {
-    if (M <= GEMV_MAX_M) return 0;
+    if (M <= AUTO_CUDA_MAX_M) return 0;  // larger M may run the GEMM, which needs row sums
     return gemm_ws_bytes(M, N, K);
 }
 
@@ -271,7 +279,7 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
     if (s) return s;
     const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
     const GemvProblem prob = {x, nullptr, W_p, beta, y, (int)K, (int)N};
-    if (M <= GEMV_MAX_M && use_tc((int)M, &prob, 1, dev))  // quantiser fused, workspace unused
+    if (pick_path((int)M, &prob, 1, dev) == PATH_TC)  // quantiser fused, workspace unused
         return from_cuda(launch_decode_tc(&prob, 1, (int)M, x_dtype, mode, dev, as_stream(stream)));
     if (!need)
         return from_cuda(launch_gemv_fused(x, x_dtype == BL_BF16, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev,
@@ -320,7 +328,7 @@ bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int6
     bl_status s = current_device(dev);
     if (s) return s;
     const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
-    if (use_tc((int)M, probs, count, dev))
+    if (pick_path((int)M, probs, count, dev) == PATH_TC)
         return from_cuda(launch_decode_tc(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
     return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
 }

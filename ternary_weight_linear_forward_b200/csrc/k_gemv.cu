@@ -71,6 +71,7 @@ struct Shared {
     uint64_t full[GEMV_MAX_STAGES];
     uint64_t empty[GEMV_MAX_STAGES];
     int abort_flag;
+    float beta;  // read at CTA start (a weight input, like W_p)
     int rowsum[GEMV_MAX_M];
     float fscale[GEMV_MAX_M];
     unsigned red_u[GEMV_MAX_CWARPS][GEMV_SMALL_MAX_M];
@@ -184,36 +185,48 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 __device__ __forceinline__ int xq_slot(int c) { return c ^ ((c >> 3) & 3); }
 
 // Fill the shared x_q rows (tokens 0..MT-1; tokens >= M are zero), rowsum[]
-// and fscale[].  Runs on the consumer threads only.
+// and fscale[].  Runs on the consumer threads only.  The first XC chunks per
+// token of every thread are loaded at once into registers and serve both the
+// absmax pass and the quantisation pass, so the stage costs one memory round
+// trip (x was just written by the preceding kernel and sits in L2).
 template <int MT, int XM>
 __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& sh, int4* xsm, int ctid, int cthreads,
                                                   int cwarps) {
     const int G = p.K / 16;  // 16-byte chunks per token
     const int lane = ctid & 31, warp = ctid >> 5;
+    constexpr int XC = XM == X_F32 ? (MT <= 2 ? 2 / MT : 0) : 4 / MT;  // <= 32 registers of cache
+    constexpr int XCA = XC > 0 ? XC : 1;
+    const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : XM == X_F32 ? 4 : 1);
+    const char* xbase = XM == X_QUANTISED ? reinterpret_cast<const char*>(p.x_q) : reinterpret_cast<const char*>(p.x);
+    XChunk<XM> cache[MT][XCA];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            const int g = ctid + i * cthreads;
+            if (m < p.M && g < G) ld_chunk<XM>(xbase + (size_t)m * xrow, g, cache[m][i]);
+        }
+    }
     float s[MT];
     float gam[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) s[m] = gam[m] = 0.0f;
     if (XM != X_QUANTISED) {
         // pass 1: per-token absmax over the row (exact, order-free)
-        unsigned amax[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) amax[m] = 0u;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
+            unsigned a = 0u;
             if (m < p.M) {
-                const char* xr = reinterpret_cast<const char*>(p.x) + (long long)m * p.K * (XM == X_BF16 ? 2 : 4);
-                for (int g = ctid; g < G; g += cthreads) {
-                    float v[16];
-                    load16<XM>(xr, g, v);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) amax[m] = max(amax[m], __float_as_uint(fabsf(v[i])));
+                for (int i = 0; i < XC; ++i)
+                    if (ctid + i * cthreads < G) a = chunk_absmax<XM>(cache[m][i], a);
+                for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
+                    XChunk<XM> c;
+                    ld_chunk<XM>(xbase + (size_t)m * xrow, g, c);
+                    a = chunk_absmax<XM>(c, a);
                 }
             }
-        }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            unsigned a = __reduce_max_sync(0xffffffffu, amax[m]);
+            a = __reduce_max_sync(0xffffffffu, a);
             if (lane == 0) sh.red_u[warp][m] = a;
         }
         consumer_sync(cthreads);
@@ -229,25 +242,27 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
     // pass 2: write x_q chunks into their swizzled slots, accumulate row sums
     int rs[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) rs[m] = 0;
-#pragma unroll
     for (int m = 0; m < MT; ++m) {
+        rs[m] = 0;
         int4* dst = xsm + (size_t)m * G;
-        for (int g = ctid; g < G; g += cthreads) {
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            const int g = ctid + i * cthreads;
+            if (g < G) {
+                int4 q = make_int4(0, 0, 0, 0);
+                if (m < p.M) {
+                    q = chunk_codes<XM>(cache[m][i], s[m]);
+                    rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
+                }
+                dst[xq_slot(g)] = q;
+            }
+        }
+        for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
             int4 q = make_int4(0, 0, 0, 0);
             if (m < p.M) {
-                if (XM == X_QUANTISED) {
-                    q = __ldg(reinterpret_cast<const int4*>(p.x_q + (long long)m * p.K) + g);
-                } else {
-                    const char* xr =
-                        reinterpret_cast<const char*>(p.x) + (long long)m * p.K * (XM == X_BF16 ? 2 : 4);
-                    float v[16];
-                    load16<XM>(xr, g, v);
-                    q.x = (int)pack4(q8(v[0], s[m]), q8(v[1], s[m]), q8(v[2], s[m]), q8(v[3], s[m]));
-                    q.y = (int)pack4(q8(v[4], s[m]), q8(v[5], s[m]), q8(v[6], s[m]), q8(v[7], s[m]));
-                    q.z = (int)pack4(q8(v[8], s[m]), q8(v[9], s[m]), q8(v[10], s[m]), q8(v[11], s[m]));
-                    q.w = (int)pack4(q8(v[12], s[m]), q8(v[13], s[m]), q8(v[14], s[m]), q8(v[15], s[m]));
-                }
+                XChunk<XM> c;
+                ld_chunk<XM>(xbase + (size_t)m * xrow, g, c);
+                q = chunk_codes<XM>(c, s[m]);
                 rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
             }
             dst[xq_slot(g)] = q;
@@ -269,7 +284,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
         float f = 0.0f;
         if (p.mode != Y_ACC && m < p.M) {
             const float g = XM == X_QUANTISED ? __ldg(p.gamma + m) : gam[m];
-            f = __fdiv_rn(__fmul_rn(__ldg(p.beta), g), 127.0f);
+            f = __fdiv_rn(__fmul_rn(sh.beta, g), 127.0f);
         }
         sh.fscale[m] = f;
     }
@@ -334,6 +349,9 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
             mbar_init(&sh.empty[s], p.rpc * p.ks);  // every K slice of every row releases once
         }
         sh.abort_flag = 0;
+        // beta and W_p are weight inputs, not written by the preceding kernel:
+        // read before waiting for it
+        sh.beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         fence_mbar_init();
         produce(p, sh, ring, r0, nrows, 0, min(nchunks, p.stages));
     }

@@ -58,8 +58,10 @@ int decode_tc_max_m();
 bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev);
 cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode, const DevInfo& dev,
                              cudaStream_t st);
-// api.cu: the process-wide engine choice applied to a decode problem set
-bool decode_use_tc(int M, const GemvProblem* probs, int count, const DevInfo& dev);
+// api.cu: the kernel that runs a problem set with M tokens under the
+// process-wide engine choice
+enum DecodePath : int { PATH_CUDA = 0, PATH_TC = 1, PATH_GEMM = 2 };
+DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev);
 
 // k_gemm.cu  (M > 64, tcgen05 int8 tensor cores)
 size_t gemm_ws_bytes(long long M, long long N, long long K);

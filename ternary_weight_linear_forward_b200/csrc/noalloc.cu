@@ -71,7 +71,6 @@ bool overlap_na(const void* a, size_t na, const void* b, size_t nb) {
     return na && nb && x < y + nb && y < x + na;
 }
 
-constexpr int64_t NOALLOC_GEMV_MAX_M = 64;  // decode path: no scratch at all
 
 }  // namespace
 }  // namespace bl
@@ -98,9 +97,10 @@ extern "C" bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* g
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
     const GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
-    if (M <= NOALLOC_GEMV_MAX_M && decode_use_tc((int)M, &prob, 1, d->info))
+    const DecodePath path = decode_path((int)M, &prob, 1, d->info);
+    if (path == PATH_TC)
         e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, d->info, st);
-    else if (M <= NOALLOC_GEMV_MAX_M)
+    else if (path == PATH_CUDA)
         e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->info, st);
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->scratch, d->info, st);

@@ -310,8 +310,10 @@ def test_gemm_matches_gemv_on_same_inputs(dev):
     y_gemm = bl.forward(x_q, gamma, W_p, beta).cpu().numpy()
     for lo in (0, 64, 66):
         # slices are cloned: the ABI requires 16-byte aligned pointers
-        y_gemv = bl.forward(x_q[lo:lo + 64].clone(), gamma[lo:lo + 64].clone(), W_p, beta).cpu().numpy()
-        np.testing.assert_array_equal(y_gemm[lo:lo + 64], y_gemv)
+        for m, engine in ((64, "cuda_cores"), (64, "auto"), (4, "auto"), (16, "tensor_cores")):
+            with bl.decode_engine(engine):
+                y_gemv = bl.forward(x_q[lo:lo + m].clone(), gamma[lo:lo + m].clone(), W_p, beta).cpu().numpy()
+            np.testing.assert_array_equal(y_gemm[lo:lo + m], y_gemv)
 
 
 def _sampled_rows_check(dev, shape, n_rows=48):
