@@ -59,7 +59,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("k_gemv.cu", "common.cuh", "kernels.cuh"):
+    for name in ("k_gemv.cu", "act_inl.cuh", "common.cuh", "kernels.cuh"):
         with open(os.path.join(ROOT, "ternary_weight_linear_forward_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -409,6 +409,37 @@ def main():
         prefill["int8_peak_source"] = (f"{peak_kind} bf16_tflops {peaks['bf16_tflops']} x nominal int8/bf16 ratio "
                                        f"{INT8_OVER_BF16}")
 
+    # ---- small-batch decode (M = 4, 16, 64; K = 4096; N = 4096, 11008) ----
+    small = None
+    if not args.no_prefill:
+        small = {}
+        for s in workloads.W3.shapes:
+            W = torch.from_numpy(s.weights()).to(dev)
+            W_t, beta = bl.quantize_weights(W)
+            W_p0 = bl.pack(W_t)
+            del W, W_t
+            nc = max(2, int(4 * L2 // (W_p0.numel() * 4)) + 1)
+            W_ps = [W_p0] + [W_p0.clone() for _ in range(nc - 1)]
+            x = torch.from_numpy(s.inputs()).to(dev)
+            y = torch.empty((s.M, s.N), dtype=torch.float32, device=dev)
+            ws = torch.empty(max(1, bl.forward_fp_workspace(s.M, s.N, s.K)), dtype=torch.uint8, device=dev)
+            reps = 4 * nc
+            with torch.cuda.stream(stream):
+                for i in range(4):
+                    bl.forward_fp(x, W_ps[i % nc], beta, out=y, ws=ws, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(reps):
+                        bl.forward_fp(x, W_ps[i % nc], beta, out=y, ws=ws, stream=stream)
+            g.replay()
+            t = timed_run([g])
+            gbs = s.algorithmic_bytes * reps / t / 1e9
+            small[s.name] = {"us_per_call": t / reps * 1e6, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                             "path": "CUDA-core GEMV" if s.M <= 4 else
+                                     ("tcgen05 swap-AB decode" if s.M <= 16 else "tcgen05 GEMM")}
+            del g, W_ps, W_p0, x, y, ws
+
     # ---- decoder block at batch-1 decode (hidden 2560, intermediate 6912) ----
     block = None
     if not args.no_prefill:
@@ -456,7 +487,7 @@ def main():
                              f"({copies * packed_bytes / 1e6:.0f} MB vs L2 {L2 / 1e6:.0f} MB)",
                        "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks, "prefill": prefill, "block": block,
+            "gpu_launches": args.steps, "clocks": clocks, "prefill": prefill, "small_batch": small, "block": block,
             "device": props.name,
         }
         print(json.dumps(line), flush=True)

@@ -175,6 +175,10 @@ def forward(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: tor
     return out
 
 
+def forward_fp_workspace(M: int, N: int, K: int) -> int:
+    return int(lib().bitlinear_forward_fp_workspace(M, N, K))
+
+
 def forward_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype=torch.float32, out=None,
                ws=None, stream=None) -> torch.Tensor:
     """quant_act + forward in one call (one kernel for M <= 4); bit-identical to the two calls."""

@@ -47,6 +47,7 @@ constexpr int GEMV_MT_CWARPS = 8;  // consumer warps of the mt kernel
 constexpr int GEMV_CHUNK_TARGET = 8192;
 constexpr int GEMV_XQ_SMEM_MAX = 64 * 1024;
 constexpr int GEMV_SMALL_MAX_M = 4;
+constexpr int GEMV_EARLY_CHUNKS = 2;  // chunks issued before the CTA barrier
 
 struct GemvParams {
     const void* x;  // fp32/bf16 activations when the quantiser is fused
@@ -341,8 +342,11 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
     int r0, nrows;
     cta_rows(p, cta, ncta, r0, nrows);
     const int nchunks = (nrows + p.rpc - 1) / p.rpc;
-    // Thread 0 sets up the barriers and puts the slab's bulk copies in flight
-    // before anyone else runs, so the HBM stream starts as early as possible.
+    // Thread 0 sets up the barriers and puts the first chunks in flight before
+    // anyone else runs, so the HBM stream starts at once; the producer warp
+    // issues the rest after the CTA barrier.  (Issuing the whole slab here
+    // stalled the CTA barrier -- and so the consumers -- for microseconds when
+    // the memory system pushed back.)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&sh.full[s], 1);
@@ -353,12 +357,12 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
         // read before waiting for it
         sh.beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         fence_mbar_init();
-        produce(p, sh, ring, r0, nrows, 0, min(nchunks, p.stages));
+        produce(p, sh, ring, r0, nrows, 0, min(nchunks, GEMV_EARLY_CHUNKS));
     }
     __syncthreads();
     pdl_launch_dependents();
     if (warp == 0) {
-        if (lane == 0 && nchunks > p.stages) produce(p, sh, ring, r0, nrows, p.stages, nchunks);
+        if (lane == 0 && nchunks > GEMV_EARLY_CHUNKS) produce(p, sh, ring, r0, nrows, GEMV_EARLY_CHUNKS, nchunks);
         return;
     }
     pdl_wait();
