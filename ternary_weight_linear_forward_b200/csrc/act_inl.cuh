@@ -20,9 +20,14 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
            ((uint32_t)(d & 0xFF) << 24);
 }
 
-// same rounding as the standalone quantiser: rint(x * s), clamp to [-127, 127]
+// rint(x * s) clamped to [-127, 127], as the standalone quantiser.  Adding
+// 1.5 * 2^23 rounds the binary32 product to an integer, ties to even, exactly
+// like rint, because |x * s| <= 127 (1 + 2^-22) is far below 2^22; the integer
+// is then the low bits of the sum.  (An FADD on the FMA pipe instead of a
+// conversion on the quarter-rate XU pipe.)
 __device__ __forceinline__ int q8(float v, float s) {
-    int r = __float2int_rn(__fmul_rn(v, s));
+    const float t = __fadd_rn(__fmul_rn(v, s), 12582912.0f);
+    const int r = __float_as_int(t) - 0x4B400000;
     return min(max(r, -127), 127);
 }
 

@@ -238,6 +238,16 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
             gam[m] = fmaxf(__uint_as_float(a), 1e-5f);
             s[m] = __fdiv_rn(127.0f, gam[m]);
         }
+        if (ctid < MT) {
+            float f = 0.0f;
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m == ctid && p.mode != Y_ACC && m < p.M) f = __fdiv_rn(__fmul_rn(sh.beta, gam[m]), 127.0f);
+            sh.fscale[ctid] = f;
+        }
+    } else if (ctid < MT) {
+        const int m = ctid;
+        sh.fscale[m] = p.mode != Y_ACC && m < p.M ? __fdiv_rn(__fmul_rn(sh.beta, __ldg(p.gamma + m)), 127.0f) : 0.0f;
     }
     for (int i = ctid; i < GEMV_KS_MAX_ROWS * GEMV_SMALL_MAX_M; i += cthreads) (&sh.part[0][0])[i] = 0;
     // pass 2: write x_q chunks into their swizzled slots, accumulate row sums
@@ -274,20 +284,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
         int v = rs[m];
 #pragma unroll
         for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) sh.red_i[warp][m] = v;
-    }
-    consumer_sync(cthreads);
-    if (ctid < MT) {
-        const int m = ctid;
-        int t = 0;
-        for (int w = 0; w < cwarps; ++w) t += sh.red_i[w][m];
-        sh.rowsum[m] = t;
-        float f = 0.0f;
-        if (p.mode != Y_ACC && m < p.M) {
-            const float g = XM == X_QUANTISED ? __ldg(p.gamma + m) : gam[m];
-            f = __fdiv_rn(__fmul_rn(sh.beta, g), 127.0f);
-        }
-        sh.fscale[m] = f;
+        if (lane == 0 && v != 0) atomicAdd(&sh.rowsum[m], v);
     }
     consumer_sync(cthreads);
 }
@@ -353,6 +350,7 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
             mbar_init(&sh.empty[s], p.rpc * p.ks);  // every K slice of every row releases once
         }
         sh.abort_flag = 0;
+        for (int m = 0; m < GEMV_SMALL_MAX_M; ++m) sh.rowsum[m] = 0;
         // beta and W_p are weight inputs, not written by the preceding kernel:
         // read before waiting for it
         sh.beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
