@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int rs = 0;
             float f = 0.0f;
             if (m < p.M) {
-                rs = __ldg(p.rowsum + m);
+                rs = __ldcg(p.rowsum + m);  // L2 only: written by the preceding kernel
                 if (p.mode != Y_ACC) f = __fdiv_rn(__fmul_rn(beta, __ldg(p.gamma + m)), 127.0f);
             }
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
