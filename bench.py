@@ -339,21 +339,32 @@ def main():
                 "alone_per_shape": per_shape}
 
     # ---- end to end through the public API with pinned host buffers ----
-    host_x = [L["x"].cpu().pin_memory() for L in layers]
-    host_y = [torch.empty_like(L["y"], device="cpu").pin_memory() for L in layers]
-    dev_x = [torch.empty_like(L["x"]) for L in layers]
-    h2d = sum(h.numel() * h.element_size() for h in host_x)
-    d2h = sum(h.numel() * h.element_size() for h in host_y)
+    # The step's inputs (both projections' x) sit in one pinned host buffer and
+    # its outputs in one device / one pinned host buffer, so a step is one H2D
+    # copy, one library call (marshalled once per weight copy) and one D2H copy.
+    xs = [L["x"].reshape(-1) for L in layers]
+    ys = [L["y"].reshape(-1) for L in layers]
+    host_x = torch.cat([x.cpu() for x in xs]).pin_memory()
+    dev_xcat = torch.empty_like(host_x, device=dev)
+    ycat = torch.empty(sum(y.numel() for y in ys), dtype=torch.float32, device=dev)
+    host_y = torch.empty_like(ycat, device="cpu").pin_memory()
+    dev_x, dev_y, ox, oy = [], [], 0, 0
+    for L, x, y in zip(layers, xs, ys):
+        dev_x.append(dev_xcat[ox:ox + x.numel()].view(L["x"].shape))
+        dev_y.append(ycat[oy:oy + y.numel()].view(L["y"].shape))
+        ox += x.numel()
+        oy += y.numel()
+    plans = [bl.BatchPlan([{"x": dev_x[j], "W_p": L["W_p"][c], "beta": L["beta"], "out": dev_y[j]}
+                           for j, L in enumerate(layers)]) for c in range(copies)]
+    h2d = host_x.numel() * host_x.element_size()
+    d2h = host_y.numel() * host_y.element_size()
     n_e2e = max(16, min(args.steps, 2000))
 
     def e2e_step(i):
         with torch.cuda.stream(stream):
-            for j in range(len(layers)):
-                dev_x[j].copy_(host_x[j], non_blocking=True)
-            bl.forward_fp_batch([{"x": dev_x[j], "W_p": L["W_p"][i % copies], "beta": L["beta"], "out": L["y"]}
-                                 for j, L in enumerate(layers)], stream=stream)
-            for j, L in enumerate(layers):
-                host_y[j].copy_(L["y"], non_blocking=True)
+            dev_xcat.copy_(host_x, non_blocking=True)
+            plans[i % copies].run(stream=stream)
+            host_y.copy_(ycat, non_blocking=True)
     for i in range(4):
         e2e_step(i)
     torch.cuda.synchronize()
@@ -373,7 +384,9 @@ def main():
         t_e2e = float(t.item())
     e2e = {"value": world * step_bytes() * n_e2e / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": n_e2e,
-           "path": "pinned H2D copies + one bitlinear_forward_fp_batch (both projections) + D2H copies, one stream, no graph"}
+           "path": "one pinned H2D copy of both inputs + bitlinear_forward_fp_batch (both projections, descriptors "
+                   "marshalled once per weight copy) + one D2H copy of both outputs; one stream, no graph; weights "
+                   f"rotate over {copies} copies"}
 
     # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
     prefill = None

@@ -210,12 +210,38 @@ class _Problem(ctypes.Structure):
                 ("K", ctypes.c_int64), ("N", ctypes.c_int64)]
 
 
+class BatchPlan:
+    """A forward_fp_batch call marshalled once: the problem descriptors are
+    checked and packed into the C array when the plan is made, and ``run``
+    only passes them to the library.  The tensors must stay alive and keep
+    their storage while the plan is used (the descriptors hold pointers)."""
+
+    def __init__(self, problems, out_dtype=torch.float32):
+        self.arr, self.outs, self.m, self.xdt, self.ydt = _pack_batch(problems, out_dtype)
+        self._keep = [dict(pr) for pr in problems]
+        self._ptr = ctypes.cast(self.arr, ctypes.c_void_p)
+
+    def run(self, stream=None):
+        _check("bitlinear_forward_fp_batch",
+               lib().bitlinear_forward_fp_batch(self._ptr, len(self.outs), self.m, self.xdt, self.ydt,
+                                                _stream(stream)))
+        return self.outs
+
+
 def forward_fp_batch(problems, out_dtype=torch.float32, stream=None):
     """Several independent decode projections in one launch.
 
     ``problems``: list of dicts with keys ``x`` ([M, K] fp32/bf16, or int8 x_q
     together with ``gamma`` [M]), ``W_p``, ``beta`` and optionally ``out``.
     All share M (<= 4) and the x dtype.  Returns the list of outputs."""
+    arr, outs, m, xdt, ydt = _pack_batch(problems, out_dtype)
+    _check("bitlinear_forward_fp_batch",
+           lib().bitlinear_forward_fp_batch(ctypes.cast(arr, ctypes.c_void_p), len(problems), m, xdt, ydt,
+                                            _stream(stream)))
+    return outs
+
+
+def _pack_batch(problems, out_dtype):
     if not 1 <= len(problems) <= 8:
         raise ValueError("1 to 8 problems")
     arr = (_Problem * len(problems))()
@@ -246,10 +272,7 @@ def forward_fp_batch(problems, out_dtype=torch.float32, stream=None):
         raise ValueError("outputs must share a dtype")
     ydt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[outs[0].dtype]
     xdt = BL_I8 if quantised else BL_BF16 if x0.dtype == torch.bfloat16 else BL_F32
-    _check("bitlinear_forward_fp_batch",
-           lib().bitlinear_forward_fp_batch(ctypes.cast(arr, ctypes.c_void_p), len(problems), x0.shape[0], xdt, ydt,
-                                            _stream(stream)))
-    return outs
+    return arr, outs, x0.shape[0], xdt, ydt
 
 
 def forward_noalloc(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,

@@ -395,3 +395,15 @@ def test_forward_fp_batch_quantised_inputs(dev):
     outs = bl.forward_fp_batch(probs)
     for pr, out in zip(probs, outs):
         np.testing.assert_array_equal(out.cpu().numpy(), bl.forward(x_q, gamma, pr["W_p"], pr["beta"]).cpu().numpy())
+
+
+def test_batch_plan_matches_call(dev):
+    # the marshal-once plan runs the same launch as forward_fp_batch, call after call
+    probs, refs = _prep_batch(dev, [(4096, 1000), (2560, 777)], 1, "bf16", seed=7)
+    outs = bl.forward_fp_batch(probs)
+    plan = bl.BatchPlan([dict(pr, out=torch.empty_like(o)) for pr, o in zip(probs, outs)])
+    for _ in range(2):
+        got = plan.run()
+        for a, b, ref in zip(outs, got, refs):
+            assert torch.equal(a, b)
+            assert_f32_close(b.cpu().numpy(), ref["y64"])
