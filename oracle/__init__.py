@@ -14,7 +14,8 @@ Each function states the passage it follows.  Sources (web pages):
   product, a third BitLinear).
 * unite.ai "Microsofts Inference Framework bringt 1-Bit grosse Sprachmodelle
   auf lokale Geraete" (German), section "Mathematische Grundlagen", eq. 2
-  "Aktivierungsquantisierung" and eq. 3 "BitLinear-Betrieb".
+  "Aktivierungsquantisierung" and eq. 3 "BitLinear-Betrieb"; item 1
+  "Gewichtsbinarisierung", eq. 1 -- the 1-bit weights Sign(W - mean(W)).
 
 Pins (tests/test_oracle_pins.py): a hand-worked 4x4 example, closed forms of
 the Gaussian absmean statistics, invariants, brute force on tiny inputs and
@@ -43,6 +44,13 @@ _i64 = ctypes.c_int64
 
 _lib.orc_exact_abs_sum.argtypes = [_f32p, _i64]
 _lib.orc_exact_abs_sum.restype = ctypes.c_double
+_lib.orc_exact_sum.argtypes = [_f32p, _i64]
+_lib.orc_exact_sum.restype = ctypes.c_double
+_lib.orc_mean_alpha.argtypes = [_f32p, _i64, _i64]
+_lib.orc_mean_alpha.restype = ctypes.c_float
+_lib.orc_binarize.argtypes = [_f32p, _i64, _i64, ctypes.c_float, _i8p]
+_lib.orc_pack_bits.argtypes = [_i8p, _i64, _i64, _u32p]
+_lib.orc_unpack_bits.argtypes = [_u32p, _i64, _i64, _i8p]
 _lib.orc_absmean_beta.argtypes = [_f32p, _i64, _i64]
 _lib.orc_absmean_beta.restype = ctypes.c_float
 _lib.orc_ternarize.argtypes = [_f32p, _i64, _i64, ctypes.c_float, ctypes.c_float, _i8p]
@@ -116,6 +124,63 @@ def unpack(W_p: np.ndarray, K: int):
     out = np.empty((N, K), np.int8)
     bad = _lib.orc_unpack(W_p, N, K, out)
     return out, int(bad)
+
+
+# ---------------------------------------------------------------------------
+# 1-bit variant: unite.ai page, "Mathematische Grundlagen", item 1
+# "Gewichtsbinarisierung", eq. 1.
+# ---------------------------------------------------------------------------
+
+def exact_sum(w: np.ndarray) -> float:
+    """Exact signed sum over binary32 values, correctly rounded to binary64."""
+    w = _c(w, np.float32).ravel()
+    return float(_lib.orc_exact_sum(w, w.size))
+
+
+def mean_alpha(W: np.ndarray) -> np.float32:
+    """alpha = mean(W) over the whole matrix (eq. 1): the exact sum rounded to
+    binary64, divided by N*K in binary64, then rounded to binary32."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    return np.float32(_lib.orc_mean_alpha(W, N, K))
+
+
+def binarize(W: np.ndarray, alpha) -> np.ndarray:
+    """W_b = Sign(W - alpha) (eq. 1), Sign(d) = +1 if d > 0 else -1, with
+    d = W - alpha one binary32 subtraction."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    out = np.empty((N, K), np.int8)
+    _lib.orc_binarize(W, N, K, np.float32(alpha), out)
+    return out
+
+
+def binarize_weights(W: np.ndarray):
+    """Binarisation of a full-precision matrix -> (W_b int8 in {-1, +1}, alpha,
+    beta).  beta, which the page names a scaling factor without a formula, is
+    read as the same absmean scale mean |W| that the ternary weights use."""
+    alpha = mean_alpha(W)
+    return binarize(W, alpha), alpha, absmean_beta(W)
+
+
+def pack_bits(W_b: np.ndarray) -> np.ndarray:
+    """1 bit per weight: k = 32j + 4s + b of a row at bit 8b + s of word j,
+    set for +1 (w > 0), clear otherwise."""
+    W_b = _c(W_b, np.int8)
+    N, K = W_b.shape
+    assert K % 32 == 0
+    out = np.empty((N, K // 32), np.uint32)
+    _lib.orc_pack_bits(W_b, N, K, out)
+    return out
+
+
+def unpack_bits(W_p: np.ndarray, K: int) -> np.ndarray:
+    """Inverse of :func:`pack_bits` (set bit -> +1, clear bit -> -1)."""
+    W_p = _c(W_p, np.uint32)
+    N = W_p.shape[0]
+    out = np.empty((N, K), np.int8)
+    _lib.orc_unpack_bits(W_p, N, K, out)
+    return out
 
 
 def quant_act(x: np.ndarray):

@@ -19,7 +19,9 @@
  *          Sprachmodelle auf lokale Geraete" (German), section "Mathematische
  *          Grundlagen": eq. 2 "Aktivierungsquantisierung" (absmax quantiser
  *          with Q_b and gamma = ||x||_inf) and eq. 3 "BitLinear-Betrieb"
- *          (y = W_f x_hat (beta gamma / Q_b)).
+ *          (y = W_f x_hat (beta gamma / Q_b)); the 1-bit variant of the
+ *          weights is item 1 "Gewichtsbinarisierung", eq. 1
+ *          (W_f = Sign(W - alpha), alpha = mean(W)).
  *
  * Readings taken where the pages are silent (each one is listed with its
  * reason in the design notes of the repository):
@@ -30,6 +32,10 @@
  *   - Q_b = 127 with a symmetric clamp to [-127, 127]; gamma is per token,
  *     floored at 1e-5; the scale s = 127 / gamma is formed first, x * s after.
  *   - the output is y = (float)acc * ((beta * gamma) / 127) in binary32.
+ *   - binary variant: alpha is the exact mean of W rounded like beta;
+ *     Sign(0) = -1 as the page's definition of Sign states; beta of a
+ *     binarised matrix is the same absmean scale (the page names beta a
+ *     scaling factor without a formula).
  */
 #include <math.h>
 #include <stdint.h>
@@ -47,30 +53,34 @@
 /* ------------------------------------------------------------------------ */
 #define ORC_LIMBS 12  /* 12 * 32 = 384 bits >= 278 value bits + 64 carry bits */
 
-double orc_exact_abs_sum(const float* w, int64_t n)
+/* Add the magnitude of the binary32 pattern u (sign ignored) to acc. */
+static void limbs_add(uint64_t acc[ORC_LIMBS], uint32_t u)
 {
-    uint64_t acc[ORC_LIMBS];
-    memset(acc, 0, sizeof acc);
-    for (int64_t i = 0; i < n; ++i) {
-        uint32_t u;
-        memcpy(&u, &w[i], 4);
-        u &= 0x7FFFFFFFu;                       /* |w| */
-        if (u == 0) continue;
-        uint32_t e = u >> 23;
-        uint64_t m = u & 0x7FFFFFu;
-        uint32_t pos;                           /* bit position of m's bit 0 */
-        if (e == 0) { pos = 0; }
-        else { m |= 0x800000u; pos = e - 1; }
-        uint64_t shifted = m << (pos % 32);     /* < 2^55 */
-        uint32_t d = pos / 32;
-        acc[d] += shifted & 0xFFFFFFFFu;
-        acc[d + 1] += shifted >> 32;
-    }
-    /* carry-normalise to 32-bit digits */
+    u &= 0x7FFFFFFFu;
+    if (u == 0) return;
+    uint32_t e = u >> 23;
+    uint64_t m = u & 0x7FFFFFu;
+    uint32_t pos;                               /* bit position of m's bit 0 */
+    if (e == 0) { pos = 0; }
+    else { m |= 0x800000u; pos = e - 1; }
+    uint64_t shifted = m << (pos % 32);         /* < 2^55 */
+    uint32_t d = pos / 32;
+    acc[d] += shifted & 0xFFFFFFFFu;
+    acc[d + 1] += shifted >> 32;
+}
+
+/* carry-normalise to 32-bit digits */
+static void limbs_normalise(uint64_t acc[ORC_LIMBS])
+{
     for (int d = 0; d + 1 < ORC_LIMBS; ++d) {
         acc[d + 1] += acc[d] >> 32;
         acc[d] &= 0xFFFFFFFFu;
     }
+}
+
+/* The normalised integer acc (units of 2^-149), rounded once to binary64. */
+static double limbs_to_double(const uint64_t acc[ORC_LIMBS])
+{
     int top = -1;
     for (int d = ORC_LIMBS - 1; d >= 0; --d)
         if (acc[d]) { top = d; break; }
@@ -97,6 +107,52 @@ double orc_exact_abs_sum(const float* w, int64_t n)
     return ldexp(d, lo - 149);
 }
 
+double orc_exact_abs_sum(const float* w, int64_t n)
+{
+    uint64_t acc[ORC_LIMBS];
+    memset(acc, 0, sizeof acc);
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t u;
+        memcpy(&u, &w[i], 4);
+        limbs_add(acc, u);
+    }
+    limbs_normalise(acc);
+    return limbs_to_double(acc);
+}
+
+/* Exact signed sum of n binary32 values, correctly rounded to binary64: the
+ * positive and the negative elements are added exactly into two integers, the
+ * smaller magnitude is subtracted from the larger, and the difference is
+ * rounded once. */
+double orc_exact_sum(const float* w, int64_t n)
+{
+    uint64_t pos[ORC_LIMBS], neg[ORC_LIMBS];
+    memset(pos, 0, sizeof pos);
+    memset(neg, 0, sizeof neg);
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t u;
+        memcpy(&u, &w[i], 4);
+        limbs_add((u >> 31) ? neg : pos, u);
+    }
+    limbs_normalise(pos);
+    limbs_normalise(neg);
+    int cmp = 0;
+    for (int d = ORC_LIMBS - 1; d >= 0 && cmp == 0; --d)
+        cmp = pos[d] > neg[d] ? 1 : pos[d] < neg[d] ? -1 : 0;
+    if (cmp == 0) return 0.0;
+    const uint64_t* big = cmp > 0 ? pos : neg;
+    const uint64_t* small = cmp > 0 ? neg : pos;
+    uint64_t diff[ORC_LIMBS];
+    uint64_t borrow = 0;
+    for (int d = 0; d < ORC_LIMBS; ++d) {
+        uint64_t sub = small[d] + borrow;           /* digits < 2^32: no wrap */
+        borrow = big[d] < sub ? 1u : 0u;
+        diff[d] = (big[d] + (borrow << 32)) - sub;
+    }
+    double r = limbs_to_double(diff);
+    return cmp > 0 ? r : -r;
+}
+
 /* [MMF] absmean: beta = mean |W| over the whole matrix (one scale per matrix). */
 float orc_absmean_beta(const float* W, int64_t N, int64_t K)
 {
@@ -117,6 +173,58 @@ void orc_ternarize(const float* W, int64_t N, int64_t K, float beta, float eps, 
         if (r < -1.0f) r = -1.0f;
         W_t[i] = (int8_t)r;
     }
+}
+
+/* [BNC] "Mathematische Grundlagen", item 1 "Gewichtsbinarisierung", eq. 1:
+ * alpha = mean(W) over the whole matrix -- the exact sum rounded once to
+ * binary64, divided by N*K in binary64, rounded to binary32 (as beta). */
+float orc_mean_alpha(const float* W, int64_t N, int64_t K)
+{
+    int64_t n = N * K;
+    if (n <= 0) return 0.0f;
+    double s = orc_exact_sum(W, n);
+    return (float)(s / (double)n);
+}
+
+/* [BNC] eq. 1: W_b = Sign(W - alpha), with Sign(d) = +1 for d > 0 and -1
+ * otherwise (zero included); d = W - alpha is one binary32 subtraction. */
+void orc_binarize(const float* W, int64_t N, int64_t K, float alpha, int8_t* W_b)
+{
+    for (int64_t i = 0; i < N * K; ++i) {
+        float d = W[i] - alpha;
+        W_b[i] = d > 0.0f ? (int8_t)1 : (int8_t)-1;
+    }
+}
+
+/* 1-bit storage of binary weights, 32 per uint32: for row n and word j, the
+ * weight at k = 32j + 4s + b (s in 0..7, b in 0..3) is bit 8b + s of
+ * W_p[n, j], set for +1 and clear for -1 (any w <= 0 is stored as -1). */
+void orc_pack_bits(const int8_t* W_b, int64_t N, int64_t K, uint32_t* W_p)
+{
+    int64_t KW = K / 32;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < KW; ++j) {
+            uint32_t word = 0;
+            for (int t = 0; t < 32; ++t) {
+                int s = t / 4, b = t % 4;
+                if (W_b[n * K + 32 * j + t] > 0) word |= 1u << (8 * b + s);
+            }
+            W_p[n * KW + j] = word;
+        }
+}
+
+/* Inverse of orc_pack_bits: set bits give +1, clear bits -1. */
+void orc_unpack_bits(const uint32_t* W_p, int64_t N, int64_t K, int8_t* W_b)
+{
+    int64_t KW = K / 32;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < KW; ++j) {
+            uint32_t word = W_p[n * KW + j];
+            for (int t = 0; t < 32; ++t) {
+                int s = t / 4, b = t % 4;
+                W_b[n * K + 32 * j + t] = ((word >> (8 * b + s)) & 1u) ? (int8_t)1 : (int8_t)-1;
+            }
+        }
 }
 
 /* 2-bit storage of the trits (the "1.58 bit" weights of [BNC] "Ternaeres
