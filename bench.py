@@ -480,6 +480,61 @@ def main():
                  "copies": nblk}
         del g, blocks
 
+    # ---- 1-bit weights (Sign(W - mean W)): decode GEMV and prefill GEMM ----
+    binary = None
+    if not args.no_prefill:
+        binary = {}
+        for s in workloads.W2.shapes:
+            W_b, _, beta = bl.binarize_weights(torch.from_numpy(s.weights()).to(dev))
+            W_p0 = bl.pack_bits(W_b)
+            del W_b
+            nc = max(2, int(4 * L2 // (W_p0.numel() * 4)) + 1)
+            W_ps = [W_p0] + [W_p0.clone() for _ in range(nc - 1)]
+            xb = torch.from_numpy(s.inputs_bf16_bits().view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((s.M, s.N), dtype=torch.float32, device=dev)
+            # algorithmic bytes: 1-bit weights, bf16 x, f32 y, beta
+            nbytes = s.N * s.K // 8 + s.M * s.K * 2 + s.M * s.N * 4 + 4
+            reps = 8 * nc
+            with torch.cuda.stream(stream):
+                for i in range(4):
+                    bl.forward_binary_fp(xb, W_ps[i % nc], beta, out=y, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(reps):
+                        bl.forward_binary_fp(xb, W_ps[i % nc], beta, out=y, stream=stream)
+            g.replay()
+            t = timed_run([g])
+            gbs = nbytes * reps / t / 1e9
+            binary["decode_" + s.name] = {"us_per_call": t / reps * 1e6, "GB/s": gbs,
+                                          "frac_of_hbm": gbs / peaks["hbm_gbs"], "bytes_per_call": nbytes,
+                                          "path": "CUDA-core GEMV on 1-bit words, quantiser fused"}
+            del g, W_ps, W_p0, xb, y
+        for s in workloads.W4.shapes:
+            W_b, _, beta = bl.binarize_weights(torch.from_numpy(s.weights()).to(dev))
+            W_p = bl.pack_bits(W_b)
+            del W_b
+            x_q, gamma = bl.quant_act(torch.from_numpy(s.inputs()).to(dev))
+            y = torch.empty((s.M, s.N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.lib().bitlinear_forward_binary_workspace(s.M, s.N, s.K), dtype=torch.uint8,
+                             device=dev)
+            reps = 20
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    bl.forward_binary(x_q, gamma, W_p, beta, out=y, ws=ws, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(reps):
+                        bl.forward_binary(x_q, gamma, W_p, beta, out=y, ws=ws, stream=stream)
+            g.replay()
+            t = timed_run([g])
+            tops = s.ops * reps / t / 1e12
+            binary["prefill_" + s.name] = {"us_per_call": t / reps * 1e6, "TOPS": tops,
+                                           "frac_of_int8_peak": tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
+                                           "path": "tcgen05 GEMM, 1-bit unpack"}
+            del g, W_p, x_q, y, ws
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -501,6 +556,7 @@ def main():
                        "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks, "prefill": prefill, "small_batch": small, "block": block,
+            "binary": binary,
             "device": props.name,
         }
         print(json.dumps(line), flush=True)

@@ -15,7 +15,8 @@
  *         Gewichtssystem" (1.58-bit ternary weights), section "Mathematische
  *         Grundlagen" eq. 2 "Aktivierungsquantisierung" and eq. 3
  *         "BitLinear-Betrieb", section "Implementierungshinweise" (the
- *         quantise -> ternary matmul -> scale shape of a forward call).
+ *         quantise -> ternary matmul -> scale shape of a forward call); the
+ *         1-bit weights of the same section, item 1 "Gewichtsbinarisierung".
  *
  * Conventions for every call:
  *   - Every pointer argument is a DEVICE pointer owned by the caller (the
@@ -238,6 +239,91 @@ bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K,
 bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
                                     const uint32_t* W_p, const float* beta, int64_t N,
                                     void* y, int y_dtype, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 1-bit weight variant                                                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [BNC] "Mathematische Grundlagen", item 1 "Gewichtsbinarisierung", eq. 1:
+ * the weights are centred on their mean and binarised,
+ *   W_b = Sign(W - alpha),  alpha = mean(W),  Sign(d) = +1 for d > 0, else -1
+ * (so an element equal to alpha gets -1), and eq. 3 applies unchanged with
+ * W_f = W_b.  The forward below is the same contraction as for ternary
+ * weights, restricted to w in {-1, +1} and stored in 1 bit per weight.
+ */
+
+/* Bytes of device workspace bitlinear_binarize_weights needs (any N, K). */
+size_t bitlinear_binarize_weights_workspace(int64_t N, int64_t K);
+
+/*
+ * Binarisation of a full-precision matrix, eq. 1 above.
+ *   alpha = (float)(S / (N*K))   S = the exact sum of W rounded once to
+ *                                binary64, divided in binary64
+ *   beta  = mean |W| exactly as bitlinear_quantize_weights computes it (the
+ *           page names beta a scaling factor without a formula; this library
+ *           reads it as the absmean scale of the ternary weights)
+ *   W_b   = +1 where (W - alpha) > 0 in binary32, else -1
+ *   W     [N, K] float32 in
+ *   W_b   [N, K] int8 out, values in {-1, +1}
+ *   alpha [1] float32 out, beta [1] float32 out (distinct buffers)
+ *   ws    >= bitlinear_binarize_weights_workspace(N, K) bytes of device scratch
+ * K % 32 == 0.  Sums are exact integers on a grid set by max |W| and do not
+ * depend on thread order; alpha and beta are the exact means (as defined
+ * above) whenever every nonzero |w| >= 2^-38 * max |W|, and elements below
+ * that are truncated to the grid.
+ */
+bl_status bitlinear_binarize_weights(const float* W, int64_t N, int64_t K, int8_t* W_b, float* alpha,
+                                     float* beta, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * 1-bit packing, 32 weights per uint32.  For row n and word j, the weight at
+ * k = 32j + 4s + b (s in 0..7, b in 0..3) is bit 8b + s of W_p[n, j]: set for
+ * w > 0 (+1), clear otherwise (-1), so that (word >> s) & 0x01010101 holds
+ * the signs of k = 32j+4s .. 32j+4s+3 in its four bytes.
+ *   W_b [N, K] int8 in (values <= 0 are stored as -1)
+ *   W_p [N, K/32] uint32 out
+ * K % 32 == 0.
+ */
+bl_status bitlinear_pack_bits(const int8_t* W_b, int64_t N, int64_t K, uint32_t* W_p, void* stream);
+
+/* Bytes of device workspace bitlinear_forward_binary needs for this shape (may be 0). */
+size_t bitlinear_forward_binary_workspace(int64_t M, int64_t N, int64_t K);
+
+/*
+ * BitLinear forward with 1-bit weights, eq. 3 with W_f = W_b:
+ *   acc[m, n] = sum_k W_b[n, k] * x_q[m, k]
+ *             = 2 * sum_{k: W_b = +1} x_q[m, k] - sum_k x_q[m, k]  (int32, exact)
+ *   y[m, n]   = (float)acc[m, n] * ((beta * gamma_m) / 127)      (binary32, this order)
+ * Arguments as for bitlinear_forward, with W_p [N, K/32] in the
+ * bitlinear_pack_bits layout.  K % 128 == 0, K <= BL_MAX_K.  M <= 4 tokens
+ * (with M rounded up to 1, 2 or 4, times K <= 65536) run the CUDA-core GEMV,
+ * which streams 1 bit per weight; other shapes run the tcgen05 GEMM.  The
+ * decode engine setting does not apply.  The same rule on W_p and beta as
+ * for bitlinear_forward (they are read before the preceding kernel ends).
+ */
+bl_status bitlinear_forward_binary(const int8_t* x_q, const float* gamma, int64_t M, int64_t K,
+                                   const uint32_t* W_p, const float* beta, int64_t N,
+                                   void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* Integer accumulators of bitlinear_forward_binary (same kernels, rescale skipped). */
+bl_status bitlinear_forward_binary_acc(const int8_t* x_q, int64_t M, int64_t K,
+                                       const uint32_t* W_p, int64_t N, int32_t* acc,
+                                       void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace bitlinear_forward_binary_fp needs for this shape (may be 0). */
+size_t bitlinear_forward_binary_fp_workspace(int64_t M, int64_t N, int64_t K);
+
+/*
+ * bitlinear_quant_act(x) followed by bitlinear_forward_binary, bit-identical
+ * to the two calls.  Where the GEMV runs (see above) the quantiser is fused
+ * into its prologue and the workspace is 0.
+ *   x [M, K] float32 (BL_F32) or bfloat16 (BL_BF16) in; other arguments as
+ *   for bitlinear_forward_binary.  K % 128 == 0, K <= BL_MAX_K.
+ */
+bl_status bitlinear_forward_binary_fp(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* W_p,
+                                      const float* beta, int64_t N, void* y, int y_dtype, void* ws,
+                                      size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decoder-block glue                                                        */

@@ -41,6 +41,14 @@ SIGNATURES = {
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_binarize_weights_workspace": (_SZ, [_I64, _I64]),
+    "bitlinear_binarize_weights": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "bitlinear_pack_bits": (_I, [_P, _I64, _I64, _P, _P]),
+    "bitlinear_forward_binary_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_forward_binary": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_binary_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_forward_binary_fp_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_forward_binary_fp": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_set_decode_engine": (_I, [_I]),
     "bitlinear_get_decode_engine": (_I, []),
     "bitlinear_device_status": (_I, [_P]),
@@ -315,6 +323,101 @@ def forward_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=None) -> t
            lib().bitlinear_forward_acc(_ptr(x_q), M, K, _ptr(W_p), N, _ptr(acc), _ptr(ws),
                                        0 if ws is None else ws.numel(), _stream(stream)))
     return acc
+
+
+# --------------------------------------------------------------------------
+# 1-bit weights (unite.ai page, "Mathematische Grundlagen", item 1
+# "Gewichtsbinarisierung": W_b = Sign(W - mean(W)))
+# --------------------------------------------------------------------------
+
+def binarize_weights(W: torch.Tensor, stream=None):
+    """Binarisation -> (W_b int8 [N, K] in {-1, +1}, alpha float32 [1], beta float32 [1])."""
+    _need(W, torch.float32, 2, "W")
+    N, K = W.shape
+    W_b = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    ab = torch.empty(8, dtype=torch.float32, device=W.device)
+    alpha, beta = ab[0:1], ab[4:5]  # distinct 16-byte-aligned scalars
+    nws = lib().bitlinear_binarize_weights_workspace(N, K)
+    ws = torch.empty(nws, dtype=torch.uint8, device=W.device)
+    _check("bitlinear_binarize_weights",
+           lib().bitlinear_binarize_weights(_ptr(W), N, K, _ptr(W_b), _ptr(alpha), _ptr(beta), _ptr(ws), nws,
+                                            _stream(stream)))
+    return W_b, alpha, beta
+
+
+def pack_bits(W_b: torch.Tensor, stream=None) -> torch.Tensor:
+    """1-bit packing, 32 signs per uint32 -> W_p int32 [N, K/32] (bit pattern of uint32)."""
+    _need(W_b, torch.int8, 2, "W_b")
+    N, K = W_b.shape
+    W_p = torch.empty((N, K // 32 if K % 32 == 0 else 1), dtype=torch.int32, device=W_b.device)
+    _check("bitlinear_pack_bits", lib().bitlinear_pack_bits(_ptr(W_b), N, K, _ptr(W_p), _stream(stream)))
+    return W_p
+
+
+def _bits_shape(W_p, K):
+    if W_p.shape[1] * 32 != K:
+        raise ValueError("W_p must be [N, K/32]")
+    return W_p.shape[0]
+
+
+def forward_binary(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,
+                   out_dtype=torch.float32, out=None, ws=None, stream=None) -> torch.Tensor:
+    """y = BitLinear(x_q) with 1-bit weights and the fused rescale."""
+    _need(x_q, torch.int8, 2, "x_q")
+    _need(W_p, torch.int32, 2, "W_p")
+    _need(gamma, torch.float32, 1, "gamma")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x_q.shape
+    N = _bits_shape(W_p, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = int(lib().bitlinear_forward_binary_workspace(M, N, K))
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward_binary",
+           lib().bitlinear_forward_binary(_ptr(x_q), _ptr(gamma), M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                          _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_binary_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """int32 accumulators sum_k W_b[n, k] x_q[m, k] of the 1-bit forward."""
+    _need(x_q, torch.int8, 2, "x_q")
+    _need(W_p, torch.int32, 2, "W_p")
+    M, K = x_q.shape
+    N = _bits_shape(W_p, K)
+    acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
+    nws = int(lib().bitlinear_forward_binary_workspace(M, N, K))
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward_binary_acc",
+           lib().bitlinear_forward_binary_acc(_ptr(x_q), M, K, _ptr(W_p), N, _ptr(acc), _ptr(ws),
+                                              0 if ws is None else ws.numel(), _stream(stream)))
+    return acc
+
+
+def forward_binary_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype=torch.float32, out=None,
+                      ws=None, stream=None) -> torch.Tensor:
+    """quant_act + forward_binary in one call (one kernel for M <= 4)."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, 2, "x")
+    _need(W_p, torch.int32, 2, "W_p")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x.shape
+    N = _bits_shape(W_p, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = int(lib().bitlinear_forward_binary_fp_workspace(M, N, K))
+    if nws and ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x.device)
+    xdt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_forward_binary_fp",
+           lib().bitlinear_forward_binary_fp(_ptr(x), xdt, M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                             _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return out
 
 
 def quant_act_rms(a: torch.Tensor, b: torch.Tensor | None = None, combine: str = "none", h=None,

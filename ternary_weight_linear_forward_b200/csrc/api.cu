@@ -65,17 +65,18 @@ bl_status check_nk(int64_t N, int64_t K, int64_t k_mult) {
     return BL_OK;
 }
 
+// wbits: 2 for packed trits (K % 64 == 0), 1 for packed signs (K % 128 == 0)
 bl_status check_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
-                        const float* beta, int64_t N, const void* y, size_t y_elem) {
+                        const float* beta, int64_t N, const void* y, size_t y_elem, int wbits = 2) {
     if (!x_q || !W_p || !y || (y_elem != 4 && (!gamma || !beta))) return BL_ERR_NULL;
     if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
-    bl_status s = check_nk(N, K, 64);
+    bl_status s = check_nk(N, K, wbits == 2 ? 64 : 128);
     if (s) return s;
     if (!aligned16(x_q) || !aligned16(W_p) || !aligned16(y) || (gamma && !aligned16(gamma)) ||
         (beta && !aligned16(beta)))
         return BL_ERR_ALIGN;
     const size_t ybytes = (size_t)M * N * y_elem;
-    if (overlap(y, ybytes, x_q, (size_t)M * K) || overlap(y, ybytes, W_p, (size_t)N * (K / 16) * 4) ||
+    if (overlap(y, ybytes, x_q, (size_t)M * K) || overlap(y, ybytes, W_p, (size_t)N * K * wbits / 8) ||
         overlap(y, ybytes, gamma, gamma ? (size_t)M * 4 : 0) || overlap(y, ybytes, beta, beta ? 4 : 0))
         return BL_ERR_ALIAS;
     return BL_OK;
@@ -124,6 +125,32 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
         e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
+    return from_cuda(e);
+}
+
+// 1-bit weights: the CUDA-core GEMV for a few tokens whose x_hat fits its
+// shared memory, the tensor-core GEMM otherwise.
+bool bits_on_gemv(int64_t M, int64_t K) { return M <= AUTO_CUDA_MAX_M && gemv_bits_ok(M, K); }
+
+size_t forward_bits_ws(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || K < 1 || bits_on_gemv(M, K)) return 0;
+    return gemm_ws_bytes(M, N, K);
+}
+
+bl_status run_forward_bits(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
+                           const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes,
+                           void* stream) {
+    const size_t need = forward_bits_ws(M, N, K);
+    if (need && (!ws || ws_bytes < need)) return BL_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return BL_ERR_ALIGN;
+    DevInfo dev;
+    bl_status s = current_device(dev);
+    if (s) return s;
+    cudaError_t e;
+    if (bits_on_gemv(M, K))
+        e = launch_gemv_bits(x_q, BL_I8, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
+    else
+        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream), 1);
     return from_cuda(e);
 }
 
@@ -210,6 +237,48 @@ bl_status bitlinear_pack(const int8_t* W_t, int64_t N, int64_t K, uint32_t* W_p,
     s = current_device(dev);
     if (s) return s;
     return from_cuda(launch_pack(W_t, (long long)(n / 16), W_p, dev.num_sms, as_stream(stream)));
+}
+
+size_t bitlinear_binarize_weights_workspace(int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return binarize_weights_ws_bytes();
+}
+
+bl_status bitlinear_binarize_weights(const float* W, int64_t N, int64_t K, int8_t* W_b, float* alpha, float* beta,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    if (!W || !W_b || !alpha || !beta) return BL_ERR_NULL;
+    bl_status s = check_nk(N, K, 32);
+    if (s) return s;
+    if (!ws || ws_bytes < binarize_weights_ws_bytes()) return BL_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(W_b) || !aligned16(alpha) || !aligned16(beta) || !aligned16(ws))
+        return BL_ERR_ALIGN;
+    const size_t n = (size_t)N * K;
+    const void* outs[4] = {W_b, alpha, beta, ws};
+    const size_t sizes[4] = {n, 4, 4, ws_bytes};
+    for (int i = 0; i < 4; ++i) {
+        if (overlap(outs[i], sizes[i], W, n * 4)) return BL_ERR_ALIAS;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlap(outs[i], sizes[i], outs[j], sizes[j])) return BL_ERR_ALIAS;
+    }
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(
+        launch_binarize_weights(W, (long long)n, W_b, alpha, beta, ws, dev.num_sms, as_stream(stream)));
+}
+
+bl_status bitlinear_pack_bits(const int8_t* W_b, int64_t N, int64_t K, uint32_t* W_p, void* stream) {
+    if (!W_b || !W_p) return BL_ERR_NULL;
+    bl_status s = check_nk(N, K, 32);
+    if (s) return s;
+    if (!aligned16(W_b) || !aligned16(W_p)) return BL_ERR_ALIGN;
+    const size_t n = (size_t)N * K;
+    if (overlap(W_p, n / 8, W_b, n)) return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_pack_bits(W_b, (long long)(n / 32), W_p, dev.num_sms, as_stream(stream)));
 }
 
 bl_status bitlinear_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, int8_t* x_q, float* gamma,
@@ -334,6 +403,67 @@ bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int6
     if (pick_path((int)M, probs, count, dev) == PATH_TC)
         return from_cuda(launch_decode_tc(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
     return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
+}
+
+size_t bitlinear_forward_binary_workspace(int64_t M, int64_t N, int64_t K) { return forward_bits_ws(M, N, K); }
+
+bl_status bitlinear_forward_binary(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
+                                   const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    if (!gamma || !beta) return BL_ERR_NULL;
+    if (y_dtype != BL_F32 && y_dtype != BL_BF16) {
+        if (!x_q || !W_p || !y) return BL_ERR_NULL;
+        return BL_ERR_DTYPE;
+    }
+    bl_status s = check_forward(x_q, gamma, M, K, W_p, beta, N, y, y_dtype == BL_F32 ? 4 : 2, 1);
+    if (s) return s;
+    return run_forward_bits(x_q, gamma, M, K, W_p, beta, N, y, y_dtype == BL_F32 ? Y_F32 : Y_BF16, ws, ws_bytes,
+                            stream);
+}
+
+bl_status bitlinear_forward_binary_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,
+                                       int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
+    bl_status s = check_forward(x_q, nullptr, M, K, W_p, nullptr, N, acc, 4, 1);
+    if (s) return s;
+    return run_forward_bits(x_q, nullptr, M, K, W_p, nullptr, N, acc, Y_ACC, ws, ws_bytes, stream);
+}
+
+size_t bitlinear_forward_binary_fp_workspace(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || K < 1 || bits_on_gemv(M, K)) return 0;
+    return round256((size_t)M * K) + round256((size_t)M * 4) + forward_bits_ws(M, N, K);
+}
+
+bl_status bitlinear_forward_binary_fp(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* W_p,
+                                      const float* beta, int64_t N, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                                      void* stream) {
+    if (!x || !W_p || !beta || !y) return BL_ERR_NULL;
+    if ((x_dtype != BL_F32 && x_dtype != BL_BF16) || (y_dtype != BL_F32 && y_dtype != BL_BF16)) return BL_ERR_DTYPE;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 128);
+    if (s) return s;
+    if (!aligned16(x) || !aligned16(W_p) || !aligned16(beta) || !aligned16(y)) return BL_ERR_ALIGN;
+    const size_t ye = y_dtype == BL_F32 ? 4 : 2;
+    const size_t ybytes = (size_t)M * N * ye, xb = (size_t)M * K * (x_dtype == BL_BF16 ? 2 : 4);
+    if (overlap(y, ybytes, x, xb) || overlap(y, ybytes, W_p, (size_t)N * K / 8) || overlap(y, ybytes, beta, 4))
+        return BL_ERR_ALIAS;
+    const size_t need = bitlinear_forward_binary_fp_workspace(M, N, K);
+    if (need && (!ws || ws_bytes < need)) return BL_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return BL_ERR_ALIGN;
+    if (need && (overlap(ws, need, x, xb) || overlap(ws, need, y, ybytes))) return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
+    if (!need)  // quantiser fused into the GEMV prologue
+        return from_cuda(launch_gemv_bits(x, x_dtype, nullptr, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev,
+                                          as_stream(stream)));
+    int8_t* x_q = reinterpret_cast<int8_t*>(ws);
+    float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
+    char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * 4);
+    cudaError_t e = launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream));
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    return run_forward_bits(x_q, gamma, M, K, W_p, beta, N, y, mode, fws,
+                            ws_bytes - (size_t)(fws - reinterpret_cast<char*>(ws)), stream);
 }
 
 bl_status bitlinear_forward_acc(const int8_t* x_q, int64_t M, int64_t K, const uint32_t* W_p, int64_t N,

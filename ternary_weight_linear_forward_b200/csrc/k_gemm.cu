@@ -7,6 +7,10 @@
 //
 //   D[m, n] = sum_k x_q[m, k] * c[n, k]      (c = w + 1 in {0, 1, 2}, s8 x s8 -> s32)
 //   acc     = D[m, n] - rowsum_m             (rowsum_m = sum_k x_q[m, k])
+//
+// The same kernel serves the 1-bit weights of the page's "Gewichtsbinarisierung"
+// (w in {-1, +1}, 32 signs per word): their codes c = w + 1 are {0, 2}, so only
+// the unpack differs.
 //   y       = (float)acc * ((beta * gamma_m) / 127)
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles, K in blocks of
@@ -40,7 +44,7 @@ constexpr int BK = 128;  // bytes of K per stage
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;           // 16 KiB
 constexpr int BC_BYTES = BN * BK;          // 32 KiB unpacked codes
-constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words
+constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words (2-bit; 1-bit uses half)
 constexpr int STAGE_BYTES = A_BYTES + BC_BYTES + BP_BYTES;
 constexpr int HDR_BYTES = 1024;
 constexpr int GEMM_SMEM = 1024 /* alignment slack */ + HDR_BYTES + STAGES * STAGE_BYTES;
@@ -48,7 +52,11 @@ constexpr int UNPACK_WARPS = 8;
 constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;               // epilogue warps EPI_WARP0 .. +3
 constexpr int GEMM_THREADS = (EPI_WARP0 + 4) * 32;
-constexpr int WORDS_PER_THREAD = BN * (BK / 16) / UNPACK_THREADS;  // packed words per K-block
+// packed words per row and K-block: 8 of 16 trits, or 4 of 32 signs
+template <int WB>
+constexpr int words_per_row() { return BK * WB / 32; }
+template <int WB>
+constexpr int words_per_thread() { return BN * words_per_row<WB>() / UNPACK_THREADS; }
 constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators
 
 constexpr uint32_t IDESC = idesc_i8(BM, BN, true, true);  // s8 x s8 -> s32, 128 x 256
@@ -146,6 +154,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int m, int n0, 
     }
 }
 
+template <int WB>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
@@ -191,9 +200,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!wait_or_abort(h, &h.empty[s], ph ^ 1)) goto done;
                     unsigned char* st = stages + (size_t)s * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&h.full[s], A_BYTES + BP_BYTES);
+                    mbar_arrive_expect_tx(&h.full[s], A_BYTES + BN * words_per_row<WB>() * 4);
                     tma_load_2d(st, &tmap_a, kb * BK, mb * BM, &h.full[s]);
-                    tma_load_2d(st + A_BYTES + BC_BYTES, &tmap_b, kb * (BK / 16), nb * BN, &h.full[s]);
+                    tma_load_2d(st + A_BYTES + BC_BYTES, &tmap_b, kb * words_per_row<WB>(), nb * BN, &h.full[s]);
                 }
             }
         }
@@ -226,15 +235,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else if (warp < EPI_WARP0) {
         // ------------------------------------------------ unpack
+        constexpr int WPR = words_per_row<WB>(), WPT = words_per_thread<WB>();
         const int ut = threadIdx.x - 64;  // 0 .. UNPACK_THREADS - 1
-        // word w = ut + UNPACK_THREADS * i of the packed tile is row n = w / 8,
-        // word j = w % 8: its 16 codes go to 16-byte chunk j ^ (n % 8) of row n
-        uint32_t dst_off[WORDS_PER_THREAD];
+        // word w = ut + UNPACK_THREADS * i of the packed tile is row n = w / WPR,
+        // word j = w % WPR.  2-bit: its 16 codes go to 16-byte chunk j ^ (n % 8)
+        // of row n.  1-bit: its 32 codes go to chunks 2j and 2j + 1 (swizzled
+        // the same way); dst_off holds the first, the second is found by ^ 16.
+        uint32_t dst_off[WPT];
 #pragma unroll
-        for (int i = 0; i < WORDS_PER_THREAD; ++i) {
+        for (int i = 0; i < WPT; ++i) {
             const int w = ut + UNPACK_THREADS * i;
-            const int n = w >> 3, j = w & 7;
-            dst_off[i] = (uint32_t)(n * BK + ((j ^ (n & 7)) << 4));
+            const int n = w / WPR, j = w % WPR;
+            const int c = WB == 2 ? j : 2 * j;
+            dst_off[i] = (uint32_t)(n * BK + ((c ^ (n & 7)) << 4));
         }
         int it = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
@@ -245,18 +258,37 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 unsigned char* st = stages + (size_t)s * STAGE_BYTES;
                 const uint32_t* bp = reinterpret_cast<const uint32_t*>(st + A_BYTES + BC_BYTES);
                 const uint32_t bc = smem_u32(st + A_BYTES);
-                uint32_t word[WORDS_PER_THREAD];
+                uint32_t word[WPT];
 #pragma unroll
-                for (int i = 0; i < WORDS_PER_THREAD; ++i) word[i] = bp[ut + UNPACK_THREADS * i];
+                for (int i = 0; i < WPT; ++i) word[i] = bp[ut + UNPACK_THREADS * i];
 #pragma unroll
-                for (int i = 0; i < WORDS_PER_THREAD; ++i) {
-                    const uint32_t t0 = word[i] & 0x03030303u;
-                    const uint32_t t1 = (word[i] >> 2) & 0x03030303u;
-                    const uint32_t t2 = (word[i] >> 4) & 0x03030303u;
-                    const uint32_t t3 = (word[i] >> 6) & 0x03030303u;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(bc + dst_off[i]), "r"(t0), "r"(t1),
-                                 "r"(t2), "r"(t3)
-                                 : "memory");
+                for (int i = 0; i < WPT; ++i) {
+                    if constexpr (WB == 2) {
+                        const uint32_t t0 = word[i] & 0x03030303u;
+                        const uint32_t t1 = (word[i] >> 2) & 0x03030303u;
+                        const uint32_t t2 = (word[i] >> 4) & 0x03030303u;
+                        const uint32_t t3 = (word[i] >> 6) & 0x03030303u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(bc + dst_off[i]), "r"(t0),
+                                     "r"(t1), "r"(t2), "r"(t3)
+                                     : "memory");
+                    } else {
+                        // sign bit of k = 32j + 4s + b at bit 8b + s -> code 2 * bit in byte b of int s
+                        const uint32_t w = word[i];
+                        const uint32_t t0 = (w << 1) & 0x02020202u;
+                        const uint32_t t1 = w & 0x02020202u;
+                        const uint32_t t2 = (w >> 1) & 0x02020202u;
+                        const uint32_t t3 = (w >> 2) & 0x02020202u;
+                        const uint32_t t4 = (w >> 3) & 0x02020202u;
+                        const uint32_t t5 = (w >> 4) & 0x02020202u;
+                        const uint32_t t6 = (w >> 5) & 0x02020202u;
+                        const uint32_t t7 = (w >> 6) & 0x02020202u;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(bc + dst_off[i]), "r"(t0),
+                                     "r"(t1), "r"(t2), "r"(t3)
+                                     : "memory");
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(bc + (dst_off[i] ^ 16u)),
+                                     "r"(t4), "r"(t5), "r"(t6), "r"(t7)
+                                     : "memory");
+                    }
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&h.unpacked[s]);
@@ -327,7 +359,8 @@ size_t gemm_ws_bytes(long long M, long long N, long long K) {
 }
 
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
-                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st) {
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits) {
+    if (wbits != 1 && wbits != 2) return cudaErrorInvalidValue;
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     if (dev.max_smem_optin < GEMM_SMEM) return cudaErrorNotSupported;
@@ -343,9 +376,10 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
             return cudaErrorInvalidValue;
     }
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
-        const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t box[2] = {BK / 16, BN};
+        // row of K * wbits / 8 bytes; a box of one K-block (BK * wbits / 32 words) x BN rows
+        const cuuint64_t dims[2] = {(cuuint64_t)(K * wbits / 32), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K * wbits / 8)};
+        const cuuint32_t box[2] = {(cuuint32_t)(BK * wbits / 32), BN};
         const cuuint32_t estr[2] = {1, 1};
         if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(W_p), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -370,9 +404,10 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     p.num_kb = (K + BK - 1) / BK;
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = std::max(1, std::min(tiles, dev.num_sms));
-    e = ensure_smem_optin(reinterpret_cast<const void*>(gemm_kernel), GEMM_SMEM);
+    auto kernel = wbits == 2 ? gemm_kernel<2> : gemm_kernel<1>;
+    e = ensure_smem_optin(reinterpret_cast<const void*>(kernel), GEMM_SMEM);
     if (e != cudaSuccess) return e;
-    return launch_pdl(gemm_kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
+    return launch_pdl(kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
 }
 
 }  // namespace bl

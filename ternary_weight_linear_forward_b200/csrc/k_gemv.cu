@@ -57,6 +57,7 @@ struct GemvParams {
     const float* beta;
     void* y;
     int M, K, N, mode, x_mode;
+    int rb;            // bytes per packed weight row: K / 4 (2-bit trits) or K / 8 (1-bit signs)
     int rpc;           // packed rows per chunk (a power of two)
     int rpc_shift;     // log2(rpc)
     int reuse;         // 0: every chunk has its own ring slot (slot = chunk, parity 0)
@@ -108,6 +109,36 @@ __device__ __forceinline__ int combine4(int a0, int a1, int a2, int a3) {
     return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);  // each a_s is a multiple of 4^s
 }
 
+// 1-bit weights (unite.ai page, "Gewichtsbinarisierung"): the sign of
+// k = 32j + 4s + b is bit 8b + s of word j (set for +1).  Masking with
+// 0x01010101 << s leaves 2^s * bit in the four bytes; the upper half
+// (s = 4..7) is brought down by one shift of the word, so four chains of
+// 2^s * sum(bit * x) cover the 32 weights.  x0 holds x of k = 32j .. 32j+15
+// (int s = k 4s .. 4s+3) and x1 of k = 32j+16 .. 32j+31.
+__device__ __forceinline__ void bits_dot(uint32_t w, const int4& x0, const int4& x1, int& a0, int& a1, int& a2,
+                                         int& a3) {
+    a0 = dp4a_us(w & 0x01010101u, x0.x, a0);
+    a1 = dp4a_us(w & 0x02020202u, x0.y, a1);
+    a2 = dp4a_us(w & 0x04040404u, x0.z, a2);
+    a3 = dp4a_us(w & 0x08080808u, x0.w, a3);
+    const uint32_t h = w >> 4;
+    a0 = dp4a_us(h & 0x01010101u, x1.x, a0);
+    a1 = dp4a_us(h & 0x02020202u, x1.y, a1);
+    a2 = dp4a_us(h & 0x04040404u, x1.z, a2);
+    a3 = dp4a_us(h & 0x08080808u, x1.w, a3);
+}
+
+__device__ __forceinline__ int combine_bits(int a0, int a1, int a2, int a3) {
+    return a0 + (a1 >> 1) + (a2 >> 2) + (a3 >> 3);  // each a_s is a multiple of 2^s
+}
+
+// Row result from the contraction with the stored codes: ternary codes
+// c = w + 1 give sum c x - sum x; sign bits give 2 sum bit x - sum x.
+template <int WB>
+__device__ __forceinline__ int finish_acc(int dot, int rowsum) {
+    return WB == 2 ? dot - rowsum : 2 * dot - rowsum;
+}
+
 // Ring slot and phase parity of chunk c.  Without reuse the whole slab fits
 // (slot = c, first phase); otherwise slots cycle through the ring.
 __device__ __forceinline__ int chunk_slot(const GemvParams& p, int c) { return p.reuse ? c % p.stages : c; }
@@ -119,7 +150,7 @@ __device__ __forceinline__ uint32_t chunk_parity(const GemvParams& p, int c) {
 // into the ring (a chunk is rpc rows; chunk c goes to slot c % stages).
 __device__ __forceinline__ void produce(const GemvParams& p, Shared& sh, unsigned char* ring, int r0, int nrows,
                                         int c0, int c1) {
-    const int RB = p.K / 4;
+    const int RB = p.rb;
     const uint64_t pol = policy_evict_first();
     const unsigned char* src = reinterpret_cast<const unsigned char*>(p.W_p) + (long long)r0 * RB;
     for (int c = c0; c < c1; ++c) {
@@ -155,7 +186,7 @@ __device__ __forceinline__ void release_row(const GemvParams& p, Shared& sh, int
 __device__ __forceinline__ const uint4* row_ptr(const GemvParams& p, const unsigned char* ring, int i) {
     const int c = i >> p.rpc_shift;
     return reinterpret_cast<const uint4*>(ring + (size_t)chunk_slot(p, c) * p.stage_stride +
-                                          (size_t)(i & (p.rpc - 1)) * (p.K / 4));
+                                          (size_t)(i & (p.rpc - 1)) * p.rb);
 }
 
 __device__ __forceinline__ void cta_rows(const GemvParams& p, int cta, int ncta, int& r0, int& nrows) {
@@ -181,16 +212,19 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// 16-byte chunk c of a token's x_q row is stored at slot c ^ ((c >> 3) & 3):
-// lane l of a team reads chunks 4l + q, which this maps to distinct bank groups.
-__device__ __forceinline__ int xq_slot(int c) { return c ^ ((c >> 3) & 3); }
+// 16-byte chunk c of a token's x_q row is stored at slot c ^ ((c >> 3) & 3)
+// for 2-bit weights, where lane l of a team reads chunks 4l + q, and at slot
+// c ^ ((c >> 3) & 7) for 1-bit weights, where it reads chunks 8l + q: either
+// way the eight lanes of one shared-memory phase hit distinct bank groups.
+template <int WB>
+__device__ __forceinline__ int xq_slot(int c) { return c ^ ((c >> 3) & (WB == 2 ? 3 : 7)); }
 
 // Fill the shared x_q rows (tokens 0..MT-1; tokens >= M are zero), rowsum[]
 // and fscale[].  Runs on the consumer threads only.  The first XC chunks per
 // token of every thread are loaded at once into registers and serve both the
 // absmax pass and the quantisation pass, so the stage costs one memory round
 // trip (x was just written by the preceding kernel and sits in L2).
-template <int MT, int XM>
+template <int MT, int XM, int WB>
 __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& sh, int4* xsm, int ctid, int cthreads,
                                                   int cwarps) {
     const int G = p.K / 16;  // 16-byte chunks per token
@@ -265,7 +299,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
                     q = chunk_codes<XM>(cache[m][i], s[m]);
                     rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
                 }
-                dst[xq_slot(g)] = q;
+                dst[xq_slot<WB>(g)] = q;
             }
         }
         for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
@@ -276,7 +310,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
                 q = chunk_codes<XM>(c, s[m]);
                 rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
             }
-            dst[xq_slot(g)] = q;
+            dst[xq_slot<WB>(g)] = q;
         }
     }
 #pragma unroll
@@ -328,7 +362,7 @@ __device__ __forceinline__ int team_reduce(const int (&v)[V], int tl, int& which
 // ---------------------------------------------------------------- M <= 4
 
 // One CTA's share (CTA `cta` of `ncta` working on problem p) of the M <= 4 forward.
-template <int LPR, int MT, int R, int XM>
+template <int LPR, int MT, int R, int XM, int WB>
 __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, int ncta, unsigned char* smem) {
     Shared& sh = *reinterpret_cast<Shared*>(smem);
     int4* xsm = reinterpret_cast<int4*>(smem + GEMV_HDR);
@@ -365,14 +399,14 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
     }
     pdl_wait();
     const int ctid = threadIdx.x - 32;
-    stage_activations<MT, XM>(p, sh, xsm, ctid, cthreads, cwarps);
+    stage_activations<MT, XM, WB>(p, sh, xsm, ctid, cthreads, cwarps);
 
     constexpr int V = R * MT;
     const int T = cthreads / LPR;  // teams
     const int team = ctid / LPR;
     const int tl = ctid % LPR;
-    const int K4 = p.K / 64;  // 16-byte groups of packed weights per row
-    const int G = p.K / 16;   // 16-byte chunks of x_q per token
+    const int K4 = p.rb / 16;  // 16-byte groups of packed weights per row
+    const int G = p.K / 16;    // 16-byte chunks of x_q per token
     const int KS = p.ks;
     // work item = (group of R rows, K slice); warp-uniform trip count
     const int items = (nrows + R - 1) / R * KS;
@@ -410,17 +444,36 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
                 const int nxt = idx + LPR < k_hi ? idx + LPR : idx;
 #pragma unroll
                 for (int r = 0; r < R; ++r) wn[r] = *reinterpret_cast<const uint4*>(ring + ro[r] + 16 * nxt);
-                const int key = (idx >> 1) & 3;  // swizzle of chunks 4 idx .. 4 idx + 3
-                const int4* xb = xsm + 4 * idx;
+                if constexpr (WB == 2) {
+                    const int key = (idx >> 1) & 3;  // swizzle of chunks 4 idx .. 4 idx + 3
+                    const int4* xb = xsm + 4 * idx;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 4; ++q) {
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        const int4 xv = xb[m * G + (q ^ key)];
+                        for (int m = 0; m < MT; ++m) {
+                            const int4 xv = xb[m * G + (q ^ key)];
 #pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            const uint32_t wq = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
-                            word_dot(wq, xv.x, xv.y, xv.z, xv.w, a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
+                            for (int r = 0; r < R; ++r) {
+                                const uint32_t wq = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+                                word_dot(wq, xv.x, xv.y, xv.z, xv.w, a[r][m][0], a[r][m][1], a[r][m][2],
+                                         a[r][m][3]);
+                            }
+                        }
+                    }
+                } else {
+                    const int key = idx & 7;  // swizzle of chunks 8 idx .. 8 idx + 7
+                    const int4* xb = xsm + 8 * idx;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+                            const int4 x0 = xb[m * G + ((2 * q) ^ key)];
+                            const int4 x1 = xb[m * G + ((2 * q + 1) ^ key)];
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                const uint32_t wq = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+                                bits_dot(wq, x0, x1, a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
+                            }
                         }
                     }
                 }
@@ -430,7 +483,9 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int m = 0; m < MT; ++m) vals[r * MT + m] = combine4(a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
+            for (int m = 0; m < MT; ++m)
+                vals[r * MT + m] = WB == 2 ? combine4(a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3])
+                                           : combine_bits(a[r][m][0], a[r][m][1], a[r][m][2], a[r][m][3]);
         int which;
         const int tot = team_reduce<LPR, V>(vals, tl, which);
         // lane tl = which * (LPR / V) is the first lane that owns value `which`
@@ -439,7 +494,7 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
             if (r < nvalid) {
                 if (m == 0) release_row(p, sh, b + r);
                 if (KS == 1) {
-                    if (m < p.M) store_y(p, m, r0 + b + r, tot - sh.rowsum[m], sh.fscale[m]);
+                    if (m < p.M) store_y(p, m, r0 + b + r, finish_acc<WB>(tot, sh.rowsum[m]), sh.fscale[m]);
                 } else {
                     atomicAdd(&sh.part[b + r][m], tot);
                 }
@@ -455,15 +510,15 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
         consumer_sync(cthreads);
         for (int i = ctid; i < nrows * MT; i += cthreads) {
             const int r = i / MT, m = i % MT;
-            if (m < p.M) store_y(p, m, r0 + r, sh.part[r][m] - sh.rowsum[m], sh.fscale[m]);
+            if (m < p.M) store_y(p, m, r0 + r, finish_acc<WB>(sh.part[r][m], sh.rowsum[m]), sh.fscale[m]);
         }
     }
 }
 
-template <int LPR, int MT, int R, int XM>
+template <int LPR, int MT, int R, int XM, int WB>
 __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_small_kernel(const GemvParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    gemv_small_body<LPR, MT, R, XM>(p, blockIdx.x, gridDim.x, smem);
+    gemv_small_body<LPR, MT, R, XM, WB>(p, blockIdx.x, gridDim.x, smem);
 }
 
 // Several independent problems (same M, same x / y formats) in one launch:
@@ -485,11 +540,11 @@ __global__ void __launch_bounds__(GEMV_MAX_THREADS, GEMV_CO_RESIDENT) gemv_group
     while (i + 1 < g.count && (int)blockIdx.x >= g.cta0[i + 1]) ++i;
     const int cta = blockIdx.x - g.cta0[i], ncta = g.cta0[i + 1] - g.cta0[i];
     if (g.lpr[i] == 32)
-        gemv_small_body<32, MT, R, XM>(g.prob[i], cta, ncta, smem);
+        gemv_small_body<32, MT, R, XM, 2>(g.prob[i], cta, ncta, smem);
     else if (g.lpr[i] == 16)
-        gemv_small_body<16, MT, R, XM>(g.prob[i], cta, ncta, smem);
+        gemv_small_body<16, MT, R, XM, 2>(g.prob[i], cta, ncta, smem);
     else
-        gemv_small_body<8, MT, R, XM>(g.prob[i], cta, ncta, smem);
+        gemv_small_body<8, MT, R, XM, 2>(g.prob[i], cta, ncta, smem);
 }
 
 // ------------------------------------------------------------ 4 < M <= 64
@@ -588,28 +643,35 @@ cudaError_t launch_with_smem(KernelT kernel, int grid, int threads, size_t smem,
 using GemvKernel = void (*)(const GemvParams);
 using GroupKernel = void (*)(const GroupParams);
 
-template <int LPR, int XM>
+template <int LPR, int XM, int WB>
 GemvKernel small_kernel_for(int mt, int r) {
-    if (mt == 1 && r == 1) return gemv_small_kernel<LPR, 1, 1, XM>;
-    if (mt == 1 && r == 2) return gemv_small_kernel<LPR, 1, 2, XM>;
-    if (mt == 1 && r == 4) return gemv_small_kernel<LPR, 1, 4, XM>;
-    if (mt == 2 && r == 1) return gemv_small_kernel<LPR, 2, 1, XM>;
-    if (mt == 2 && r == 2) return gemv_small_kernel<LPR, 2, 2, XM>;
-    return gemv_small_kernel<LPR, 4, 1, XM>;
+    if (mt == 1 && r == 1) return gemv_small_kernel<LPR, 1, 1, XM, WB>;
+    if (mt == 1 && r == 2) return gemv_small_kernel<LPR, 1, 2, XM, WB>;
+    if (mt == 1 && r == 4) return gemv_small_kernel<LPR, 1, 4, XM, WB>;
+    if (mt == 2 && r == 1) return gemv_small_kernel<LPR, 2, 1, XM, WB>;
+    if (mt == 2 && r == 2) return gemv_small_kernel<LPR, 2, 2, XM, WB>;
+    return gemv_small_kernel<LPR, 4, 1, XM, WB>;
 }
 
-template <int XM>
+template <int XM, int WB>
 GemvKernel small_kernel_for(int lpr, int mt, int r) {
-    if (lpr == 32) return small_kernel_for<32, XM>(mt, r);
-    if (lpr == 16) return small_kernel_for<16, XM>(mt, r);
-    return small_kernel_for<8, XM>(mt, r);
+    if (lpr == 32) return small_kernel_for<32, XM, WB>(mt, r);
+    if (lpr == 16) return small_kernel_for<16, XM, WB>(mt, r);
+    return small_kernel_for<8, XM, WB>(mt, r);
+}
+
+template <int WB>
+GemvKernel small_kernel_for_mode(int x_mode, int lpr, int mt, int r) {
+    return x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED, WB>(lpr, mt, r)
+           : x_mode == X_F32     ? small_kernel_for<X_F32, WB>(lpr, mt, r)
+                                 : small_kernel_for<X_BF16, WB>(lpr, mt, r);
 }
 
 // Ring geometry for a CTA slab of `rows_per_cta` rows and `ring_bytes` of
 // space: chunks of a power-of-two number of rows (about 8 KiB), one slot per
 // chunk when the slab fits, otherwise a ring of as many slots as fit.
 void ring_geometry(GemvParams& p, int rows_per_cta, int ring_bytes) {
-    const int RB = p.K / 4;
+    const int RB = p.rb;
     const int cap = std::max(1, std::min(rows_per_cta, GEMV_CHUNK_TARGET / RB));
     p.rpc_shift = 0;
     while ((2 << p.rpc_shift) <= cap) ++p.rpc_shift;
@@ -634,7 +696,7 @@ SmallShape configure_small(GemvParams& p, const DevInfo& dev, int co_resident) {
     const int K = p.K, N = p.N;
     const int grid = std::max(1, std::min(N, dev.num_sms));
     const int rows_per_cta = (N + grid - 1) / grid;
-    const int K4 = K / 64;
+    const int K4 = p.rb / 16;  // 16-byte groups of packed weights per row
     const int mt = small_mt(p.M);
     // Launch shape (measured on B200 over lanes-per-row x rows-per-team x
     // K-slices x warps for the 4096x11008 and 11008x4096 decode shapes):
@@ -660,7 +722,7 @@ SmallShape configure_small(GemvParams& p, const DevInfo& dev, int co_resident) {
     p.xq_bytes = (mt * K + 127) / 128 * 128;
     // leave room for the other CTAs on the same SM
     const int budget = (dev.max_smem_optin - 1024) / co_resident;
-    const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * (K / 4));
+    const int ring_bytes = std::max(budget - GEMV_HDR - p.xq_bytes, 2 * p.rb);
     ring_geometry(p, rows_per_cta, ring_bytes);
     if (p.reuse) {
         // one team per warp, and the rows of one iteration (ceil(teams / ks) * r)
@@ -694,9 +756,7 @@ cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st)
     if (small_ok(M, p.K)) {
         const SmallShape sh = configure_small(p, dev, GEMV_CO_RESIDENT);
         const int mt = small_mt(M);
-        GemvKernel k = p.x_mode == X_QUANTISED ? small_kernel_for<X_QUANTISED>(sh.lpr, mt, sh.r)
-                       : p.x_mode == X_F32     ? small_kernel_for<X_F32>(sh.lpr, mt, sh.r)
-                                               : small_kernel_for<X_BF16>(sh.lpr, mt, sh.r);
+        GemvKernel k = small_kernel_for_mode<2>(p.x_mode, sh.lpr, mt, sh.r);
         return launch_with_smem(k, sh.grid, (sh.cwarps + 1) * 32, sh.smem, st, p);
     }
     if (p.x_mode != X_QUANTISED) return cudaErrorInvalidValue;  // callers quantise first
@@ -733,6 +793,7 @@ GemvParams make_params(const int8_t* x_q, const float* gamma, int M, int K, cons
     p.N = N;
     p.mode = mode;
     p.x_mode = X_QUANTISED;
+    p.rb = K / 4;
     return p;
 }
 
@@ -788,6 +849,26 @@ cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, 
     cudaError_t e = ensure_smem_optin(reinterpret_cast<const void*>(k), smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(k, dim3(cta), dim3(threads), smem, st, g);
+}
+
+bool gemv_bits_ok(long long M, long long K) { return gemv_fused_quant_ok(M, K); }
+
+cudaError_t launch_gemv_bits(const void* x, int x_dtype, const float* gamma, int M, int K, const uint32_t* W_p,
+                             const float* beta, int N, void* y, YMode mode, const DevInfo& dev, cudaStream_t st) {
+    // x_dtype: 0 fp32, 1 bf16 (quantiser fused), 2 int8 x_q with gamma
+    if (!small_ok(M, K)) return cudaErrorInvalidValue;
+    GemvParams p = make_params(nullptr, nullptr, M, K, W_p, beta, N, y, mode);
+    p.rb = K / 8;
+    if (x_dtype == 2) {
+        p.x_q = static_cast<const int8_t*>(x);
+        p.gamma = gamma;
+    } else {
+        p.x = x;
+        p.x_mode = x_dtype == 1 ? X_BF16 : X_F32;
+    }
+    const SmallShape sh = configure_small(p, dev, GEMV_CO_RESIDENT);
+    GemvKernel k = small_kernel_for_mode<1>(p.x_mode, sh.lpr, small_mt(M), sh.r);
+    return launch_with_smem(k, sh.grid, (sh.cwarps + 1) * 32, sh.smem, st, p);
 }
 
 cudaError_t launch_gemv_fused(const void* x, bool bf16, int M, int K, const uint32_t* W_p, const float* beta, int N,

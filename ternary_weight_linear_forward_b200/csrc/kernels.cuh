@@ -26,6 +26,10 @@ size_t quantize_weights_ws_bytes();
 cudaError_t launch_quantize_weights(const float* W, long long n, float eps, int8_t* W_t, float* beta, void* ws,
                                     int num_sms, cudaStream_t st);
 cudaError_t launch_pack(const int8_t* W_t, long long nwords, uint32_t* W_p, int num_sms, cudaStream_t st);
+size_t binarize_weights_ws_bytes();
+cudaError_t launch_binarize_weights(const float* W, long long n, int8_t* W_b, float* alpha, float* beta, void* ws,
+                                    int num_sms, cudaStream_t st);
+cudaError_t launch_pack_bits(const int8_t* W_b, long long nwords, uint32_t* W_p, int num_sms, cudaStream_t st);
 
 // k_act.cu
 cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
@@ -40,6 +44,11 @@ cudaError_t launch_gemv(const int8_t* x_q, const float* gamma, int M, int K, con
 bool gemv_fused_quant_ok(long long M, long long K);
 cudaError_t launch_gemv_fused(const void* x, bool bf16, int M, int K, const uint32_t* W_p, const float* beta, int N,
                               void* y, YMode mode, const DevInfo& dev, cudaStream_t st);
+// 1-bit weights (K / 32 words per row), M <= 4 with the x_q staging of the
+// fused quantiser; x_dtype 0 fp32, 1 bf16, 2 int8 x_q with gamma
+bool gemv_bits_ok(long long M, long long K);
+cudaError_t launch_gemv_bits(const void* x, int x_dtype, const float* gamma, int M, int K, const uint32_t* W_p,
+                             const float* beta, int N, void* y, YMode mode, const DevInfo& dev, cudaStream_t st);
 
 struct GemvProblem {
     const void* x;
@@ -63,10 +72,10 @@ cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_d
 enum DecodePath : int { PATH_CUDA = 0, PATH_TC = 1, PATH_GEMM = 2 };
 DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev);
 
-// k_gemm.cu  (M > 64, tcgen05 int8 tensor cores)
+// k_gemm.cu  (M > 64, tcgen05 int8 tensor cores); wbits 2 (trits) or 1 (signs)
 size_t gemm_ws_bytes(long long M, long long N, long long K);
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
-                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st);
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits = 2);
 
 // Raise a kernel's dynamic shared-memory limit once per device (api.cu).
 cudaError_t ensure_smem_optin(const void* kernel, size_t bytes);

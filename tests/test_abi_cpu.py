@@ -179,3 +179,50 @@ def test_forward_fp_batch_validation():
     assert f(pa, 2, 1, 0, 0, None) == SHAPE
     arr[1].K = 1024
     assert f(pa, 2, 1, 0, 0, None) == DEVICE
+
+
+def test_binary_weight_calls_validation():
+    f = _L().bitlinear_binarize_weights
+    ws = _L().bitlinear_binarize_weights_workspace(16, 32)
+    assert ws > 0
+    assert f(None, 16, 32, P(A2), P(A3), P(A3 + 16), P(A4), ws, None) == NULL
+    assert f(P(A1), 16, 48, P(A2), P(A3), P(A3 + 16), P(A4), ws, None) == SHAPE     # K % 32
+    assert f(P(A1), 16, 32, P(A2), P(A3), P(A3 + 16), P(A4), ws - 1, None) == WS
+    assert f(P(A1), 16, 32, P(A2), P(A3 + 4), P(A3 + 16), P(A4), ws, None) == ALIGN
+    assert f(P(A1), 16, 32, P(A2), P(A3), P(A3), P(A4), ws, None) == ALIAS           # alpha is beta
+    assert f(P(A1), 16, 32, P(A1), P(A3), P(A3 + 16), P(A4), ws, None) == ALIAS      # W_b on W
+    assert f(P(A1), 16, 32, P(A2), P(A3), P(A3 + 16), P(A2), ws, None) == ALIAS      # ws on W_b
+    assert f(P(A1), 16, 32, P(A2), P(A3), P(A3 + 16), P(A4), ws, None) == DEVICE
+    pk = _L().bitlinear_pack_bits
+    assert pk(None, 4, 32, P(A2), None) == NULL
+    assert pk(P(A1), 4, 48, P(A2), None) == SHAPE
+    assert pk(P(A1), 4, 32, P(A2 + 4), None) == ALIGN
+    assert pk(P(A1), 4, 32, P(A1), None) == ALIAS
+    assert pk(P(A1), 4, 32, P(A2), None) == DEVICE
+
+
+def test_binary_forward_validation():
+    f = _L().bitlinear_forward_binary
+    assert f(None, P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == NULL
+    assert f(P(A1), P(A2), 1, 1088, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == SHAPE   # K % 128
+    assert f(P(A1), P(A2), 0, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == SHAPE
+    assert f(P(A1), P(A2), 1, 1024, P(A3 + 8), P(A4), 64, P(A5), 0, None, 0, None) == ALIGN
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 5, None, 0, None) == DTYPE
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A3), 0, None, 0, None) == ALIAS
+    # decode shapes need no workspace; the GEMM path (M > 4, or x_hat too large) does
+    assert _L().bitlinear_forward_binary_workspace(4, 4096, 4096) == 0
+    assert _L().bitlinear_forward_binary_workspace(4, 4096, 32768) >= 16
+    assert _L().bitlinear_forward_binary_workspace(2048, 4096, 4096) >= 2048 * 4
+    assert f(P(A1), P(A2), 2048, 1024, P(A3), P(A4), 64, P(A5), 1, None, 0, None) == WS
+    assert f(P(A1), P(A2), 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DEVICE
+    g = _L().bitlinear_forward_binary_acc
+    assert g(P(A1), 1, 1088, P(A3), 64, P(A5), None, 0, None) == SHAPE
+    assert g(P(A1), 1, 1024, P(A3), 64, P(A5), None, 0, None) == DEVICE
+    h = _L().bitlinear_forward_binary_fp
+    assert h(P(A1), 3, 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DTYPE
+    assert h(P(A1), 0, 1, 1088, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == SHAPE
+    assert _L().bitlinear_forward_binary_fp_workspace(1, 4096, 4096) == 0
+    need = _L().bitlinear_forward_binary_fp_workspace(64, 4096, 4096)
+    assert need >= 64 * 4096 + 64 * 4
+    assert h(P(A1), 0, 64, 4096, P(A3), P(A4), 64, P(A5), 0, P(A6), need - 1, None) == WS
+    assert h(P(A1), 0, 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DEVICE
