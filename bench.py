@@ -208,8 +208,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="run the decode step only (no extra sections)")
+    ap.add_argument("--sections", default="prefill,small,block,binary",
+                    help="extra measured sections after the decode step, comma separated")
     args = ap.parse_args()
+    sections = set() if args.no_prefill else {x for x in args.sections.split(",") if x}
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
@@ -390,7 +393,7 @@ def main():
 
     # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
     prefill = None
-    if not args.no_prefill:
+    if "prefill" in sections:
         prefill = {}
         int8_peak_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
         for s in workloads.W4.shapes:
@@ -424,7 +427,7 @@ def main():
 
     # ---- small-batch decode (M = 4, 16, 64; K = 4096; N = 4096, 11008) ----
     small = None
-    if not args.no_prefill:
+    if "small" in sections:
         small = {}
         for s in workloads.W3.shapes:
             W = torch.from_numpy(s.weights()).to(dev)
@@ -455,7 +458,7 @@ def main():
 
     # ---- decoder block at batch-1 decode (hidden 2560, intermediate 6912) ----
     block = None
-    if not args.no_prefill:
+    if "block" in sections:
         bw = {p: torch.from_numpy(w).to(dev) for p, w in workloads.block_weights().items()}
         nblk = max(2, int(1.2 * L2 // sum(w.numel() // 4 for w in bw.values())) + 1)   # >= 1.2x L2 of weights
         blocks = [bl.DecoderBlock.from_float(bw) for _ in range(nblk)]
@@ -482,7 +485,7 @@ def main():
 
     # ---- 1-bit weights (Sign(W - mean W)): decode GEMV and prefill GEMM ----
     binary = None
-    if not args.no_prefill:
+    if "binary" in sections:
         binary = {}
         for s in workloads.W2.shapes:
             W_b, _, beta = bl.binarize_weights(torch.from_numpy(s.weights()).to(dev))
