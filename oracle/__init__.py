@@ -11,7 +11,8 @@ Each function states the passage it follows.  Sources (web pages):
   multiplies become negate/zero/pass-through.  Figure item "RMS norm" --
   activations are normalised before quantisation.  Section "Kerncomponenten:
   MLGRU en GLU" -- the MatMul-free GLU (two BitLinears, SiLU, elementwise
-  product, a third BitLinear).
+  product, a third BitLinear): ``glu`` for any number of tokens, and the
+  decoder block at batch-1 decode.
 * unite.ai "Microsofts Inference Framework bringt 1-Bit grosse Sprachmodelle
   auf lokale Geraete" (German), section "Mathematische Grundlagen", eq. 2
   "Aktivierungsquantisierung" and eq. 3 "BitLinear-Betrieb"; item 1
@@ -308,3 +309,28 @@ def block_decode(x: np.ndarray, tern: dict) -> dict:
                x_q_o=o["x_q"], x_q_mlp=gate["x_q"], x_q_down=down["x_q"],
                acc_down=down["acc"])
     return out
+
+
+# ---------------------------------------------------------------------------
+# MatMul-free GLU channel mixer, any number of tokens.
+# ---------------------------------------------------------------------------
+
+def glu(x: np.ndarray, tern: dict) -> dict:
+    """The MatMul-free GLU of the MatMul-free blog, section "Kerncomponenten:
+    MLGRU en GLU": the input goes through two separate BitLinear layers, SiLU
+    of one output is multiplied elementwise by the other, and the gated result
+    goes through a third BitLinear.  Every BitLinear input is RMS-normalised
+    before quantisation (figure item "RMS norm"), token by token.
+    ``tern[p] = (W_t, beta)`` for p in gate, up ([F, D]) and down ([D, F])."""
+    x = _c(x, np.float32)
+    out = {k: [] for k in ("x_q", "gamma", "gate", "up", "u", "u_q", "gamma_u", "acc_down", "y")}
+    for m in range(x.shape[0]):
+        gate = bitlinear_rms(x[m], *tern["gate"])
+        up = bitlinear_rms(x[m], *tern["up"])
+        u = silu_mul(gate["y"], up["y"])
+        down = bitlinear_rms(u, *tern["down"])
+        for k, v in (("x_q", gate["x_q"][0]), ("gamma", gate["gamma"][0]), ("gate", gate["y"][0]),
+                     ("up", up["y"][0]), ("u", u), ("u_q", down["x_q"][0]), ("gamma_u", down["gamma"][0]),
+                     ("acc_down", down["acc"][0]), ("y", down["y"][0])):
+            out[k].append(v)
+    return {k: np.stack(v) for k, v in out.items()}

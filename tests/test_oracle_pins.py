@@ -350,3 +350,55 @@ def test_block_decode_structure():
     np.testing.assert_array_equal(r["h1"], (x + r["o"]).astype(np.float32))
     xq_u, _ = oracle.quant_act(r["u"])
     np.testing.assert_array_equal(r["x_q_down"], xq_u)
+
+
+# --------------------------------------------------------------------------
+# MatMul-free GLU (composition of pinned parts): structural pins
+# --------------------------------------------------------------------------
+
+def _glu_weights(D, F, seed):
+    return {p: oracle.quantize_weights(workloads.latent_weights(seed + i, *shape))
+            for i, (p, shape) in enumerate((("gate", (F, D)), ("up", (F, D)), ("down", (D, F))))}
+
+
+def test_glu_zero_gate_gives_zero():
+    # W_gate = 0: gate = 0, SiLU(0) = 0, u = 0, its codes 0, y = 0 exactly
+    D, F = 128, 192
+    tern = _glu_weights(D, F, 70)
+    tern["gate"] = (np.zeros((F, D), np.int8), tern["gate"][1])
+    r = oracle.glu(workloads.activations(71, 3, D, outliers=True), tern)
+    assert not r["gate"].any() and not r["u"].any() and not r["u_q"].any() and not r["y"].any()
+
+
+def test_glu_odd_in_up_and_down():
+    # -W_up negates u exactly (binary64 product, symmetric rounding) and so y;
+    # -W_down negates y exactly; the codes of x are untouched
+    D, F = 256, 320
+    tern = _glu_weights(D, F, 80)
+    x = workloads.activations(81, 2, D, outliers=True)
+    r = oracle.glu(x, tern)
+    neg_up = dict(tern, up=(-tern["up"][0], tern["up"][1]))
+    r2 = oracle.glu(x, neg_up)
+    np.testing.assert_array_equal(r2["u"], -r["u"])
+    np.testing.assert_array_equal(r2["y"], -r["y"])
+    neg_down = dict(tern, down=(-tern["down"][0], tern["down"][1]))
+    np.testing.assert_array_equal(oracle.glu(x, neg_down)["y"], -r["y"])
+
+
+def test_glu_tokens_are_independent_and_match_the_block():
+    D, F = 128, 256
+    tern = _glu_weights(D, F, 90)
+    x = workloads.activations(91, 4, D, outliers=True)
+    r = oracle.glu(x, tern)
+    for m in range(4):
+        rm = oracle.glu(x[m:m + 1], tern)
+        for k in ("gate", "up", "u", "y"):
+            np.testing.assert_array_equal(rm[k][0], r[k][m])
+    # the block's MLP half is the GLU of h1
+    blk = {p: tern[p] for p in ("gate", "up", "down")}
+    blk.update({p: oracle.quantize_weights(workloads.latent_weights(95 + i, D, D))
+                for i, p in enumerate(("q", "k", "v", "o"))})
+    ref = oracle.block_decode(x[0], blk)
+    g = oracle.glu(ref["h1"], tern)
+    for k, kb in (("gate", "gate"), ("up", "up"), ("u", "u"), ("y", "down")):
+        np.testing.assert_array_equal(g[k].ravel(), np.asarray(ref[kb]).ravel())
