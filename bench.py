@@ -13,8 +13,12 @@ step reads its weights from HBM (working set > L2).
 Printed metric: algorithmic GB/s (packed weights + activations + outputs per
 step / step time), whole job over all ranks, plus the roofline of the GEMV
 against the measured HBM copy bandwidth, the CPU oracle timed on the host,
-an end-to-end figure through the public API with host buffers, the prefill
-GEMM (M = 2048) in int8 TOPS against the int8 tensor peak, and SM clocks.
+an end-to-end figure through the public API with host buffers (per step one
+H2D copy, one call, one D2H copy, recorded in CUDA graphs; the same sequence
+issued eagerly is reported beside it), and SM clocks.  Extra sections
+(--sections): the prefill GEMM (M = 2048) in int8 TOPS against the int8
+tensor peak, small-batch decode, a decoder block, the 1-bit weight variant
+(decode GEMV and prefill GEMM) and the MatMul-free GLU channel mixer.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -209,7 +213,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="run the decode step only (no extra sections)")
-    ap.add_argument("--sections", default="prefill,small,block,binary",
+    ap.add_argument("--sections", default="prefill,small,block,binary,glu",
                     help="extra measured sections after the decode step, comma separated")
     args = ap.parse_args()
     sections = set() if args.no_prefill else {x for x in args.sections.split(",") if x}
@@ -368,28 +372,63 @@ def main():
             dev_xcat.copy_(host_x, non_blocking=True)
             plans[i % copies].run(stream=stream)
             host_y.copy_(ycat, non_blocking=True)
+
+    def e2e_timed(fn):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3
+        if world > 1:
+            t_ = torch.tensor([t], device=dev)
+            dist.all_reduce(t_, op=dist.ReduceOp.MAX)
+            t = float(t_.item())
+        return t
+
+    def e2e_eager():
+        for i in range(n_e2e):
+            e2e_step(i)
+
+    # The same per-step sequence (H2D copy, library call, D2H copy) recorded in
+    # CUDA graphs of at most CHUNK steps and replayed: the copies still run
+    # every step, the host no longer issues them one by one.
+    def e2e_graphs(n):
+        gs, done = [], 0
+        while done < n:
+            k = min(CHUNK, n - done)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(k):
+                        e2e_step(done + i)
+            gs.append(g)
+            done += k
+        return gs
+
     for i in range(4):
         e2e_step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(n_e2e):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_e2e = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([t_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_e2e = float(t.item())
+    t_eager = e2e_timed(e2e_eager)
+    eg = e2e_graphs(n_e2e)
+    with torch.cuda.stream(stream):
+        run(e2e_graphs(8))
+    def e2e_replay():
+        with torch.cuda.stream(stream):
+            run(eg)
+    t_e2e = e2e_timed(e2e_replay)
+    del eg
     e2e = {"value": world * step_bytes() * n_e2e / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "steps": n_e2e,
-           "path": "one pinned H2D copy of both inputs + bitlinear_forward_fp_batch (both projections, descriptors "
-                   "marshalled once per weight copy) + one D2H copy of both outputs; one stream, no graph; weights "
-                   f"rotate over {copies} copies"}
+           "d2h_bytes_per_step": d2h, "steps": n_e2e, "us_per_step": t_e2e / n_e2e * 1e6,
+           "path": "per step: one pinned H2D copy of both inputs + bitlinear_forward_fp_batch (both projections, "
+                   "descriptors marshalled once per weight copy) + one D2H copy of both outputs into pinned memory, "
+                   f"recorded in CUDA graphs of <= {CHUNK} steps and replayed; weights rotate over {copies} copies",
+           "eager": {"value": world * step_bytes() * n_e2e / t_eager / 1e9, "us_per_step": t_eager / n_e2e * 1e6,
+                     "path": "the same three operations issued from the host every step, no graph"}}
 
     # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
     prefill = None
@@ -538,6 +577,48 @@ def main():
                                            "path": "tcgen05 GEMM, 1-bit unpack"}
             del g, W_p, x_q, y, ws
 
+    # ---- MatMul-free GLU channel mixer (hidden 2560, intermediate 6912) ----
+    glu = None
+    if "glu" in sections:
+        glu = {}
+        D, F = 2560, 6912
+        gw = {p: workloads.latent_weights(1060 + i, *shape)
+              for i, (p, shape) in enumerate((("gate", (F, D)), ("up", (F, D)), ("down", (D, F))))}
+        base = {p: bl.BitLinear.from_float(torch.from_numpy(w).to(dev)) for p, w in gw.items()}
+        del gw
+        wbytes = sum(L.W_p.numel() * 4 for L in base.values())
+        for M in (1, 2048):
+            nc = max(2, int(4 * L2 // wbytes) + 1) if M == 1 else 1
+            sets = [base] + [{p: bl.BitLinear(L.W_p.clone(), L.beta) for p, L in base.items()}
+                             for _ in range(nc - 1)]
+            x = torch.from_numpy(workloads.activations(2060, M, D, outliers=True)).to(dev)
+            y = torch.empty((M, D), dtype=torch.float32, device=dev)
+            ws = torch.empty(bl.lib().bitlinear_glu_workspace(M, D, F), dtype=torch.uint8, device=dev)
+            reps = 8 * nc if M == 1 else 10
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    S = sets[i % nc]
+                    bl.glu_forward(x, S["gate"], S["up"], S["down"], out=y, ws=ws, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(reps):
+                        S = sets[i % nc]
+                        bl.glu_forward(x, S["gate"], S["up"], S["down"], out=y, ws=ws, stream=stream)
+            g.replay()
+            t = timed_run([g]) / reps
+            if M == 1:
+                glu["decode_m1"] = {"us_per_call": t * 1e6, "weight_bytes": wbytes, "GB/s": wbytes / t / 1e9,
+                                    "frac_of_hbm": wbytes / t / 1e9 / peaks["hbm_gbs"], "launches": 4,
+                                    "copies": nc}
+            else:
+                ops = 2 * M * 3 * D * F
+                glu["prefill_m2048"] = {"us_per_call": t * 1e6, "TOPS": ops / t / 1e12,
+                                        "frac_of_int8_peak": ops / t / 1e12 / (peaks["bf16_tflops"] * INT8_OVER_BF16),
+                                        "launches": 8}
+            del g, sets, x, y, ws
+        del base
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -559,7 +640,7 @@ def main():
                        "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks, "prefill": prefill, "small_batch": small, "block": block,
-            "binary": binary,
+            "binary": binary, "glu": glu,
             "device": props.name,
         }
         print(json.dumps(line), flush=True)

@@ -354,6 +354,38 @@ enum { BL_COMBINE_NONE = 0, BL_COMBINE_ADD = 1, BL_COMBINE_SILU_MUL = 2 };
 bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, int64_t M, int64_t K,
                                   float* h, int8_t* x_q, float* gamma, void* stream);
 
+/* Bytes of device workspace bitlinear_glu_forward needs for this shape. */
+size_t bitlinear_glu_workspace(int64_t M, int64_t D, int64_t F);
+
+/*
+ * The MatMul-free GLU channel mixer, [MMF] "Kerncomponenten: MLGRU en GLU":
+ * the input goes through two BitLinear layers, SiLU of one output is
+ * multiplied elementwise by the other, and the gated result goes through a
+ * third BitLinear.  Every BitLinear input is RMS-normalised before
+ * quantisation ([MMF] figure item "RMS norm"), as bitlinear_quant_act_rms
+ * does it, token by token:
+ *   (x_q, gamma)   = quant_act_rms(x)                   codes shared by gate and up
+ *   gate, up       = forward(x_q, gamma, W_gate | W_up)  [M, F] float32
+ *   u              = SiLU(gate) * up                    (binary64, rounded once)
+ *   (u_q, gamma_u) = quant_act_rms(u)
+ *   y              = forward(u_q, gamma_u, W_down)       [M, D] float32
+ * Results are bit-identical to those calls made one by one.  For M <= 4
+ * tokens (with M rounded up to 1, 2 or 4, times D <= 65536) gate and up run
+ * in one launch; otherwise each runs on the kernel bitlinear_forward picks.
+ *   x       [M, D] float32 in
+ *   W_gate, W_up [F, D/16] uint32 (bitlinear_pack layout), beta_gate, beta_up [1] float32, in
+ *   W_down  [D, F/16] uint32, beta_down [1] float32, in
+ *   y       [M, D] float32 out
+ *   u       [M, F] float32 out, may be NULL (not written)
+ *   ws      >= bitlinear_glu_workspace(M, D, F) bytes (holds x_q, gate, up, u_q, scales)
+ * D % 64 == 0, F % 64 == 0, D and F <= BL_MAX_K.
+ */
+bl_status bitlinear_glu_forward(const float* x, int64_t M, int64_t D, int64_t F,
+                                const uint32_t* W_gate, const float* beta_gate,
+                                const uint32_t* W_up, const float* beta_up,
+                                const uint32_t* W_down, const float* beta_down,
+                                float* y, float* u, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Decode engine                                                             */
 /* ------------------------------------------------------------------------ */

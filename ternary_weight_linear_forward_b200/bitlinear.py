@@ -41,6 +41,8 @@ SIGNATURES = {
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_glu_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_glu_forward": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_binarize_weights_workspace": (_SZ, [_I64, _I64]),
     "bitlinear_binarize_weights": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_pack_bits": (_I, [_P, _I64, _I64, _P, _P]),
@@ -498,6 +500,31 @@ class BitLinear:
 
     def __call__(self, x: torch.Tensor, out_dtype=torch.float32, out=None) -> torch.Tensor:
         return forward_fp(x, self.W_p, self.beta, out_dtype=out_dtype, out=out)
+
+
+def glu_forward(x: torch.Tensor, gate, up, down, want_u: bool = False, out=None, ws=None, stream=None):
+    """The MatMul-free GLU channel mixer on x [M, D]: down(SiLU(gate(x)) * up(x)),
+    every BitLinear input RMS-normalised.  gate, up and down are BitLinear
+    layers (or (W_p, beta) pairs).  Returns y [M, D], or (y, u) with u [M, F]."""
+    _need(x, torch.float32, 2, "x")
+    (Wg, bg), (Wu, bu), (Wd, bd) = [(L.W_p, L.beta) if isinstance(L, BitLinear) else L for L in (gate, up, down)]
+    for t, n in ((Wg, "W_gate"), (Wu, "W_up"), (Wd, "W_down")):
+        _need(t, torch.int32, 2, n)
+    for t, n in ((bg, "beta_gate"), (bu, "beta_up"), (bd, "beta_down")):
+        _need(t, torch.float32, 1, n)
+    M, D = x.shape
+    F = Wg.shape[0]
+    if Wg.shape[1] * 16 != D or Wu.shape != Wg.shape or Wd.shape[0] != D or Wd.shape[1] * 16 != F:
+        raise ValueError("W_gate and W_up must be [F, D/16], W_down [D, F/16]")
+    y = torch.empty((M, D), dtype=torch.float32, device=x.device) if out is None else out
+    u = torch.empty((M, F), dtype=torch.float32, device=x.device) if want_u else None
+    nws = int(lib().bitlinear_glu_workspace(M, D, F))
+    if ws is None:
+        ws = torch.empty(nws, dtype=torch.uint8, device=x.device)
+    _check("bitlinear_glu_forward",
+           lib().bitlinear_glu_forward(_ptr(x), M, D, F, _ptr(Wg), _ptr(bg), _ptr(Wu), _ptr(bu), _ptr(Wd), _ptr(bd),
+                                       _ptr(y), _ptr(u), _ptr(ws), ws.numel(), _stream(stream)))
+    return (y, u) if want_u else y
 
 
 class DecoderBlock:

@@ -501,6 +501,78 @@ bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, i
                                           as_stream(stream)));
 }
 
+size_t bitlinear_glu_workspace(int64_t M, int64_t D, int64_t F) {
+    if (M < 1 || D < 1 || F < 1) return 0;
+    const size_t fw = std::max(bitlinear_forward_workspace(M, F, D), bitlinear_forward_workspace(M, D, F));
+    return round256((size_t)M * D) + round256((size_t)M * 4) + 2 * round256((size_t)M * F * 4) +
+           round256((size_t)M * F) + round256((size_t)M * 4) + round256(fw);
+}
+
+bl_status bitlinear_glu_forward(const float* x, int64_t M, int64_t D, int64_t F, const uint32_t* W_gate,
+                                const float* beta_gate, const uint32_t* W_up, const float* beta_up,
+                                const uint32_t* W_down, const float* beta_down, float* y, float* u, void* ws,
+                                size_t ws_bytes, void* stream) {
+    if (!x || !W_gate || !beta_gate || !W_up || !beta_up || !W_down || !beta_down || !y) return BL_ERR_NULL;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(F, D, 64);
+    if (s) return s;
+    s = check_nk(D, F, 64);
+    if (s) return s;
+    const size_t need = bitlinear_glu_workspace(M, D, F);
+    if (!ws || ws_bytes < need) return BL_ERR_WORKSPACE;
+    const void* ptrs[10] = {x, W_gate, beta_gate, W_up, beta_up, W_down, beta_down, y, u, ws};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return BL_ERR_ALIGN;
+    const size_t wgu = (size_t)F * (D / 16) * 4, wd = (size_t)D * (F / 16) * 4;
+    const void* ins[7] = {x, W_gate, beta_gate, W_up, beta_up, W_down, beta_down};
+    const size_t in_bytes[7] = {(size_t)M * D * 4, wgu, 4, wgu, 4, wd, 4};
+    const void* outs[3] = {y, u, ws};
+    const size_t out_bytes[3] = {(size_t)M * D * 4, u ? (size_t)M * F * 4 : 0, ws_bytes};
+    for (int i = 0; i < 3; ++i) {
+        for (int j = 0; j < 7; ++j)
+            if (overlap(outs[i], out_bytes[i], ins[j], in_bytes[j])) return BL_ERR_ALIAS;
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(outs[i], out_bytes[i], outs[j], out_bytes[j])) return BL_ERR_ALIAS;
+    }
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    cudaStream_t st = as_stream(stream);
+    char* p = reinterpret_cast<char*>(ws);
+    int8_t* xq = reinterpret_cast<int8_t*>(p);
+    p += round256((size_t)M * D);
+    float* gx = reinterpret_cast<float*>(p);
+    p += round256((size_t)M * 4);
+    float* gate = reinterpret_cast<float*>(p);
+    p += round256((size_t)M * F * 4);
+    float* up = reinterpret_cast<float*>(p);
+    p += round256((size_t)M * F * 4);
+    int8_t* uq = reinterpret_cast<int8_t*>(p);
+    p += round256((size_t)M * F);
+    float* gu = reinterpret_cast<float*>(p);
+    p += round256((size_t)M * 4);
+    const size_t fws_bytes = ws_bytes - (size_t)(p - reinterpret_cast<char*>(ws));
+    // x -> RMS-normalised codes shared by gate and up
+    if (launch_quant_act_rms(x, nullptr, C_NONE, M, D, nullptr, xq, gx, st) != cudaSuccess) return BL_ERR_CUDA;
+    // gate and up: one launch over both for a few tokens, else one forward each
+    const GemvProblem probs[2] = {{xq, gx, W_gate, beta_gate, gate, (int)D, (int)F},
+                                  {xq, gx, W_up, beta_up, up, (int)D, (int)F}};
+    if (M <= AUTO_CUDA_MAX_M && gemv_fused_quant_ok(M, D)) {
+        cudaError_t e = pick_path((int)M, probs, 2, dev) == PATH_TC
+                            ? launch_decode_tc(probs, 2, (int)M, BL_I8, Y_F32, dev, st)
+                            : launch_gemv_fused_group(probs, 2, (int)M, BL_I8, Y_F32, dev, st);
+        if (e != cudaSuccess) return BL_ERR_CUDA;
+    } else {
+        s = run_forward(xq, gx, M, D, W_gate, beta_gate, F, gate, Y_F32, p, fws_bytes, stream);
+        if (s) return s;
+        s = run_forward(xq, gx, M, D, W_up, beta_up, F, up, Y_F32, p, fws_bytes, stream);
+        if (s) return s;
+    }
+    // u = SiLU(gate) * up, RMS-normalised codes of u
+    if (launch_quant_act_rms(gate, up, C_SILU_MUL, M, F, u, uq, gu, st) != cudaSuccess) return BL_ERR_CUDA;
+    return run_forward(uq, gu, M, F, W_down, beta_down, D, y, Y_F32, p, fws_bytes, stream);
+}
+
 bl_status bitlinear_device_status(void* stream) {
     DevInfo dev;
     bl_status s = current_device(dev);

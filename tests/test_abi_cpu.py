@@ -226,3 +226,29 @@ def test_binary_forward_validation():
     assert need >= 64 * 4096 + 64 * 4
     assert h(P(A1), 0, 64, 4096, P(A3), P(A4), 64, P(A5), 0, P(A6), need - 1, None) == WS
     assert h(P(A1), 0, 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DEVICE
+
+
+def test_glu_validation():
+    f = _L().bitlinear_glu_forward
+    ws = _L().bitlinear_glu_workspace(2, 256, 512)
+    assert ws >= 2 * 256 + 2 * 2 * 512 * 4 + 2 * 512
+    base = [P(A1), 2, 256, 512, P(A2), P(A3), P(A2 + 0x1000000), P(A3 + 16), P(A4), P(A3 + 32), P(A5), None,
+            P(A6), ws, None]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a0=None) == NULL
+    assert call(a10=None) == NULL
+    assert call(a2=200) == SHAPE            # D % 64
+    assert call(a3=520) == SHAPE            # F % 64
+    assert call(a1=0) == SHAPE
+    assert call(a12=None) == WS
+    assert call(a13=ws - 1) == WS
+    assert call(a10=P(A5 + 4)) == ALIGN
+    assert call(a10=P(A1)) == ALIAS         # y on x
+    assert call(a11=P(A5)) == ALIAS         # u on y
+    assert call(a12=P(A4)) == ALIAS         # workspace on W_down
+    assert call() == DEVICE
