@@ -394,18 +394,61 @@ def main():
         for i in range(n_e2e):
             e2e_step(i)
 
-    # The same per-step sequence (H2D copy, library call, D2H copy) recorded in
-    # CUDA graphs of at most CHUNK steps and replayed: the copies still run
-    # every step, the host no longer issues them one by one.
-    def e2e_graphs(n):
+    # Pipelined steps: NB sets of device input / output buffers and pinned
+    # output buffers; step i copies its input on s_in, runs the call on the
+    # compute stream and copies its output back on s_out, so the copies of
+    # steps i +- 1 overlap the kernel of step i.  Buffer set i % NB is reused
+    # only after the kernel (input side) and the D2H copy (output side) of
+    # step i - NB are done.  Recorded in CUDA graphs of <= CHUNK steps; every
+    # graph forks and joins the copy streams, so chunks do not overlap.
+    NB = 3
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    px = [dev_xcat] + [torch.empty_like(dev_xcat) for _ in range(NB - 1)]
+    py = [ycat] + [torch.empty_like(ycat) for _ in range(NB - 1)]
+    phy = [host_y] + [torch.empty_like(host_y).pin_memory() for _ in range(NB - 1)]
+    pplans = []
+    for bi in range(NB):
+        dx, dy, ox, oy = [], [], 0, 0
+        for L, x, y in zip(layers, xs, ys):
+            dx.append(px[bi][ox:ox + x.numel()].view(L["x"].shape))
+            dy.append(py[bi][oy:oy + y.numel()].view(L["y"].shape))
+            ox += x.numel()
+            oy += y.numel()
+        pplans.append([bl.BatchPlan([{"x": dx[j], "W_p": L["W_p"][c], "beta": L["beta"], "out": dy[j]}
+                                     for j, L in enumerate(layers)]) for c in range(copies)])
+
+    def pipe_graphs(n):
         gs, done = [], 0
         while done < n:
             k = min(CHUNK, n - done)
             g = torch.cuda.CUDAGraph()
+            ev_in = [torch.cuda.Event() for _ in range(NB)]
+            ev_comp = [torch.cuda.Event() for _ in range(NB)]
+            ev_out = [torch.cuda.Event() for _ in range(NB)]
+            used = set()
             with torch.cuda.stream(stream):
                 with torch.cuda.graph(g, stream=stream):
-                    for i in range(k):
-                        e2e_step(done + i)
+                    s_in.wait_stream(stream)
+                    s_out.wait_stream(stream)
+                    for j in range(k):
+                        i, bi = done + j, j % NB
+                        if bi in used:
+                            s_in.wait_event(ev_comp[bi])     # kernel of step i - NB has read px[bi]
+                        with torch.cuda.stream(s_in):
+                            px[bi].copy_(host_x, non_blocking=True)
+                            ev_in[bi].record(s_in)
+                        stream.wait_event(ev_in[bi])
+                        if bi in used:
+                            stream.wait_event(ev_out[bi])    # D2H of step i - NB has read py[bi]
+                        pplans[bi][i % copies].run(stream=stream)
+                        ev_comp[bi].record(stream)
+                        s_out.wait_event(ev_comp[bi])
+                        with torch.cuda.stream(s_out):
+                            phy[bi].copy_(py[bi], non_blocking=True)
+                            ev_out[bi].record(s_out)
+                        used.add(bi)
+                    stream.wait_stream(s_in)
+                    stream.wait_stream(s_out)
             gs.append(g)
             done += k
         return gs
@@ -414,9 +457,11 @@ def main():
         e2e_step(i)
     torch.cuda.synchronize()
     t_eager = e2e_timed(e2e_eager)
-    eg = e2e_graphs(n_e2e)
+    eg = pipe_graphs(n_e2e)
     with torch.cuda.stream(stream):
-        run(e2e_graphs(8))
+        run(pipe_graphs(8))
+    torch.cuda.synchronize()
+
     def e2e_replay():
         with torch.cuda.stream(stream):
             run(eg)
@@ -424,11 +469,14 @@ def main():
     del eg
     e2e = {"value": world * step_bytes() * n_e2e / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": n_e2e, "us_per_step": t_e2e / n_e2e * 1e6,
-           "path": "per step: one pinned H2D copy of both inputs + bitlinear_forward_fp_batch (both projections, "
-                   "descriptors marshalled once per weight copy) + one D2H copy of both outputs into pinned memory, "
-                   f"recorded in CUDA graphs of <= {CHUNK} steps and replayed; weights rotate over {copies} copies",
+           "path": "per step: one pinned H2D copy of both inputs (copy stream) + bitlinear_forward_fp_batch "
+                   "(both projections, descriptors marshalled once per buffer set and weight copy) + one D2H copy "
+                   f"of both outputs into pinned memory (second copy stream); {NB} buffer sets, so copies of "
+                   f"neighbouring steps overlap the kernel; recorded in CUDA graphs of <= {CHUNK} steps and "
+                   f"replayed; weights rotate over {copies} copies",
            "eager": {"value": world * step_bytes() * n_e2e / t_eager / 1e9, "us_per_step": t_eager / n_e2e * 1e6,
-                     "path": "the same three operations issued from the host every step, no graph"}}
+                     "path": "the same three operations issued from the host every step on one stream, "
+                             "no graph, no overlap"}}
 
     # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
     prefill = None
