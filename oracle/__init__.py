@@ -334,3 +334,63 @@ def glu(x: np.ndarray, tern: dict) -> dict:
                      ("acc_down", down["acc"][0]), ("y", down["y"][0])):
             out[k].append(v)
     return {k: np.stack(v) for k, v in out.items()}
+
+
+# ---------------------------------------------------------------------------
+# Group quantisation: unite.ai page, section "Gruppenquantisierung und
+# -normalisierung" -- weights and activations are divided into G groups and
+# each group gets its own parameters.  Groups are G contiguous, equal blocks
+# of the contraction dimension K (the split that divides both W and x).
+# ---------------------------------------------------------------------------
+
+def _groups(K: int, G: int):
+    assert G >= 1 and K % G == 0
+    Kg = K // G
+    return [slice(g * Kg, (g + 1) * Kg) for g in range(G)]
+
+
+def quantize_weights_grouped(W: np.ndarray, G: int, eps=EPS_W):
+    """absmean ternarisation per column group: beta_g = mean |W[:, K_g]| and
+    W_t[:, K_g] = clip(round(W[:, K_g] / (beta_g + eps)), -1, 1).
+    Returns (W_t [N, K], beta [G])."""
+    W = _c(W, np.float32)
+    W_t = np.empty(W.shape, np.int8)
+    beta = np.empty(G, np.float32)
+    for g, sl in enumerate(_groups(W.shape[1], G)):
+        W_t[:, sl], beta[g] = quantize_weights(W[:, sl], eps)
+    return W_t, beta
+
+
+def quant_act_grouped(x: np.ndarray, G: int):
+    """Per-token absmax quantiser per channel group: gamma[m, g] =
+    max(||x[m, K_g]||_inf, 1e-5), codes as eq. 2 with that gamma.
+    Returns (x_q [M, K], gamma [M, G])."""
+    x = _c(x, np.float32)
+    x_q = np.empty(x.shape, np.int8)
+    gamma = np.empty((x.shape[0], G), np.float32)
+    for g, sl in enumerate(_groups(x.shape[1], G)):
+        x_q[:, sl], gamma[:, g] = quant_act(x[:, sl])
+    return x_q, gamma
+
+
+def forward_grouped(x: np.ndarray, W_t: np.ndarray, beta, G: int):
+    """Group-quantised forward: acc_g = sum_{k in K_g} W_t x_hat (int32) and
+    y = sum over g = 0, 1, ... of (float)acc_g * ((beta_g * gamma_{m,g}) / 127),
+    each term binary32 as eq. 3, added in binary32 in increasing g.
+    Returns x_q, gamma, acc [G, M, N], y and the binary64 y64."""
+    x_q, gamma = quant_act_grouped(x, G)
+    M, N = x.shape[0], W_t.shape[0]
+    acc = np.empty((G, M, N), np.int32)
+    y = np.zeros((M, N), np.float32)
+    y64 = np.zeros((M, N), np.float64)
+    for g, sl in enumerate(_groups(x.shape[1], G)):
+        acc[g] = ternary_acc(x_q[:, sl], W_t[:, sl])
+        t = rescale_f32(acc[g], beta[g], gamma[:, g])
+        y = t if g == 0 else (y + t).astype(np.float32)
+        y64 += rescale_f64(acc[g], beta[g], gamma[:, g])
+    return {"x_q": x_q, "gamma": gamma, "acc": acc, "y": y, "y64": y64}
+
+
+def group_major(a: np.ndarray, G: int) -> np.ndarray:
+    """[R, K] -> [G, R, K/G]: column group g of every row, groups one after another."""
+    return np.stack([a[:, sl] for sl in _groups(a.shape[1], G)])

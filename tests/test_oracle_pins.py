@@ -402,3 +402,57 @@ def test_glu_tokens_are_independent_and_match_the_block():
     g = oracle.glu(ref["h1"], tern)
     for k, kb in (("gate", "gate"), ("up", "up"), ("u", "u"), ("y", "down")):
         np.testing.assert_array_equal(g[k].ravel(), np.asarray(ref[kb]).ravel())
+
+
+# --------------------------------------------------------------------------
+# Group quantisation: reductions to the ungrouped, pinned path
+# --------------------------------------------------------------------------
+
+def test_grouped_g1_is_the_ungrouped_path():
+    W = workloads.latent_weights(120, 77, 256)
+    x = workloads.activations(121, 3, 256, outliers=True)
+    W_t, beta = oracle.quantize_weights_grouped(W, 1)
+    W_t1, beta1 = oracle.quantize_weights(W)
+    np.testing.assert_array_equal(W_t, W_t1)
+    assert beta[0] == beta1
+    r, r1 = oracle.forward_grouped(x, W_t, beta, 1), oracle.forward(x, W_t1, beta1)
+    np.testing.assert_array_equal(r["acc"][0], r1["acc"])
+    np.testing.assert_array_equal(r["y"], r1["y"])
+    np.testing.assert_array_equal(r["gamma"][:, 0], r1["gamma"])
+
+
+def test_grouped_duplicate_halves_double_exactly():
+    # W = [A | A], x = [a | a], G = 2: equal parameters and accumulators in both
+    # groups, so y = fl(t + t) = 2 t exactly
+    A = workloads.latent_weights(130, 50, 128)
+    a = workloads.activations(131, 2, 128, outliers=True)
+    W_t, beta = oracle.quantize_weights_grouped(np.hstack([A, A]), 2)
+    assert beta[0] == beta[1] == oracle.absmean_beta(A)
+    r = oracle.forward_grouped(np.hstack([a, a]), W_t, beta, 2)
+    At, bA = oracle.quantize_weights(A)
+    np.testing.assert_array_equal(r["y"], 2 * oracle.forward(a, At, bA)["y"])
+
+
+def test_grouped_zero_group_and_group_scales():
+    # a zero column group contributes exactly 0; scaling one group by 2^3
+    # scales only its beta and leaves every code unchanged
+    W = workloads.latent_weights(140, 40, 256)
+    x = workloads.activations(141, 2, 256)
+    W0 = W.copy()
+    W0[:, 128:] = 0
+    W_t, beta = oracle.quantize_weights_grouped(W0, 2)
+    assert beta[1] == 0 and not W_t[:, 128:].any()
+    r = oracle.forward_grouped(x, W_t, beta, 2)
+    Wt_a, b_a = oracle.quantize_weights(W[:, :128])
+    np.testing.assert_array_equal(r["y"], oracle.forward(x[:, :128], Wt_a, b_a)["y"])
+    W8 = W.copy()
+    W8[:, 64:128] *= np.float32(8)
+    # (eps = 0: the divisor guard would break the exact power-of-two scaling)
+    W_t4, beta4 = oracle.quantize_weights_grouped(W, 4, eps=0.0)
+    W_t8, beta8 = oracle.quantize_weights_grouped(W8, 4, eps=0.0)
+    np.testing.assert_array_equal(W_t8, W_t4)
+    assert beta8[1] == 8 * beta4[1] and all(beta8[g] == beta4[g] for g in (0, 2, 3))
+    # activation groups: gamma per group is that group's absmax
+    _, gam = oracle.quant_act_grouped(x, 4)
+    for g in range(4):
+        np.testing.assert_array_equal(gam[:, g], np.maximum(np.abs(x[:, 64 * g:64 * (g + 1)]).max(1), 1e-5))
