@@ -377,18 +377,23 @@ def forward_grouped(x: np.ndarray, W_t: np.ndarray, beta, G: int):
     """Group-quantised forward: acc_g = sum_{k in K_g} W_t x_hat (int32) and
     y = sum over g = 0, 1, ... of (float)acc_g * ((beta_g * gamma_{m,g}) / 127),
     each term binary32 as eq. 3, added in binary32 in increasing g.
-    Returns x_q, gamma, acc [G, M, N], y and the binary64 y64."""
+    Returns x_q, gamma, acc [G, M, N], y, the binary64 y64 and yabs64, the
+    binary64 sum of the terms' magnitudes (terms of different groups can
+    cancel, so binary32 evaluation is bounded relative to yabs64, not y)."""
     x_q, gamma = quant_act_grouped(x, G)
     M, N = x.shape[0], W_t.shape[0]
     acc = np.empty((G, M, N), np.int32)
     y = np.zeros((M, N), np.float32)
     y64 = np.zeros((M, N), np.float64)
+    yabs64 = np.zeros((M, N), np.float64)
     for g, sl in enumerate(_groups(x.shape[1], G)):
         acc[g] = ternary_acc(x_q[:, sl], W_t[:, sl])
         t = rescale_f32(acc[g], beta[g], gamma[:, g])
         y = t if g == 0 else (y + t).astype(np.float32)
-        y64 += rescale_f64(acc[g], beta[g], gamma[:, g])
-    return {"x_q": x_q, "gamma": gamma, "acc": acc, "y": y, "y64": y64}
+        t64 = rescale_f64(acc[g], beta[g], gamma[:, g])
+        y64 += t64
+        yabs64 += np.abs(t64)
+    return {"x_q": x_q, "gamma": gamma, "acc": acc, "y": y, "y64": y64, "yabs64": yabs64}
 
 
 def group_major(a: np.ndarray, G: int) -> np.ndarray:

@@ -421,6 +421,18 @@ def test_grouped_g1_is_the_ungrouped_path():
     np.testing.assert_array_equal(r["gamma"][:, 0], r1["gamma"])
 
 
+def test_grouped_error_bound_from_the_arithmetic():
+    # binary32 evaluation against binary64: within (G + 2) 2^-24 of the sum of
+    # the terms' magnitudes, even where the terms of different groups cancel
+    W = workloads.latent_weights(150, 300, 2048)
+    x = workloads.activations(151, 4, 2048, outliers=True)
+    for G in (2, 4, 8):
+        W_t, beta = oracle.quantize_weights_grouped(W, G)
+        r = oracle.forward_grouped(x, W_t, beta, G)
+        assert (np.abs(r["y"] - r["y64"]) <= (G + 2) * 2.0 ** -24 * r["yabs64"]).all()
+        assert (r["yabs64"] >= np.abs(r["y64"])).all()
+
+
 def test_grouped_duplicate_halves_double_exactly():
     # W = [A | A], x = [a | a], G = 2: equal parameters and accumulators in both
     # groups, so y = fl(t + t) = 2 t exactly
