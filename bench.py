@@ -18,7 +18,8 @@ H2D copy, one call, one D2H copy, recorded in CUDA graphs; the same sequence
 issued eagerly is reported beside it), and SM clocks.  Extra sections
 (--sections): the prefill GEMM (M = 2048) in int8 TOPS against the int8
 tensor peak, small-batch decode, a decoder block, the 1-bit weight variant
-(decode GEMV and prefill GEMM) and the MatMul-free GLU channel mixer.
+(decode GEMV and prefill GEMM), the MatMul-free GLU channel mixer and group
+quantisation (G = 4) at decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -213,7 +214,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="run the decode step only (no extra sections)")
-    ap.add_argument("--sections", default="prefill,small,block,binary,glu",
+    ap.add_argument("--sections", default="prefill,small,block,binary,glu,grouped",
                     help="extra measured sections after the decode step, comma separated")
     args = ap.parse_args()
     sections = set() if args.no_prefill else {x for x in args.sections.split(",") if x}
@@ -625,6 +626,39 @@ def main():
                                            "path": "tcgen05 GEMM, 1-bit unpack"}
             del g, W_p, x_q, y, ws
 
+    # ---- group quantisation along K (G = 4): decode M = 1 on the FFN shapes ----
+    grouped = None
+    if "grouped" in sections:
+        grouped = {}
+        G = 4
+        for s in workloads.W2.shapes:
+            W_t, beta = bl.quantize_weights_grouped(torch.from_numpy(s.weights()).to(dev), G)
+            W_p0 = bl.pack_grouped(W_t)
+            del W_t
+            nc = max(2, int(4 * L2 // (W_p0.numel() * 4)) + 1)
+            W_ps = [W_p0] + [W_p0.clone() for _ in range(nc - 1)]
+            xb = torch.from_numpy(s.inputs_bf16_bits().view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((s.M, s.N), dtype=torch.float32, device=dev)
+            ws = torch.empty(bl.lib().bitlinear_forward_grouped_fp_workspace(s.M, s.N, s.K, G), dtype=torch.uint8,
+                             device=dev)
+            reps = 8 * nc
+            with torch.cuda.stream(stream):
+                for i in range(4):
+                    bl.forward_grouped_fp(xb, W_ps[i % nc], beta, out=y, ws=ws, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(reps):
+                        bl.forward_grouped_fp(xb, W_ps[i % nc], beta, out=y, ws=ws, stream=stream)
+            g.replay()
+            t = timed_run([g])
+            gbs = s.algorithmic_bytes * reps / t / 1e9
+            grouped["decode_g4_" + s.name] = {"us_per_call": t / reps * 1e6, "GB/s": gbs,
+                                              "frac_of_hbm": gbs / peaks["hbm_gbs"], "launches": 3,
+                                              "path": "grouped quantiser + one GEMV launch over the 4 groups "
+                                                      "(int32 per group) + ordered per-group rescale"}
+            del g, W_ps, W_p0, xb, y, ws
+
     # ---- MatMul-free GLU channel mixer (hidden 2560, intermediate 6912) ----
     glu = None
     if "glu" in sections:
@@ -688,7 +722,7 @@ def main():
                        "parallelism": f"replicas x{world}", "graph_chunk_steps": CHUNK},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks, "prefill": prefill, "small_batch": small, "block": block,
-            "binary": binary, "glu": glu,
+            "binary": binary, "glu": glu, "grouped": grouped,
             "device": props.name,
         }
         print(json.dumps(line), flush=True)

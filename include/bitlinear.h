@@ -16,7 +16,8 @@
  *         Grundlagen" eq. 2 "Aktivierungsquantisierung" and eq. 3
  *         "BitLinear-Betrieb", section "Implementierungshinweise" (the
  *         quantise -> ternary matmul -> scale shape of a forward call); the
- *         1-bit weights of the same section, item 1 "Gewichtsbinarisierung".
+ *         1-bit weights of the same section, item 1 "Gewichtsbinarisierung";
+ *         section "Gruppenquantisierung und -normalisierung" (group quantisation).
  *
  * Conventions for every call:
  *   - Every pointer argument is a DEVICE pointer owned by the caller (the
@@ -353,6 +354,81 @@ enum { BL_COMBINE_NONE = 0, BL_COMBINE_ADD = 1, BL_COMBINE_SILU_MUL = 2 };
  */
 bl_status bitlinear_quant_act_rms(const float* a, const float* b, int combine, int64_t M, int64_t K,
                                   float* h, int8_t* x_q, float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Group quantisation                                                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [BNC] section "Gruppenquantisierung und -normalisierung": weights and
+ * activations are divided into G groups, each with its own parameters, so
+ * that the groups can be processed in parallel without exchanging them.
+ * Here the groups are G contiguous, equal blocks of the contraction
+ * dimension: K_g = [g*K/G, (g+1)*K/G).  Group g of W (all rows, columns K_g)
+ * has its absmean beta_g; group g of a token x_m has its absmax gamma_{m,g}.
+ *   acc_g[m, n] = sum_{k in K_g} W_t[n, k] * x_q[m, k]                   (int32)
+ *   y[m, n]     = sum over g = 0, 1, ... of (float)acc_g[m, n] * ((beta_g * gamma_{m,g}) / 127)
+ * with every product, quotient and add one binary32 operation, the adds in
+ * increasing g.  G = 1 is exactly the ungrouped path.
+ *
+ * Layouts are group-major, so every group is an ordinary matrix:
+ *   W_t [G][N][K/G] int8; W_p [G][N][K/(16G)] uint32 = bitlinear_pack of W_t
+ *       viewed as G*N rows of K/G trits; beta [G] float32;
+ *   x_q [G][M][K/G] int8; gamma [M][G] float32.
+ * 1 <= G <= BL_MAX_GROUPS, K % (64 G) == 0 for every call below.
+ */
+#define BL_MAX_GROUPS 8
+
+/* Bytes of device workspace bitlinear_quantize_weights_grouped needs (4*N*K + a few KiB). */
+size_t bitlinear_quantize_weights_grouped_workspace(int64_t N, int64_t K, int64_t G);
+
+/*
+ * Per-group absmean ternarisation: beta_g and W_t[:, K_g] exactly as
+ * bitlinear_quantize_weights computes them for the matrix W[:, K_g] alone.
+ *   W [N, K] float32 in; W_t [G][N][K/G] int8 out; beta [G] float32 out.
+ * The workspace holds W regrouped to [G][N][K/G] (4*N*K bytes) and the sums.
+ */
+bl_status bitlinear_quantize_weights_grouped(const float* W, int64_t N, int64_t K, int64_t G, float eps,
+                                             int8_t* W_t, float* beta, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Per-token, per-group absmax quantiser: gamma[m][g] and the codes of
+ * x[m, K_g] exactly as bitlinear_quant_act computes them for that block alone.
+ *   x [M, K] float32 (BL_F32) or bfloat16 (BL_BF16) in;
+ *   x_q [G][M][K/G] int8 out; gamma [M][G] float32 out.
+ */
+bl_status bitlinear_quant_act_grouped(const void* x, int x_dtype, int64_t M, int64_t K, int64_t G,
+                                      int8_t* x_q, float* gamma, void* stream);
+
+/* Bytes of device workspace bitlinear_forward_grouped and _grouped_acc need (> 0). */
+size_t bitlinear_forward_grouped_workspace(int64_t M, int64_t N, int64_t K, int64_t G);
+
+/*
+ * Group-quantised forward (formula above).  The G contractions run as the
+ * ungrouped ones would on each group (for M <= 4 tokens, with M rounded up to
+ * 1, 2 or 4 times K/G <= 65536, all groups in one launch), writing int32
+ * accumulators to the workspace; one more kernel applies the per-group scales
+ * in order.  Arguments as for bitlinear_forward with the grouped layouts.
+ */
+bl_status bitlinear_forward_grouped(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, int64_t G,
+                                    const uint32_t* W_p, const float* beta, int64_t N, void* y, int y_dtype,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The per-group accumulators of bitlinear_forward_grouped: acc_g[m, n] at
+ * acc[g * S + m * N + n], S = M*N rounded up to a multiple of 4 (so acc holds
+ * G*S int32).  For exact comparisons in tests.
+ */
+bl_status bitlinear_forward_grouped_acc(const int8_t* x_q, int64_t M, int64_t K, int64_t G, const uint32_t* W_p,
+                                        int64_t N, int32_t* acc, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace bitlinear_forward_grouped_fp needs. */
+size_t bitlinear_forward_grouped_fp_workspace(int64_t M, int64_t N, int64_t K, int64_t G);
+
+/* bitlinear_quant_act_grouped(x) then bitlinear_forward_grouped, bit-identical to the two calls. */
+bl_status bitlinear_forward_grouped_fp(const void* x, int x_dtype, int64_t M, int64_t K, int64_t G,
+                                       const uint32_t* W_p, const float* beta, int64_t N, void* y, int y_dtype,
+                                       void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace bitlinear_glu_forward needs for this shape. */
 size_t bitlinear_glu_workspace(int64_t M, int64_t D, int64_t F);

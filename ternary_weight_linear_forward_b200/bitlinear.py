@@ -41,6 +41,14 @@ SIGNATURES = {
     "bitlinear_forward_acc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "bitlinear_forward_noalloc": (_I, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _I, _P]),
     "bitlinear_quant_act_rms": (_I, [_P, _P, _I, _I64, _I64, _P, _P, _P, _P]),
+    "bitlinear_quantize_weights_grouped_workspace": (_SZ, [_I64, _I64, _I64]),
+    "bitlinear_quantize_weights_grouped": (_I, [_P, _I64, _I64, _I64, _F, _P, _P, _P, _SZ, _P]),
+    "bitlinear_quant_act_grouped": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P]),
+    "bitlinear_forward_grouped_workspace": (_SZ, [_I64, _I64, _I64, _I64]),
+    "bitlinear_forward_grouped": (_I, [_P, _P, _I64, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_grouped_acc": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_forward_grouped_fp_workspace": (_SZ, [_I64, _I64, _I64, _I64]),
+    "bitlinear_forward_grouped_fp": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_glu_workspace": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_glu_forward": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_binarize_weights_workspace": (_SZ, [_I64, _I64]),
@@ -500,6 +508,113 @@ class BitLinear:
 
     def __call__(self, x: torch.Tensor, out_dtype=torch.float32, out=None) -> torch.Tensor:
         return forward_fp(x, self.W_p, self.beta, out_dtype=out_dtype, out=out)
+
+
+# --------------------------------------------------------------------------
+# Group quantisation along K (unite.ai page, "Gruppenquantisierung und
+# -normalisierung"); group-major layouts, see include/bitlinear.h
+# --------------------------------------------------------------------------
+
+def quantize_weights_grouped(W: torch.Tensor, G: int, eps: float = EPS_W, stream=None):
+    """Per-group absmean ternarisation -> (W_t int8 [G, N, K/G], beta float32 [G])."""
+    _need(W, torch.float32, 2, "W")
+    N, K = W.shape
+    W_t = torch.empty((G, N, K // G), dtype=torch.int8, device=W.device)
+    beta = torch.empty(max(G, 4), dtype=torch.float32, device=W.device)[:G]
+    nws = int(lib().bitlinear_quantize_weights_grouped_workspace(N, K, G))
+    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=W.device)
+    _check("bitlinear_quantize_weights_grouped",
+           lib().bitlinear_quantize_weights_grouped(_ptr(W), N, K, G, float(eps), _ptr(W_t), _ptr(beta), _ptr(ws),
+                                                    nws, _stream(stream)))
+    return W_t, beta
+
+
+def pack_grouped(W_t: torch.Tensor, stream=None) -> torch.Tensor:
+    """2-bit packing of group-major trits [G, N, K/G] -> W_p int32 [G, N, K/(16G)]."""
+    _need(W_t, torch.int8, 3, "W_t")
+    G, N, Kg = W_t.shape
+    return pack(W_t.view(G * N, Kg), stream=stream).view(G, N, -1)
+
+
+def quant_act_grouped(x: torch.Tensor, G: int, stream=None):
+    """Per-token, per-group absmax quantiser -> (x_q int8 [G, M, K/G], gamma float32 [M, G])."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, 2, "x")
+    M, K = x.shape
+    x_q = torch.empty((G, M, K // G), dtype=torch.int8, device=x.device)
+    gamma = torch.empty(max(M * G, 4), dtype=torch.float32, device=x.device)[:M * G].view(M, G)
+    dt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_quant_act_grouped",
+           lib().bitlinear_quant_act_grouped(_ptr(x), dt, M, K, G, _ptr(x_q), _ptr(gamma), _stream(stream)))
+    return x_q, gamma
+
+
+def _grouped_shapes(W_p, G, K):
+    _need(W_p, torch.int32, 3, "W_p")
+    if W_p.shape[0] != G or W_p.shape[2] * 16 * G != K:
+        raise ValueError("W_p must be [G, N, K/(16G)]")
+    return W_p.shape[1]
+
+
+def forward_grouped(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor,
+                    out_dtype=torch.float32, out=None, ws=None, stream=None) -> torch.Tensor:
+    """Group-quantised forward from group-major x_q [G, M, K/G] and gamma [M, G]."""
+    _need(x_q, torch.int8, 3, "x_q")
+    _need(gamma, torch.float32, 2, "gamma")
+    _need(beta, torch.float32, 1, "beta")
+    G, M, Kg = x_q.shape
+    K = G * Kg
+    N = _grouped_shapes(W_p, G, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = int(lib().bitlinear_forward_grouped_workspace(M, N, K, G))
+    if ws is None:
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward_grouped",
+           lib().bitlinear_forward_grouped(_ptr(x_q), _ptr(gamma), M, K, G, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                           _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def forward_grouped_acc(x_q: torch.Tensor, W_p: torch.Tensor, stream=None) -> torch.Tensor:
+    """Per-group int32 accumulators -> [G, M, N]."""
+    _need(x_q, torch.int8, 3, "x_q")
+    G, M, Kg = x_q.shape
+    K = G * Kg
+    N = _grouped_shapes(W_p, G, K)
+    S = (M * N + 3) // 4 * 4
+    acc = torch.empty(G * S, dtype=torch.int32, device=x_q.device)
+    nws = int(lib().bitlinear_forward_grouped_workspace(M, N, K, G))
+    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=x_q.device)
+    _check("bitlinear_forward_grouped_acc",
+           lib().bitlinear_forward_grouped_acc(_ptr(x_q), M, K, G, _ptr(W_p), N, _ptr(acc), _ptr(ws), nws,
+                                               _stream(stream)))
+    return acc.view(G, S)[:, :M * N].reshape(G, M, N)
+
+
+def forward_grouped_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype=torch.float32, out=None,
+                       ws=None, stream=None) -> torch.Tensor:
+    """quant_act_grouped + forward_grouped in one call."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, x.dtype, 2, "x")
+    _need(beta, torch.float32, 1, "beta")
+    M, K = x.shape
+    G = beta.shape[0]
+    N = _grouped_shapes(W_p, G, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
+    nws = int(lib().bitlinear_forward_grouped_fp_workspace(M, N, K, G))
+    if ws is None:
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=x.device)
+    xdt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
+    _check("bitlinear_forward_grouped_fp",
+           lib().bitlinear_forward_grouped_fp(_ptr(x), xdt, M, K, G, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
+                                              _ptr(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 def glu_forward(x: torch.Tensor, gate, up, down, want_u: bool = False, out=None, ws=None, stream=None):

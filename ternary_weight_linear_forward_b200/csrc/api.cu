@@ -154,6 +154,43 @@ bl_status run_forward_bits(const int8_t* x_q, const float* gamma, int64_t M, int
     return from_cuda(e);
 }
 
+// ---- group quantisation along K (G contiguous groups of K / G channels) ----
+
+bool groups_ok(int64_t K, int64_t G) { return G >= 1 && G <= BL_MAX_GROUPS && K % (64 * G) == 0; }
+
+// int32 elements between the starts of two groups' [M, N] accumulator blocks
+// (rounded up so that every block starts 16-byte aligned)
+long long group_acc_stride(int64_t M, int64_t N) { return (M * N + 3) / 4 * 4; }
+
+size_t round256z(size_t n) { return (n + 255) / 256 * 256; }
+
+// acc[g] (at acc + g * stride) = sum over group g of W_t x_q, for every group
+bl_status run_grouped_acc(const int8_t* x_q, int64_t M, int64_t K, int64_t G, const uint32_t* W_p, int64_t N,
+                          int* acc, long long stride, void* fws, size_t fws_bytes, const DevInfo& dev, void* stream) {
+    const int64_t Kg = K / G;
+    if (M <= AUTO_CUDA_MAX_M && gemv_fused_quant_ok(M, Kg)) {
+        // every group is one problem of a single launch
+        GemvProblem probs[BL_MAX_GROUPS];
+        for (int64_t g = 0; g < G; ++g)
+            probs[g] = {x_q + g * M * Kg, nullptr, W_p + g * N * (Kg / 16), nullptr, acc + g * stride, (int)Kg, (int)N};
+        const cudaError_t e = pick_path((int)M, probs, (int)G, dev) == PATH_TC
+                                  ? launch_decode_tc(probs, (int)G, (int)M, BL_I8, Y_ACC, dev, as_stream(stream))
+                                  : launch_gemv_fused_group(probs, (int)G, (int)M, BL_I8, Y_ACC, dev, as_stream(stream));
+        return from_cuda(e);
+    }
+    for (int64_t g = 0; g < G; ++g) {
+        bl_status s = run_forward(x_q + g * M * Kg, nullptr, M, Kg, W_p + g * N * (Kg / 16), nullptr, N,
+                                  acc + g * stride, Y_ACC, fws, fws_bytes, stream);
+        if (s) return s;
+    }
+    return BL_OK;
+}
+
+size_t grouped_ws(int64_t M, int64_t N, int64_t K, int64_t G) {
+    if (M < 1 || N < 1 || !groups_ok(K, G)) return 0;
+    return round256z((size_t)group_acc_stride(M, N) * G * 4) + round256z(bitlinear_forward_workspace(M, N, K / G));
+}
+
 }  // namespace
 
 DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
@@ -571,6 +608,151 @@ bl_status bitlinear_glu_forward(const float* x, int64_t M, int64_t D, int64_t F,
     // u = SiLU(gate) * up, RMS-normalised codes of u
     if (launch_quant_act_rms(gate, up, C_SILU_MUL, M, F, u, uq, gu, st) != cudaSuccess) return BL_ERR_CUDA;
     return run_forward(uq, gu, M, F, W_down, beta_down, D, y, Y_F32, p, fws_bytes, stream);
+}
+
+size_t bitlinear_quantize_weights_grouped_workspace(int64_t N, int64_t K, int64_t G) {
+    if (N < 1 || !groups_ok(K, G)) return 0;
+    return regroup_ws_bytes(N, K) + quantize_weights_ws_bytes();
+}
+
+bl_status bitlinear_quantize_weights_grouped(const float* W, int64_t N, int64_t K, int64_t G, float eps,
+                                             int8_t* W_t, float* beta, void* ws, size_t ws_bytes, void* stream) {
+    if (!W || !W_t || !beta) return BL_ERR_NULL;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    if (!groups_ok(K, G)) return BL_ERR_SHAPE;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return BL_ERR_SHAPE;
+    const size_t need = bitlinear_quantize_weights_grouped_workspace(N, K, G);
+    if (!ws || ws_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(W_t) || !aligned16(beta) || !aligned16(ws)) return BL_ERR_ALIGN;
+    const size_t n = (size_t)N * K;
+    if (overlap(W_t, n, W, n * 4) || overlap(beta, (size_t)G * 4, W, n * 4) || overlap(W_t, n, beta, (size_t)G * 4) ||
+        overlap(ws, ws_bytes, W, n * 4) || overlap(ws, ws_bytes, W_t, n) || overlap(ws, ws_bytes, beta, (size_t)G * 4))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    cudaStream_t st = as_stream(stream);
+    float* Wg = reinterpret_cast<float*>(ws);  // [G][N][K/G]
+    void* qws = reinterpret_cast<char*>(ws) + regroup_ws_bytes(N, K);
+    if (launch_regroup(W, N, K, (int)G, Wg, dev.num_sms, st) != cudaSuccess) return BL_ERR_CUDA;
+    const size_t ng = n / (size_t)G;
+    for (int64_t g = 0; g < G; ++g)
+        if (launch_quantize_weights(Wg + g * ng, (long long)ng, eps, W_t + g * ng, beta + g, qws, dev.num_sms, st) !=
+            cudaSuccess)
+            return BL_ERR_CUDA;
+    return BL_OK;
+}
+
+bl_status bitlinear_quant_act_grouped(const void* x, int x_dtype, int64_t M, int64_t K, int64_t G, int8_t* x_q,
+                                      float* gamma, void* stream) {
+    if (!x || !x_q || !gamma) return BL_ERR_NULL;
+    if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_DTYPE;
+    if (M < 1 || M > (int64_t)INT32_MAX / BL_MAX_GROUPS) return BL_ERR_SHAPE;
+    bl_status s = check_nk(1, K, 64);
+    if (s) return s;
+    if (!groups_ok(K, G)) return BL_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(x_q) || !aligned16(gamma)) return BL_ERR_ALIGN;
+    const size_t xb = (size_t)M * K * (x_dtype == BL_BF16 ? 2 : 4), gb = (size_t)M * G * 4;
+    if (overlap(x_q, (size_t)M * K, x, xb) || overlap(gamma, gb, x, xb) || overlap(gamma, gb, x_q, (size_t)M * K))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return from_cuda(launch_quant_act_grouped(x, x_dtype == BL_BF16, M, K, (int)G, x_q, gamma, as_stream(stream)));
+}
+
+size_t bitlinear_forward_grouped_workspace(int64_t M, int64_t N, int64_t K, int64_t G) {
+    return grouped_ws(M, N, K, G);
+}
+
+// shared checks of the grouped forward calls (x_q group-major, W_p group-major)
+static bl_status check_grouped(const int8_t* x_q, int64_t M, int64_t K, int64_t G, const uint32_t* W_p, int64_t N,
+                               const void* out, size_t out_bytes, void* ws, size_t ws_bytes) {
+    if (!x_q || !W_p || !out) return BL_ERR_NULL;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    if (!groups_ok(K, G)) return BL_ERR_SHAPE;
+    const size_t need = grouped_ws(M, N, K, G);
+    if (!ws || ws_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(x_q) || !aligned16(W_p) || !aligned16(out) || !aligned16(ws)) return BL_ERR_ALIGN;
+    if (overlap(out, out_bytes, x_q, (size_t)M * K) || overlap(out, out_bytes, W_p, (size_t)N * K / 4) ||
+        overlap(ws, ws_bytes, x_q, (size_t)M * K) || overlap(ws, ws_bytes, W_p, (size_t)N * K / 4) ||
+        overlap(ws, ws_bytes, out, out_bytes))
+        return BL_ERR_ALIAS;
+    return BL_OK;
+}
+
+bl_status bitlinear_forward_grouped(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, int64_t G,
+                                    const uint32_t* W_p, const float* beta, int64_t N, void* y, int y_dtype, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    if (!gamma || !beta) return BL_ERR_NULL;
+    if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_DTYPE;
+    const size_t yb = (size_t)M * N * (y_dtype == BL_F32 ? 4 : 2);
+    bl_status s = check_grouped(x_q, M, K, G, W_p, N, y, yb, ws, ws_bytes);
+    if (s) return s;
+    if (!aligned16(gamma) || !aligned16(beta)) return BL_ERR_ALIGN;
+    if (overlap(y, yb, gamma, (size_t)M * G * 4) || overlap(y, yb, beta, (size_t)G * 4) ||
+        overlap(ws, ws_bytes, gamma, (size_t)M * G * 4) || overlap(ws, ws_bytes, beta, (size_t)G * 4))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    const long long stride = group_acc_stride(M, N);
+    int* acc = reinterpret_cast<int*>(ws);
+    char* fws = reinterpret_cast<char*>(ws) + round256z((size_t)stride * G * 4);
+    s = run_grouped_acc(x_q, M, K, G, W_p, N, acc, stride, fws, ws_bytes - (size_t)(fws - reinterpret_cast<char*>(ws)),
+                        dev, stream);
+    if (s) return s;
+    return from_cuda(launch_grouped_rescale(acc, stride, gamma, beta, (int)M, (int)N, (int)G, y,
+                                            y_dtype == BL_F32 ? Y_F32 : Y_BF16, dev.num_sms, as_stream(stream)));
+}
+
+bl_status bitlinear_forward_grouped_acc(const int8_t* x_q, int64_t M, int64_t K, int64_t G, const uint32_t* W_p,
+                                        int64_t N, int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
+    if (M < 1 || N < 1 || !groups_ok(K, G)) return BL_ERR_SHAPE;
+    const long long stride = group_acc_stride(M, N);
+    bl_status s = check_grouped(x_q, M, K, G, W_p, N, acc, (size_t)stride * G * 4, ws, ws_bytes);
+    if (s) return s;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    return run_grouped_acc(x_q, M, K, G, W_p, N, acc, stride, ws, ws_bytes, dev, stream);
+}
+
+size_t bitlinear_forward_grouped_fp_workspace(int64_t M, int64_t N, int64_t K, int64_t G) {
+    const size_t f = grouped_ws(M, N, K, G);
+    if (!f) return 0;
+    return round256((size_t)M * K) + round256((size_t)M * G * 4) + f;
+}
+
+bl_status bitlinear_forward_grouped_fp(const void* x, int x_dtype, int64_t M, int64_t K, int64_t G,
+                                       const uint32_t* W_p, const float* beta, int64_t N, void* y, int y_dtype,
+                                       void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !W_p || !beta || !y) return BL_ERR_NULL;
+    if ((x_dtype != BL_F32 && x_dtype != BL_BF16) || (y_dtype != BL_F32 && y_dtype != BL_BF16)) return BL_ERR_DTYPE;
+    if (M < 1 || M > (int64_t)INT32_MAX / BL_MAX_GROUPS) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    if (!groups_ok(K, G)) return BL_ERR_SHAPE;
+    const size_t need = bitlinear_forward_grouped_fp_workspace(M, N, K, G);
+    if (!ws || ws_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(W_p) || !aligned16(beta) || !aligned16(y) || !aligned16(ws)) return BL_ERR_ALIGN;
+    const size_t xb = (size_t)M * K * (x_dtype == BL_BF16 ? 2 : 4), yb = (size_t)M * N * (y_dtype == BL_F32 ? 4 : 2);
+    if (overlap(y, yb, x, xb) || overlap(y, yb, W_p, (size_t)N * K / 4) || overlap(y, yb, beta, (size_t)G * 4) ||
+        overlap(ws, ws_bytes, x, xb) || overlap(ws, ws_bytes, y, yb))
+        return BL_ERR_ALIAS;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    int8_t* x_q = reinterpret_cast<int8_t*>(ws);
+    float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
+    char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * G * 4);
+    if (launch_quant_act_grouped(x, x_dtype == BL_BF16, M, K, (int)G, x_q, gamma, as_stream(stream)) != cudaSuccess)
+        return BL_ERR_CUDA;
+    return bitlinear_forward_grouped(x_q, gamma, M, K, G, W_p, beta, N, y, y_dtype, fws,
+                                     ws_bytes - (size_t)(fws - reinterpret_cast<char*>(ws)), stream);
 }
 
 bl_status bitlinear_device_status(void* stream) {

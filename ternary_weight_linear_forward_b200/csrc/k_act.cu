@@ -89,15 +89,11 @@ __device__ __forceinline__ double block_sum_f64(double v, double* sm) {
     return r;
 }
 
+// Quantise the n activations at xr (n % 16 == 0) with their own absmax:
+// codes to qr, the floored absmax to *gamma_out.  Called by whole CTAs.
 template <bool BF16>
-__global__ void __launch_bounds__(ACT_THREADS) quant_act_kernel(const void* __restrict__ x, int K,
-                                                                int8_t* __restrict__ x_q, float* __restrict__ gamma) {
-    __shared__ unsigned sm[ACT_THREADS / 32];
-    pdl_launch_dependents();
-    pdl_wait();
-    const long long row = blockIdx.x;
-    const char* xr = reinterpret_cast<const char*>(x) + row * (long long)K * (BF16 ? 2 : 4);
-    const int G = K / 16;
+__device__ __forceinline__ void quant_row(const char* xr, int n, int8_t* qr, float* gamma_out, unsigned* sm) {
+    const int G = n / 16;
     float amax = 0.0f;
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
         float v[16];
@@ -108,13 +104,41 @@ __global__ void __launch_bounds__(ACT_THREADS) quant_act_kernel(const void* __re
     amax = block_max_nonneg(amax, sm);
     const float gm = fmaxf(amax, 1e-5f);
     const float s = __fdiv_rn(127.0f, gm);
-    int8_t* qr = x_q + row * (long long)K;
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
         float v[16];
         load16<BF16>(xr, g, v);
         store16(qr, g, v, s);
     }
-    if (threadIdx.x == 0) gamma[row] = gm;
+    if (threadIdx.x == 0) *gamma_out = gm;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(ACT_THREADS) quant_act_kernel(const void* __restrict__ x, int K,
+                                                                int8_t* __restrict__ x_q, float* __restrict__ gamma) {
+    __shared__ unsigned sm[ACT_THREADS / 32];
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long row = blockIdx.x;
+    const char* xr = reinterpret_cast<const char*>(x) + row * (long long)K * (BF16 ? 2 : 4);
+    quant_row<BF16>(xr, K, x_q + row * (long long)K, gamma + row, sm);
+}
+
+// Group quantisation (unite.ai page, "Gruppenquantisierung und
+// -normalisierung"): one CTA per (token m, channel group g) quantises
+// x[m, g*Kg .. (g+1)*Kg) with its own absmax; codes go to the group-major
+// x_q[g][m][:], the scale to gamma[m][g].
+template <bool BF16>
+__global__ void __launch_bounds__(ACT_THREADS) quant_act_grouped_kernel(const void* __restrict__ x, int K, int G,
+                                                                        int M, int8_t* __restrict__ x_q,
+                                                                        float* __restrict__ gamma) {
+    __shared__ unsigned sm[ACT_THREADS / 32];
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long m = blockIdx.x / G;
+    const int g = blockIdx.x % G;
+    const int Kg = K / G;
+    const char* xr = reinterpret_cast<const char*>(x) + (m * K + (long long)g * Kg) * (BF16 ? 2 : 4);
+    quant_row<BF16>(xr, Kg, x_q + ((long long)g * M + m) * Kg, gamma + m * G + g, sm);
 }
 
 // h = combine(a, b) for 16 consecutive elements of group g.
@@ -198,6 +222,16 @@ cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K,
     if (bf16)
         return launch_pdl(quant_act_kernel<true>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
     return launch_pdl(quant_act_kernel<false>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
+}
+
+cudaError_t launch_quant_act_grouped(const void* x, bool bf16, long long M, long long K, int G, int8_t* x_q,
+                                     float* gamma, cudaStream_t st) {
+    const dim3 grid((unsigned)(M * G));
+    if (bf16)
+        return launch_pdl(quant_act_grouped_kernel<true>, grid, dim3(ACT_THREADS), 0, st, x, (int)K, G, (int)M, x_q,
+                          gamma);
+    return launch_pdl(quant_act_grouped_kernel<false>, grid, dim3(ACT_THREADS), 0, st, x, (int)K, G, (int)M, x_q,
+                      gamma);
 }
 
 cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,

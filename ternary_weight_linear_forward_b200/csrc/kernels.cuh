@@ -34,6 +34,8 @@ cudaError_t launch_pack_bits(const int8_t* W_b, long long nwords, uint32_t* W_p,
 // k_act.cu
 cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
                              cudaStream_t st);
+cudaError_t launch_quant_act_grouped(const void* x, bool bf16, long long M, long long K, int G, int8_t* x_q,
+                                     float* gamma, cudaStream_t st);
 cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,
                                  int8_t* x_q, float* gamma, cudaStream_t st);
 
@@ -76,6 +78,13 @@ DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo
 size_t gemm_ws_bytes(long long M, long long N, long long K);
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
                         int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits = 2);
+
+// k_group.cu  (group quantisation along K)
+size_t regroup_ws_bytes(long long N, long long K);
+cudaError_t launch_regroup(const float* W, long long N, long long K, int G, float* out, int num_sms,
+                           cudaStream_t st);
+cudaError_t launch_grouped_rescale(const int* acc, long long acc_stride, const float* gamma, const float* beta, int M,
+                                   int N, int G, void* y, YMode mode, int num_sms, cudaStream_t st);
 
 // Raise a kernel's dynamic shared-memory limit once per device (api.cu).
 cudaError_t ensure_smem_optin(const void* kernel, size_t bytes);
