@@ -63,10 +63,17 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of what defines the decode GEMV's device code: its source, the two
+    device headers it includes, and the output-mode enum it reads (the rest of
+    kernels.cuh declares host launchers)."""
+    import re
+    csrc = os.path.join(ROOT, "ternary_weight_linear_forward_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("k_gemv.cu", "act_inl.cuh", "common.cuh", "kernels.cuh"):
-        with open(os.path.join(ROOT, "ternary_weight_linear_forward_b200", "csrc", name), "rb") as f:
+    for name in ("k_gemv.cu", "act_inl.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(csrc, "kernels.cuh")) as f:
+        h.update(re.search(r"enum YMode[^}]*\}", f.read()).group(0).encode())
     return h.hexdigest()[:16]
 
 
