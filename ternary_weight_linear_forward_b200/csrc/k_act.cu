@@ -170,12 +170,17 @@ __device__ __forceinline__ void combine16(const float* ar, const float* br, int 
     }
 }
 
+// CACHE: the combined row h is kept in dynamic shared memory (K floats)
+// between the two passes, so pass 2 neither re-reads a and b nor evaluates
+// SiLU again; pass 1 (and so every reduction order) is the same either way.
+template <bool CACHE>
 __global__ void __launch_bounds__(ACT_THREADS) quant_act_rms_kernel(const float* __restrict__ a,
                                                                     const float* __restrict__ b, int combine, int K,
                                                                     float* __restrict__ h, int8_t* __restrict__ x_q,
                                                                     float* __restrict__ gamma) {
     __shared__ unsigned smu[ACT_THREADS / 32];
     __shared__ double smd[ACT_THREADS / 32];
+    extern __shared__ float4 hcache[];  // K / 4 entries when CACHE
     pdl_launch_dependents();
     pdl_wait();
     const long long row = blockIdx.x;
@@ -188,6 +193,10 @@ __global__ void __launch_bounds__(ACT_THREADS) quant_act_rms_kernel(const float*
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
         float v[16];
         combine16(ar, br, combine, g, v);
+        if (CACHE) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hcache[4 * g + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
         if (hr) {
             float4* ph = reinterpret_cast<float4*>(hr) + 4 * g;
 #pragma unroll
@@ -207,9 +216,21 @@ __global__ void __launch_bounds__(ACT_THREADS) quant_act_rms_kernel(const float*
     const double ms = __dadd_rn(__ddiv_rn(ss, (double)K), 1e-6);
     const float rho = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(ms)));
     int8_t* qr = x_q + row * (long long)K;
+    // (the block reductions above end in __syncthreads: the cache is complete)
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
         float v[16];
-        combine16(ar, br, combine, g, v);
+        if (CACHE) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 c = hcache[4 * g + i];
+                v[4 * i] = c.x;
+                v[4 * i + 1] = c.y;
+                v[4 * i + 2] = c.z;
+                v[4 * i + 3] = c.w;
+            }
+        } else {
+            combine16(ar, br, combine, g, v);
+        }
         store16(qr, g, v, s);
     }
     if (threadIdx.x == 0) gamma[row] = __fmul_rn(rho, gm);
@@ -236,8 +257,13 @@ cudaError_t launch_quant_act_grouped(const void* x, bool bf16, long long M, long
 
 cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,
                                  int8_t* x_q, float* gamma, cudaStream_t st) {
-    return launch_pdl(quant_act_rms_kernel, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, a, b, combine, (int)K, h,
-                      x_q, gamma);
+    // rows of up to 12288 channels (48 KiB, no opt-in needed) are cached between the passes
+    constexpr long long CACHE_MAX_K = 48 * 1024 / 4;
+    if (x_q && K <= CACHE_MAX_K)
+        return launch_pdl(quant_act_rms_kernel<true>, dim3((unsigned)M), dim3(ACT_THREADS), (size_t)K * 4, st, a, b,
+                          combine, (int)K, h, x_q, gamma);
+    return launch_pdl(quant_act_rms_kernel<false>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, a, b, combine, (int)K,
+                      h, x_q, gamma);
 }
 
 }  // namespace bl
