@@ -179,6 +179,24 @@ def run_cpu_oracle(budget_s: float, max_steps: int | None = None, step=None):
 REF_ROW_FRAC = 1.0 / 8.0
 
 
+def max_over_ranks(t: float, world: int, device) -> float:
+    """The slowest rank's time.  Every rank must call it at the same point
+    (one all-reduce); with one rank the time is returned as it is."""
+    if world <= 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    x = torch.tensor([t], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def job_gbs(bytes_per_rank_step: int, steps: int, world: int, t_max: float) -> float:
+    """Whole-job throughput: every rank moves its bytes per step; the job
+    takes as long as its slowest rank."""
+    return world * bytes_per_rank_step * steps / t_max / 1e9
+
+
 def reference_arm(args):
     """The reference arm is the CPU oracle (there is no other implementation):
     W untimed warm-up steps, then exactly K timed steps, each over the first
@@ -319,13 +337,9 @@ def main():
         torch.cuda.synchronize()
         t_step = timed_run(timed)
     clocks = clk.summary()
-    t_max = t_step
-    if world > 1:
-        t = torch.tensor([t_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(t_step, world, dev)
     ms_per_step = t_max / args.steps * 1e3
-    value = world * step_bytes() * args.steps / t_max / 1e9
+    value = job_gbs(step_bytes(), args.steps, world, t_max)
 
     # ---- roofline of the dominant kernel: one batched GEMV launch per step, so
     # the per-launch time is the timed region's per-step time; each projection
@@ -391,12 +405,7 @@ def main():
         fn()
         e1.record(stream)
         torch.cuda.synchronize()
-        t = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            t_ = torch.tensor([t], device=dev)
-            dist.all_reduce(t_, op=dist.ReduceOp.MAX)
-            t = float(t_.item())
-        return t
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
     def e2e_eager():
         for i in range(n_e2e):
@@ -475,14 +484,14 @@ def main():
             run(eg)
     t_e2e = e2e_timed(e2e_replay)
     del eg
-    e2e = {"value": world * step_bytes() * n_e2e / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_gbs(step_bytes(), n_e2e, world, t_e2e), "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": n_e2e, "us_per_step": t_e2e / n_e2e * 1e6,
            "path": "per step: one pinned H2D copy of both inputs (copy stream) + bitlinear_forward_fp_batch "
                    "(both projections, descriptors marshalled once per buffer set and weight copy) + one D2H copy "
                    f"of both outputs into pinned memory (second copy stream); {NB} buffer sets, so copies of "
                    f"neighbouring steps overlap the kernel; recorded in CUDA graphs of <= {CHUNK} steps and "
                    f"replayed; weights rotate over {copies} copies",
-           "eager": {"value": world * step_bytes() * n_e2e / t_eager / 1e9, "us_per_step": t_eager / n_e2e * 1e6,
+           "eager": {"value": job_gbs(step_bytes(), n_e2e, world, t_eager), "us_per_step": t_eager / n_e2e * 1e6,
                      "path": "the same three operations issued from the host every step on one stream, "
                              "no graph, no overlap"}}
 
