@@ -18,11 +18,18 @@ Each function states the passage it follows.  Sources (web pages):
   "Aktivierungsquantisierung" and eq. 3 "BitLinear-Betrieb"; item 1
   "Gewichtsbinarisierung", eq. 1 -- the 1-bit weights Sign(W - mean(W)).
 
-Pins (tests/test_oracle_pins.py): a hand-worked 4x4 example, closed forms of
-the Gaussian absmean statistics, invariants, brute force on tiny inputs and
-reduction of the contraction to numpy's int64 matmul; the exact |W| sum is
-checked against ``math.fsum``.  Parity unpinned: ``silu_mul`` beyond its
-binary64 error bound (exp is a library routine on both sides).
+Pins (tests/test_oracle_pins.py, tests/test_oracle_binary_pins.py): hand-worked
+4x4 examples for the ternary and the 1-bit weights (tests/golden/), closed
+forms of the Gaussian absmean and mean statistics, invariants, brute force on
+tiny inputs (every 3^8 trit half-word, every 2^16 sign pattern), reduction of
+the contraction to numpy's int64 matmul; the exact |W| and signed sums are
+checked against ``math.fsum`` (sticky-bit ties included).  Composite functions
+are pinned by reduction to pinned parts: ``forward_grouped`` (G = 1 is the
+ungrouped path, duplicated halves, zero groups, power-of-two group scales, its
+binary32 error bound) and ``glu`` (zero gate, oddness in W_up and W_down,
+token independence, the decoder block's MLP half).  Parity unpinned:
+``silu_mul`` beyond its binary64 error bound (exp is a library routine on both
+sides), and so ``glu``'s gated intermediate to the same extent.
 """
 from __future__ import annotations
 
