@@ -425,7 +425,13 @@ bl_status bitlinear_forward_grouped_acc(const int8_t* x_q, int64_t M, int64_t K,
 /* Bytes of device workspace bitlinear_forward_grouped_fp needs. */
 size_t bitlinear_forward_grouped_fp_workspace(int64_t M, int64_t N, int64_t K, int64_t G);
 
-/* bitlinear_quant_act_grouped(x) then bitlinear_forward_grouped, bit-identical to the two calls. */
+/*
+ * bitlinear_quant_act_grouped(x) then bitlinear_forward_grouped, bit-identical
+ * to the two calls.  For one token (M = 1, K/G <= 65536) each group's slice of
+ * x is contiguous: the quantiser then runs inside one GEMV launch over all
+ * groups, which writes every group's binary32 term, and one more kernel adds
+ * them in increasing g (2 launches).
+ */
 bl_status bitlinear_forward_grouped_fp(const void* x, int x_dtype, int64_t M, int64_t K, int64_t G,
                                        const uint32_t* W_p, const float* beta, int64_t N, void* y, int y_dtype,
                                        void* ws, size_t ws_bytes, void* stream);

@@ -746,6 +746,25 @@ bl_status bitlinear_forward_grouped_fp(const void* x, int x_dtype, int64_t M, in
     DevInfo dev;
     s = current_device(dev);
     if (s) return s;
+    const int64_t Kg = K / G;
+    if (M == 1 && gemv_fused_quant_ok(1, Kg)) {
+        // One token: group g of x is the contiguous slice x[g*Kg, (g+1)*Kg), so
+        // every group is one problem of a fused quantiser + GEMV launch that
+        // writes its rescaled binary32 term; a second pass adds them in order.
+        const size_t xe = x_dtype == BL_BF16 ? 2 : 4;
+        const long long stride = group_acc_stride(M, N);
+        float* t = reinterpret_cast<float*>(ws);
+        GemvProblem probs[BL_MAX_GROUPS];
+        for (int64_t g = 0; g < G; ++g)
+            probs[g] = {reinterpret_cast<const char*>(x) + g * Kg * xe, nullptr, W_p + g * N * (Kg / 16), beta + g,
+                        t + g * stride, (int)Kg, (int)N};
+        const cudaError_t e = pick_path(1, probs, (int)G, dev) == PATH_TC
+                                  ? launch_decode_tc(probs, (int)G, 1, x_dtype, Y_F32, dev, as_stream(stream))
+                                  : launch_gemv_fused_group(probs, (int)G, 1, x_dtype, Y_F32, dev, as_stream(stream));
+        if (e != cudaSuccess) return BL_ERR_CUDA;
+        return from_cuda(launch_grouped_sum(t, stride, N, (int)G, y, y_dtype == BL_F32 ? Y_F32 : Y_BF16, dev.num_sms,
+                                            as_stream(stream)));
+    }
     int8_t* x_q = reinterpret_cast<int8_t*>(ws);
     float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
     char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * G * 4);

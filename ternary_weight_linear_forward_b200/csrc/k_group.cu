@@ -12,7 +12,7 @@
 //
 // Storage is group-major ([G][N][K/G] weights, [G][M][K/G] codes), so every
 // group is an ordinary matrix for the existing quantisation, packing and
-// contraction kernels; only the two passes below are particular to groups.
+// contraction kernels; only the passes below are particular to groups.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -62,7 +62,32 @@ __global__ void __launch_bounds__(GROUP_THREADS) grouped_rescale_kernel(const in
     }
 }
 
+// y[m, n] = t_0 + t_1 + ... + t_{G-1} in binary32, in increasing g, where
+// group g's terms t_g (already rescaled) start at t + g * t_stride.
+__global__ void __launch_bounds__(GROUP_THREADS) grouped_sum_kernel(const float* __restrict__ t, long long t_stride,
+                                                                    long long MN, int G, void* __restrict__ y,
+                                                                    int mode) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < MN;
+         i += (long long)gridDim.x * blockDim.x) {
+        float v = __ldcg(t + i);
+        for (int g = 1; g < G; ++g) v = __fadd_rn(v, __ldcg(t + g * t_stride + i));
+        if (mode == Y_F32)
+            reinterpret_cast<float*>(y)[i] = v;
+        else
+            reinterpret_cast<uint16_t*>(y)[i] = f32_to_bf16_rn(v);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_grouped_sum(const float* t, long long t_stride, long long MN, int G, void* y, YMode mode,
+                               int num_sms, cudaStream_t st) {
+    const int grid =
+        (int)std::max<long long>(1, std::min<long long>((MN + GROUP_THREADS - 1) / GROUP_THREADS, (long long)num_sms * 8));
+    return launch_pdl(grouped_sum_kernel, dim3(grid), dim3(GROUP_THREADS), 0, st, t, t_stride, MN, G, y, (int)mode);
+}
 
 size_t regroup_ws_bytes(long long N, long long K) { return (size_t)(N * K * 4 + 255) / 256 * 256; }
 

@@ -83,6 +83,8 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
 size_t regroup_ws_bytes(long long N, long long K);
 cudaError_t launch_regroup(const float* W, long long N, long long K, int G, float* out, int num_sms,
                            cudaStream_t st);
+cudaError_t launch_grouped_sum(const float* t, long long t_stride, long long MN, int G, void* y, YMode mode,
+                               int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_rescale(const int* acc, long long acc_stride, const float* gamma, const float* beta, int M,
                                    int N, int G, void* y, YMode mode, int num_sms, cudaStream_t st);
 

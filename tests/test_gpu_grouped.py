@@ -106,6 +106,8 @@ def test_grouped_bf16(dev):
 @pytest.mark.parametrize("engine", ["cuda_cores", "tensor_cores"])
 def test_grouped_engines(dev, engine):
     with bl.decode_engine(engine):
+        run_case(dev, 1, 4096, 3000, 4, 69)      # one token: quantiser fused per group
+        run_case(dev, 1, 2048, 500, 8, 68, y_dtype="bf16", x_dtype="bf16")
         run_case(dev, 2, 4096, 3000, 4, 70)
         run_case(dev, 12, 4096, 900, 2, 71)
 
