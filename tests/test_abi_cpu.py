@@ -297,3 +297,45 @@ def test_grouped_validation():
     assert wsf > ws
     assert h(P(A1), 0, 3, 512, 4, P(A3), P(A4), 100, P(A5), 0, P(A6), wsf, None) == DEVICE
     assert h(P(A1), 0, 3, 512, 4, P(A3), P(A4), 100, P(A5), 0, P(A6), wsf - 1, None) == WS
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "bitlinear.h"
+
+/* A plain C client: only calls whose arguments fail host validation, so
+   nothing reaches a device. */
+int main(void) {
+    int bad = 0;
+    if (strcmp(bitlinear_status_string(BL_OK), "ok") != 0) bad |= 1;
+    if (bitlinear_forward(NULL, NULL, 1, 1024, NULL, NULL, 64, NULL, BL_F32, NULL, 0, NULL) != BL_ERR_NULL) bad |= 2;
+    if (bitlinear_pack((const int8_t*)16, 4, 24, (uint32_t*)4096, NULL) != BL_ERR_SHAPE) bad |= 4;
+    if (bitlinear_forward_workspace(2048, 4096, 4096) < 2048 * 4) bad |= 8;
+    if (bitlinear_set_decode_engine(99) != BL_ERR_SHAPE) bad |= 16;
+    if (bitlinear_forward_grouped_workspace(1, 64, 512, 3) != 0) bad |= 32;
+    printf("%d\n", bad);
+    return bad;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_runs():
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(B.LIB_PATH)
+    out = os.path.join(libdir, "_build")          # the library's own (git-ignored) build folder
+    os.makedirs(out, exist_ok=True)
+    src = os.path.join(out, "abi_client.c")
+    with open(src, "w") as f:
+        f.write(C_CLIENT)
+    exe = os.path.join(out, "abi_client")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                        "-L", libdir, "-l:libbitlinear.so", "-Wl,-rpath," + libdir, "-o", exe],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "0", (r.returncode, r.stdout, r.stderr)
