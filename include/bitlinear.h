@@ -341,7 +341,10 @@ enum { BL_COMBINE_NONE = 0, BL_COMBINE_ADD = 1, BL_COMBINE_SILU_MUL = 2 };
  *           = a + b            (binary32 add)     (BL_COMBINE_ADD)
  *           = (float)(silu(a) * b), silu(a) = a / (1 + exp(-a)), in binary64
  *                                                 (BL_COMBINE_SILU_MUL)
- *   rho_m   = (float)(1 / sqrt(mean_k h^2 + 1e-6))    (binary64, then rounded)
+ *   rho_m   = (float)(1 / sqrt(mean_k h^2 + 1e-6))    (binary64, then rounded; the
+ *             binary64 sum of squares is added in an order of the kernel's choosing,
+ *             so rho can differ by one binary32 ulp from a sequential sum when that
+ *             sum lies within its rounding error of a binary32 rounding boundary)
  * absmax quantisation is invariant under the positive per-token scale rho,
  * so the codes are those of bitlinear_quant_act applied to h, and
  *   gamma[m] = rho_m * max(max_k |h[m, k]|, 1e-5)       (binary32 multiply).
