@@ -19,7 +19,7 @@ Each function states the passage it follows.  Sources (web pages):
   "Gewichtsbinarisierung", eq. 1 -- the 1-bit weights Sign(W - mean(W)).
 
 Pins (tests/test_oracle_pins.py, tests/test_oracle_binary_pins.py): hand-worked
-4x4 examples for the ternary and the 1-bit weights (tests/golden/), closed
+examples for the ternary, the 1-bit and the grouped weights (tests/golden/), closed
 forms of the Gaussian absmean and mean statistics, invariants, brute force on
 tiny inputs (every 3^8 trit half-word, every 2^16 sign pattern), reduction of
 the contraction to numpy's int64 matmul; the exact |W| and signed sums are

@@ -468,3 +468,25 @@ def test_grouped_zero_group_and_group_scales():
     _, gam = oracle.quant_act_grouped(x, 4)
     for g in range(4):
         np.testing.assert_array_equal(gam[:, g], np.maximum(np.abs(x[:, 64 * g:64 * (g + 1)]).max(1), 1e-5))
+
+
+def test_hand_grouped_example():
+    rows = {}
+    with open(os.path.join(GOLDEN, "hand_grouped_2x8.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows.setdefault(key, []).append(vals)
+    W = np.array([[float(v) for v in r] for r in rows["W"]], np.float32)
+    W_t, beta = oracle.quantize_weights_grouped(W, 2)
+    np.testing.assert_array_equal(beta, np.array([float(v) for v in rows["beta"][0]], np.float32))
+    np.testing.assert_array_equal(W_t, np.array([[int(v) for v in r] for r in rows["W_t"]], np.int8))
+    x = np.array([[float(v) for v in rows["x"][0]]], np.float32)
+    r = oracle.forward_grouped(x, W_t, beta, 2)
+    np.testing.assert_array_equal(r["gamma"][0], [float(v) for v in rows["gamma"][0]])
+    np.testing.assert_array_equal(r["x_q"][0], [int(v) for v in rows["x_q"][0]])
+    np.testing.assert_array_equal(r["acc"][:, 0, :], [[int(v) for v in rows["acc0"][0]], [int(v) for v in rows["acc1"][0]]])
+    exact = np.array([float(Fraction(v)) for v in rows["y"][0]])
+    np.testing.assert_allclose(r["y64"][0], exact, rtol=1e-15, atol=0)
+    assert (np.abs(r["y"][0] - exact) <= 4 * 2.0 ** -24 * r["yabs64"][0]).all()
