@@ -122,6 +122,18 @@ def test_binarize_special_matrices(dev):
     check_weights(W, dev)
 
 
+@pytest.mark.parametrize("name", ["gaussian_with_tiny_tail", "every_exponent", "subnormal_only", "one_huge",
+                                  "small_mass", "above_a_tie"])
+def test_binarize_exact_over_the_whole_binary32_range(dev, name):
+    # alpha (the signed mean) and beta (the absmean) are the exact means
+    # whatever the ratio of an element to the largest; the small elements are
+    # given a nonzero signed total
+    from test_gpu_parity import _wide_range_matrices
+    W = _wide_range_matrices()[name].copy()
+    W[W.shape[0] // 2:] = np.abs(W[W.shape[0] // 2:])
+    check_weights(W, dev)
+
+
 def test_pack_bits_of_arbitrary_codes(dev):
     rng = np.random.default_rng(8)
     W_b = rng.integers(-2, 3, (300, 512)).astype(np.int8)   # values <= 0 pack as -1
