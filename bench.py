@@ -90,6 +90,38 @@ def recorded_traffic():
     return d.get("dram_bytes_per_launch")
 
 
+_CUDA_DRV = None
+
+
+def upload_graphs(gs, stream) -> bool:
+    """Upload each graph's executable to the device on `stream` (driver
+    cuGraphUpload), so that its first replay does not pay for it.  Returns
+    False where the driver entry point is not available."""
+    global _CUDA_DRV
+    import ctypes
+    if _CUDA_DRV is None:
+        try:
+            _CUDA_DRV = ctypes.CDLL("libcuda.so.1")
+            _CUDA_DRV.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+            _CUDA_DRV.cuGraphUpload.restype = ctypes.c_int
+        except (OSError, AttributeError):
+            _CUDA_DRV = False
+    if not _CUDA_DRV:
+        return False
+    ok = True
+    for g in gs:
+        rc = _CUDA_DRV.cuGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()), ctypes.c_void_p(stream.cuda_stream))
+        ok = ok and rc == 0
+    return ok
+
+
+def lead_cycles(n_graphs: int) -> int:
+    """Device-side spin queued ahead of a timed region: long enough (about
+    50 us plus 25 us per graph at ~2 GHz) for the host to submit the graphs
+    before the start event is reached."""
+    return int((50 + 25 * n_graphs) * 2000)
+
+
 class ClockSampler:
     """nvidia-smi SM clock / throttle-reason sampler (reads only)."""
 
@@ -179,6 +211,69 @@ def run_cpu_oracle(budget_s: float, max_steps: int | None = None, step=None):
 REF_ROW_FRAC = 1.0 / 8.0
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_child(setting: str, budget_s: float):
+    """Run inside a child process: time the oracle on the full decode step
+    (both projections) and print one JSON line.  `single`: the plain build,
+    the process pinned to one core; `all`: the OpenMP build of the same
+    source on every core the process may use."""
+    cores = sorted(os.sched_getaffinity(0))
+    if setting == "single":
+        os.sched_setaffinity(0, {cores[0]})
+        threads = 1
+    else:
+        threads = len(cores)
+    step, _ = cpu_oracle_step_fn()
+    n, el = run_cpu_oracle(budget_s, step=step)
+    print(json.dumps({"steps": n, "seconds": el, "threads": threads,
+                      "cpus": sorted(os.sched_getaffinity(0))[:4]}), flush=True)
+
+
+def cpu_baseline(budget_s: float):
+    """The oracle, as it stands, timed on the host in two settings (one
+    pinned core; all cores with the OpenMP build), each in a child process
+    that touches no GPU.  Returns the cpu_baseline object of the JSON line."""
+    out = {}
+    ncores = len(os.sched_getaffinity(0))
+    for setting in ("single", "all"):
+        env = dict(os.environ)
+        if setting == "all":
+            env.update(ORACLE_OPENMP="1", OMP_NUM_THREADS=str(ncores), OMP_PROC_BIND="spread")
+        else:
+            env.update(OMP_NUM_THREADS="1")
+        env["CUDA_VISIBLE_DEVICES"] = ""
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--cpu-baseline-child", setting,
+                            "--cpu-budget", str(budget_s)], env=env, capture_output=True, text=True,
+                           timeout=budget_s * 20 + 600)
+        if r.returncode != 0:
+            out[setting] = {"error": (r.stderr or r.stdout)[-300:]}
+            continue
+        d = json.loads(r.stdout.strip().splitlines()[-1])
+        out[setting] = {"value": step_bytes() * d["steps"] / d["seconds"] / 1e9, "cores": d["threads"],
+                        "ms_per_step": d["seconds"] / d["steps"] * 1e3,
+                        "sample": f"{d['steps']} full steps of the workload (both projections) in "
+                                  f"{d['seconds']:.1f} s"}
+    main = out.get("all", {})
+    one = out.get("single", {})
+    return {"value": main.get("value"), "unit": "GB/s", "cores": main.get("cores"), "kind": "oracle",
+            "sample": ("the plain C oracle, compiled a second time with -fopenmp (the (m, n) pairs of the integer "
+                       "contraction shared among threads, arithmetic unchanged), on every host core; "
+                       + main.get("sample", main.get("error", ""))),
+            "single_core": dict(one, kind="oracle", pinned="one core (sched_setaffinity)",
+                                build="plain gcc -O2"),
+            "cpu_model": cpu_model(), "host_cores": ncores}
+
+
 def max_over_ranks(t: float, world: int, device) -> float:
     """The slowest rank's time.  Every rank must call it at the same point
     (one all-reduce); with one rank the time is returned as it is."""
@@ -241,7 +336,12 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="run the decode step only (no extra sections)")
     ap.add_argument("--sections", default="prefill,small,block,binary,glu,grouped",
                     help="extra measured sections after the decode step, comma separated")
+    ap.add_argument("--cpu-baseline-child", choices=["single", "all"], help=argparse.SUPPRESS)
+    ap.add_argument("--cpu-budget", type=float, default=float(os.environ.get("BENCH_CPU_BUDGET_S", "12")))
     args = ap.parse_args()
+    if args.cpu_baseline_child:
+        cpu_baseline_child(args.cpu_baseline_child, args.cpu_budget)
+        return 0
     sections = set() if args.no_prefill else {x for x in args.sections.split(",") if x}
     if args.warmup < 3:
         args.warmup = 3
@@ -319,11 +419,18 @@ def main():
             g.replay()
 
     def timed_run(gs):
+        # The graphs are uploaded to the device before the start event, and a
+        # short device-side spin is queued ahead of it, so the timed region
+        # holds exactly the replayed steps: neither the first replay's upload
+        # nor the host's submission of the first graph falls inside it.
         if world > 1:
             dist.barrier()
+        upload_graphs(gs, stream)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(lead_cycles(len(gs)))
         e0.record(stream)
         with torch.cuda.stream(stream):
             run(gs)
@@ -331,12 +438,13 @@ def main():
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / 1e3
 
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            run(warm)
-        torch.cuda.synchronize()
-        t_step = timed_run(timed)
-    clocks = clk.summary()
+    # SM clocks are sampled over the whole measured part of the run (the timed
+    # decode region alone is far shorter than one sampling period)
+    clk = ClockSampler(local).__enter__()
+    with torch.cuda.stream(stream):
+        run(warm)
+    torch.cuda.synchronize()
+    t_step = timed_run(timed)
     t_max = max_over_ranks(t_step, world, dev)
     ms_per_step = t_max / args.steps * 1e3
     value = job_gbs(step_bytes(), args.steps, world, t_max)
@@ -717,14 +825,14 @@ def main():
             del g, sets, x, y, ws
         del base
 
+    clk.__exit__()
+    clocks = clk.summary()
+    clocks["window"] = "whole GPU part of the run (decode warm-up and timed steps, roofline, e2e and sections)"
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fn, _ = cpu_oracle_step_fn()
-        n, el = run_cpu_oracle(float(os.environ.get("BENCH_CPU_BUDGET_S", "12")), step=fn)
-        cpu = {"value": step_bytes() * n / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} full steps of the workload (both projections), about "
-                         f"{float(os.environ.get('BENCH_CPU_BUDGET_S', '12')):.0f} s of one host core"}
+        cpu = cpu_baseline(args.cpu_budget)
 
     if rank == 0:
         line = {

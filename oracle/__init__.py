@@ -40,7 +40,9 @@ import numpy as np
 
 from . import build as _build
 
-_lib = ctypes.CDLL(_build.build())
+# ORACLE_OPENMP=1 loads the -fopenmp build of the same source (the
+# benchmark's all-core CPU baseline); results are identical.
+_lib = ctypes.CDLL(_build.build_omp() if os.environ.get("ORACLE_OPENMP") == "1" else _build.build())
 
 _f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")

@@ -7,7 +7,10 @@
  *
  * Built with gcc -O2 -fno-fast-math -ffp-contract=off (SSE arithmetic on
  * x86-64, so every float operation below is one IEEE binary32 operation with
- * round-to-nearest-even, and nothing is fused into an FMA).
+ * round-to-nearest-even, and nothing is fused into an FMA).  A second build of
+ * the same source with -fopenmp (liboracle_omp.so) only shares the integer
+ * contraction's (m, n) pairs among threads; it exists for the benchmark's
+ * all-core CPU baseline.
  *
  * Sources (web pages on ternary-weight linear layers):
  *   [MMF]  DataCamp blog "MatMul-free language models" (Dutch), section
@@ -289,6 +292,9 @@ void orc_quant_act(const float* x, int64_t M, int64_t K, int8_t* x_q, float* gam
  * contraction acc[m, n] = sum_k W_t[n, k] * x_hat[m, k], written literally. */
 void orc_ternary_acc(const int8_t* x_q, int64_t M, int64_t K, const int8_t* W_t, int64_t N, int32_t* acc)
 {
+    /* Every (m, n) is independent; an OpenMP build (the benchmark's all-core
+     * CPU baseline) shares them out, a plain build ignores the pragma. */
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             const int8_t* xr = x_q + m * K;
