@@ -80,12 +80,14 @@ size_t bitlinear_quantize_weights_workspace(int64_t N, int64_t K);
  * absmean ternarisation, [MMF] "MatMul vervangen door ternaire bewerkingen":
  *   beta   = mean over all N*K elements of |W|          (one scale per matrix)
  *   W_t    = clip(round(W / (beta + eps)), -1, 1)        (ties to even)
- * beta is the exact sum of |W| rounded to binary64, divided by N*K in
- * binary64 and rounded to binary32.  The sum is taken in fixed point: with
- * E the binary32 exponent of max|W|, every |w| is truncated to a multiple of
- * 2^(E-38-23) (exact for |w| >= 2^-38 max|W|) and the integers are added
- * exactly, so the result does not depend on thread order.  The divisor
- * beta + eps and the quotient are binary32 (IEEE add, IEEE divide).
+ * beta is the exact sum of |W| rounded once to binary64, divided by N*K in
+ * binary64 and rounded to binary32, for every finite W (subnormals
+ * included).  The sum is taken in exact integer arithmetic, so it does not
+ * depend on thread order: an element within 2^38 of max|W| is an integer on
+ * the grid 2^(E-188) (E the biased exponent of max|W|), a smaller one an
+ * integer on the grid 2^-149, and all are added without rounding before the
+ * one conversion.  The divisor beta + eps and the quotient are binary32
+ * (IEEE add, IEEE divide).
  *   W    [N, K] float32, device, read only
  *   W_t  [N, K] int8 out, values in {-1, 0, 1}
  *   beta [1] float32 out (stays on the device)
@@ -269,10 +271,10 @@ size_t bitlinear_binarize_weights_workspace(int64_t N, int64_t K);
  *   W_b   [N, K] int8 out, values in {-1, +1}
  *   alpha [1] float32 out, beta [1] float32 out (distinct buffers)
  *   ws    >= bitlinear_binarize_weights_workspace(N, K) bytes of device scratch
- * K % 32 == 0.  Sums are exact integers on a grid set by max |W| and do not
- * depend on thread order; alpha and beta are the exact means (as defined
- * above) whenever every nonzero |w| >= 2^-38 * max |W|, and elements below
- * that are truncated to the grid.
+ * K % 32 == 0.  The sums of the positive and of the negative elements are
+ * exact integers (as for bitlinear_quantize_weights) and do not depend on
+ * thread order, so alpha and beta are the exact means defined above for
+ * every finite W.
  */
 bl_status bitlinear_binarize_weights(const float* W, int64_t N, int64_t K, int8_t* W_b, float* alpha,
                                      float* beta, void* ws, size_t ws_bytes, void* stream);
@@ -481,8 +483,11 @@ enum {
                                     for M <= 4, the swap-AB decode kernel for 5 <= M <= 16
                                     where it fits, the tcgen05 GEMM otherwise */
     BL_ENGINE_CUDA_CORES = 1,    /* M <= 64 on CUDA cores (masked byte dot products) */
-    BL_ENGINE_TENSOR_CORES = 2   /* M <= 16 on the swap-AB tcgen05 decode kernel where it
+    BL_ENGINE_TENSOR_CORES = 2,  /* M <= 16 on the swap-AB tcgen05 decode kernel where it
                                     fits (weight rows on the MMA's 128 lanes), else as AUTO */
+    BL_ENGINE_CUDA_CORES_GENERAL = 3  /* as BL_ENGINE_CUDA_CORES, but one token also runs the
+                                         general small-M kernel instead of the one-token
+                                         streaming kernel */
 };
 
 /*
@@ -513,6 +518,21 @@ bl_status bitlinear_device_status(void* stream);
 
 /* Number of SMs of the current device as seen by the library (0 if none). */
 int bitlinear_num_sms(void);
+
+/*
+ * Test hook of the bounded waits (no counterpart on the pages).  With
+ * enable != 0, the next one-token decode launch of this process (the
+ * streaming CUDA-core GEMV that bitlinear_forward, _fp, _fp_batch, _acc and
+ * _noalloc run for M = 1) limits each of its waits to about 10^5 SM cycles,
+ * and the weight producer of its first CTA issues no copies, so that CTA's
+ * consumers give up waiting for data that never comes: the kernel raises the
+ * device error word and returns (no copy is in flight, nothing hangs), that
+ * CTA's outputs are unspecified, and the next bitlinear_device_status returns
+ * BL_ERR_TIMEOUT.  The request applies to one launch and then clears itself;
+ * enable == 0 withdraws it.  A launch recorded into a CUDA graph keeps it.
+ * Always returns BL_OK.
+ */
+bl_status bitlinear_test_expire_next_wait(int enable);
 
 #ifdef __cplusplus
 }

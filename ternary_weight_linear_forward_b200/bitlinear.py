@@ -63,6 +63,7 @@ SIGNATURES = {
     "bitlinear_get_decode_engine": (_I, []),
     "bitlinear_device_status": (_I, [_P]),
     "bitlinear_num_sms": (_I, []),
+    "bitlinear_test_expire_next_wait": (_I, [_I]),
 }
 
 
@@ -122,6 +123,45 @@ def _need(t, dtype, ndim, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_out(out, shape, dtypes, device, name="out"):
+    """A caller-given output buffer: the library writes shape-many elements
+    through its pointer, so the size, dtype, device and layout are checked
+    here, where they are known."""
+    if not isinstance(out, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if out.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {dtypes}, got {out.dtype}")
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    if out.device != device:
+        raise ValueError(f"{name} must be on {device}, got {out.device}")
+    if not out.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_len(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _same_device(device, **tensors):
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _check_ws(ws, device):
+    if ws is None:
+        return
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise TypeError("ws must be a contiguous torch.uint8 tensor")
+    if ws.device != device:
+        raise ValueError(f"ws must be on {device}, got {ws.device}")
+
+
+FLOAT_OUT = (torch.float32, torch.bfloat16)
+
+
 # --------------------------------------------------------------------------
 # entry points
 # --------------------------------------------------------------------------
@@ -160,6 +200,8 @@ def quant_act(x: torch.Tensor, out=None, stream=None):
         gamma = torch.empty(max(M, 4), dtype=torch.float32, device=x.device)[:M]
     else:
         x_q, gamma = out
+        _check_out(x_q, (M, K), (torch.int8,), x.device, "x_q")
+        _check_out(gamma, (M,), (torch.float32,), x.device, "gamma")
     dt = BL_BF16 if x.dtype == torch.bfloat16 else BL_F32
     _check("bitlinear_quant_act",
            lib().bitlinear_quant_act(_ptr(x), dt, M, K, _ptr(x_q), _ptr(gamma), _stream(stream)))
@@ -181,8 +223,13 @@ def forward(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, beta: tor
     N = W_p.shape[0]
     if W_p.shape[1] * 16 != K:
         raise ValueError("W_p must be [N, K/16]")
+    _check_len(gamma, (M,), "gamma")
+    _check_len(beta, (1,), "beta")
+    _same_device(x_q.device, gamma=gamma, W_p=W_p, beta=beta)
+    _check_ws(ws, x_q.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    _check_out(out, (M, N), FLOAT_OUT, x_q.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = forward_workspace(M, N, K)
     if nws and ws is None:
@@ -209,8 +256,12 @@ def forward_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, out_dtype
     N = W_p.shape[0]
     if W_p.shape[1] * 16 != K:
         raise ValueError("W_p must be [N, K/16]")
+    _check_len(beta, (1,), "beta")
+    _same_device(x.device, W_p=W_p, beta=beta)
+    _check_ws(ws, x.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(out, (M, N), FLOAT_OUT, x.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = int(lib().bitlinear_forward_fp_workspace(M, N, K))
     if nws and ws is None:
@@ -280,9 +331,14 @@ def _pack_batch(problems, out_dtype):
         N = W_p.shape[0]
         if W_p.shape[1] * 16 != K:
             raise ValueError("W_p must be [N, K/16]")
+        if quantised:
+            _check_len(gamma, (M,), "gamma")
+        _check_len(beta, (1,), "beta")
+        _same_device(x0.device, x=x, gamma=gamma if quantised else None, W_p=W_p, beta=beta)
         out = pr.get("out")
         if out is None:
             out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+        _check_out(out, (M, N), FLOAT_OUT, x0.device)
         outs.append(out)
         arr[i] = _Problem(x.data_ptr(), gamma.data_ptr() if quantised else None, W_p.data_ptr(), beta.data_ptr(),
                           out.data_ptr(), K, N)
@@ -308,8 +364,12 @@ def forward_noalloc(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, b
     N = W_p.shape[0]
     if W_p.shape[1] * 16 != K:
         raise ValueError("W_p must be [N, K/16]")
+    _check_len(gamma, (M,), "gamma")
+    _check_len(beta, (1,), "beta")
+    _same_device(x_q.device, gamma=gamma, W_p=W_p, beta=beta)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    _check_out(out, (M, N), FLOAT_OUT, x_q.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     _check("bitlinear_forward_noalloc",
            lib().bitlinear_forward_noalloc(_ptr(x_q), _ptr(gamma), M, K, _ptr(W_p), _ptr(beta), N, _ptr(out), dt,
@@ -325,6 +385,8 @@ def forward_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=None) -> t
     N = W_p.shape[0]
     if W_p.shape[1] * 16 != K:
         raise ValueError("W_p must be [N, K/16]")
+    _same_device(x_q.device, W_p=W_p)
+    _check_ws(ws, x_q.device)
     acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
     nws = forward_workspace(M, N, K)
     if nws and ws is None:
@@ -379,8 +441,13 @@ def forward_binary(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, be
     _need(beta, torch.float32, 1, "beta")
     M, K = x_q.shape
     N = _bits_shape(W_p, K)
+    _check_len(gamma, (M,), "gamma")
+    _check_len(beta, (1,), "beta")
+    _same_device(x_q.device, gamma=gamma, W_p=W_p, beta=beta)
+    _check_ws(ws, x_q.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    _check_out(out, (M, N), FLOAT_OUT, x_q.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = int(lib().bitlinear_forward_binary_workspace(M, N, K))
     if nws and ws is None:
@@ -397,6 +464,8 @@ def forward_binary_acc(x_q: torch.Tensor, W_p: torch.Tensor, ws=None, stream=Non
     _need(W_p, torch.int32, 2, "W_p")
     M, K = x_q.shape
     N = _bits_shape(W_p, K)
+    _same_device(x_q.device, W_p=W_p)
+    _check_ws(ws, x_q.device)
     acc = torch.empty((M, N), dtype=torch.int32, device=x_q.device)
     nws = int(lib().bitlinear_forward_binary_workspace(M, N, K))
     if nws and ws is None:
@@ -417,8 +486,12 @@ def forward_binary_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, ou
     _need(beta, torch.float32, 1, "beta")
     M, K = x.shape
     N = _bits_shape(W_p, K)
+    _check_len(beta, (1,), "beta")
+    _same_device(x.device, W_p=W_p, beta=beta)
+    _check_ws(ws, x.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(out, (M, N), FLOAT_OUT, x.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = int(lib().bitlinear_forward_binary_fp_workspace(M, N, K))
     if nws and ws is None:
@@ -439,14 +512,21 @@ def quant_act_rms(a: torch.Tensor, b: torch.Tensor | None = None, combine: str =
     if b is not None:
         _need(b, torch.float32, 2, "b")
     M, K = a.shape
+    if b is not None:
+        _check_len(b, (M, K), "b")
+        _same_device(a.device, b=b)
     if want_h and h is None:
         h = torch.empty_like(a)
+    if h is not None:
+        _check_out(h, (M, K), (torch.float32,), a.device, "h")
     if quantize:
         if out is None:
             x_q = torch.empty((M, K), dtype=torch.int8, device=a.device)
             gamma = torch.empty(max(M, 4), dtype=torch.float32, device=a.device)[:M]
         else:
             x_q, gamma = out
+            _check_out(x_q, (M, K), (torch.int8,), a.device, "x_q")
+            _check_out(gamma, (M,), (torch.float32,), a.device, "gamma")
     else:
         x_q = gamma = None
     _check("bitlinear_quant_act_rms",
@@ -455,11 +535,12 @@ def quant_act_rms(a: torch.Tensor, b: torch.Tensor | None = None, combine: str =
     return h, x_q, gamma
 
 
-ENGINES = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
+ENGINES = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2, "cuda_cores_general": 3}
 
 
 def set_decode_engine(name: str):
-    """Engine of later decode calls (M <= 64): 'auto', 'cuda_cores' or 'tensor_cores'."""
+    """Engine of later decode calls (M <= 64): 'auto', 'cuda_cores', 'tensor_cores' or
+    'cuda_cores_general' (CUDA cores without the one-token streaming kernel)."""
     if name not in ENGINES:
         raise ValueError(f"unknown decode engine {name!r}")
     _check("bitlinear_set_decode_engine", lib().bitlinear_set_decode_engine(ENGINES[name]))
@@ -566,8 +647,13 @@ def forward_grouped(x_q: torch.Tensor, gamma: torch.Tensor, W_p: torch.Tensor, b
     G, M, Kg = x_q.shape
     K = G * Kg
     N = _grouped_shapes(W_p, G, K)
+    _check_len(gamma, (M, G), "gamma")
+    _check_len(beta, (G,), "beta")
+    _same_device(x_q.device, gamma=gamma, W_p=W_p, beta=beta)
+    _check_ws(ws, x_q.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x_q.device)
+    _check_out(out, (M, N), FLOAT_OUT, x_q.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = int(lib().bitlinear_forward_grouped_workspace(M, N, K, G))
     if ws is None:
@@ -584,6 +670,7 @@ def forward_grouped_acc(x_q: torch.Tensor, W_p: torch.Tensor, stream=None) -> to
     G, M, Kg = x_q.shape
     K = G * Kg
     N = _grouped_shapes(W_p, G, K)
+    _same_device(x_q.device, W_p=W_p)
     S = (M * N + 3) // 4 * 4
     acc = torch.empty(G * S, dtype=torch.int32, device=x_q.device)
     nws = int(lib().bitlinear_forward_grouped_workspace(M, N, K, G))
@@ -604,8 +691,11 @@ def forward_grouped_fp(x: torch.Tensor, W_p: torch.Tensor, beta: torch.Tensor, o
     M, K = x.shape
     G = beta.shape[0]
     N = _grouped_shapes(W_p, G, K)
+    _same_device(x.device, W_p=W_p, beta=beta)
+    _check_ws(ws, x.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(out, (M, N), FLOAT_OUT, x.device)
     dt = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}[out.dtype]
     nws = int(lib().bitlinear_forward_grouped_fp_workspace(M, N, K, G))
     if ws is None:
@@ -631,7 +721,12 @@ def glu_forward(x: torch.Tensor, gate, up, down, want_u: bool = False, out=None,
     F = Wg.shape[0]
     if Wg.shape[1] * 16 != D or Wu.shape != Wg.shape or Wd.shape[0] != D or Wd.shape[1] * 16 != F:
         raise ValueError("W_gate and W_up must be [F, D/16], W_down [D, F/16]")
+    for t, n in ((bg, "beta_gate"), (bu, "beta_up"), (bd, "beta_down")):
+        _check_len(t, (1,), n)
+    _same_device(x.device, W_gate=Wg, W_up=Wu, W_down=Wd, beta_gate=bg, beta_up=bu, beta_down=bd)
+    _check_ws(ws, x.device)
     y = torch.empty((M, D), dtype=torch.float32, device=x.device) if out is None else out
+    _check_out(y, (M, D), (torch.float32,), x.device)
     u = torch.empty((M, F), dtype=torch.float32, device=x.device) if want_u else None
     nws = int(lib().bitlinear_glu_workspace(M, D, F))
     if ws is None:

@@ -85,6 +85,7 @@ bl_status check_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_
 constexpr int GEMV_MAX_M = 64;
 
 std::atomic<int> g_engine{BL_ENGINE_AUTO};
+std::atomic<int> g_expire_next_wait{0};
 
 // Which kernel runs a problem set of M tokens.  Measured on B200 (4096 x 4096
 // and 4096 x 11008, x_q given): a kind::i8 tcgen05 MMA costs about the same
@@ -98,7 +99,7 @@ constexpr int AUTO_CUDA_MAX_M = 4;
 DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
     if (M > GEMV_MAX_M) return PATH_GEMM;
     const int engine = g_engine.load(std::memory_order_relaxed);
-    if (engine == BL_ENGINE_CUDA_CORES) return PATH_CUDA;
+    if (engine == BL_ENGINE_CUDA_CORES || engine == BL_ENGINE_CUDA_CORES_GENERAL) return PATH_CUDA;
     const bool tc_first = engine == BL_ENGINE_TENSOR_CORES || M > AUTO_CUDA_MAX_M;
     if (tc_first && M <= decode_tc_max_m()) {
         bool ok = true;
@@ -122,7 +123,7 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
     if (path == PATH_TC)
         e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
     else if (path == PATH_CUDA)
-        e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev, as_stream(stream));
+        e = launch_decode_cuda(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
     return from_cuda(e);
@@ -175,7 +176,7 @@ bl_status run_grouped_acc(const int8_t* x_q, int64_t M, int64_t K, int64_t G, co
             probs[g] = {x_q + g * M * Kg, nullptr, W_p + g * N * (Kg / 16), nullptr, acc + g * stride, (int)Kg, (int)N};
         const cudaError_t e = pick_path((int)M, probs, (int)G, dev) == PATH_TC
                                   ? launch_decode_tc(probs, (int)G, (int)M, BL_I8, Y_ACC, dev, as_stream(stream))
-                                  : launch_gemv_fused_group(probs, (int)G, (int)M, BL_I8, Y_ACC, dev, as_stream(stream));
+                                  : launch_decode_cuda(probs, (int)G, (int)M, BL_I8, Y_ACC, dev, as_stream(stream));
         return from_cuda(e);
     }
     for (int64_t g = 0; g < G; ++g) {
@@ -195,6 +196,25 @@ size_t grouped_ws(int64_t M, int64_t N, int64_t K, int64_t G) {
 
 DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
     return pick_path(M, probs, count, dev);
+}
+
+bool take_wait_expiry_request() { return g_expire_next_wait.exchange(0, std::memory_order_relaxed) != 0; }
+
+// Whether the automatic engine runs one token on the streaming one-token
+// kernel (else on the general small-M kernel); BL_ENGINE_CUDA_CORES always
+// does where the kernel applies.
+constexpr bool AUTO_ONE_TOKEN_STREAMING = false;
+
+cudaError_t launch_decode_cuda(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
+                               const DevInfo& dev, cudaStream_t st) {
+    const int engine = g_engine.load(std::memory_order_relaxed);
+    const bool streaming = engine == BL_ENGINE_CUDA_CORES || (engine == BL_ENGINE_AUTO && AUTO_ONE_TOKEN_STREAMING);
+    if (M == 1 && streaming && gemv1_ok(probs, count, M, dev)) return launch_gemv1(probs, count, x_dtype, mode, dev, st);
+    const GemvProblem& q = probs[0];
+    if (count == 1 && x_dtype == BL_I8)
+        return launch_gemv(static_cast<const int8_t*>(q.x), q.gamma, M, q.K, q.W_p, q.beta, q.N, q.y, mode, dev, st);
+    if (count == 1) return launch_gemv_fused(q.x, x_dtype == BL_BF16, M, q.K, q.W_p, q.beta, q.N, q.y, mode, dev, st);
+    return launch_gemv_fused_group(probs, count, M, x_dtype, mode, dev, st);
 }
 
 cudaError_t ensure_smem_optin(const void* kernel, size_t bytes) {
@@ -391,8 +411,7 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
     if (M <= 4 && pick_path((int)M, &prob, 1, dev) == PATH_TC)  // quantiser fused, workspace unused
         return from_cuda(launch_decode_tc(&prob, 1, (int)M, x_dtype, mode, dev, as_stream(stream)));
     if (!need)
-        return from_cuda(launch_gemv_fused(x, x_dtype == BL_BF16, (int)M, (int)K, W_p, beta, (int)N, y, mode, dev,
-                                           as_stream(stream)));
+        return from_cuda(launch_decode_cuda(&prob, 1, (int)M, x_dtype, mode, dev, as_stream(stream)));
     int8_t* x_q = reinterpret_cast<int8_t*>(ws);
     float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
     char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * 4);
@@ -439,7 +458,7 @@ bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int6
     const YMode mode = y_dtype == BL_F32 ? Y_F32 : Y_BF16;
     if (pick_path((int)M, probs, count, dev) == PATH_TC)
         return from_cuda(launch_decode_tc(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
-    return from_cuda(launch_gemv_fused_group(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
+    return from_cuda(launch_decode_cuda(probs, count, (int)M, x_dtype, mode, dev, as_stream(stream)));
 }
 
 size_t bitlinear_forward_binary_workspace(int64_t M, int64_t N, int64_t K) { return forward_bits_ws(M, N, K); }
@@ -597,7 +616,7 @@ bl_status bitlinear_glu_forward(const float* x, int64_t M, int64_t D, int64_t F,
     if (M <= AUTO_CUDA_MAX_M && gemv_fused_quant_ok(M, D)) {
         cudaError_t e = pick_path((int)M, probs, 2, dev) == PATH_TC
                             ? launch_decode_tc(probs, 2, (int)M, BL_I8, Y_F32, dev, st)
-                            : launch_gemv_fused_group(probs, 2, (int)M, BL_I8, Y_F32, dev, st);
+                            : launch_decode_cuda(probs, 2, (int)M, BL_I8, Y_F32, dev, st);
         if (e != cudaSuccess) return BL_ERR_CUDA;
     } else {
         s = run_forward(xq, gx, M, D, W_gate, beta_gate, F, gate, Y_F32, p, fws_bytes, stream);
@@ -760,7 +779,7 @@ bl_status bitlinear_forward_grouped_fp(const void* x, int x_dtype, int64_t M, in
                         t + g * stride, (int)Kg, (int)N};
         const cudaError_t e = pick_path(1, probs, (int)G, dev) == PATH_TC
                                   ? launch_decode_tc(probs, (int)G, 1, x_dtype, Y_F32, dev, as_stream(stream))
-                                  : launch_gemv_fused_group(probs, (int)G, 1, x_dtype, Y_F32, dev, as_stream(stream));
+                                  : launch_decode_cuda(probs, (int)G, 1, x_dtype, Y_F32, dev, as_stream(stream));
         if (e != cudaSuccess) return BL_ERR_CUDA;
         return from_cuda(launch_grouped_sum(t, stride, N, (int)G, y, y_dtype == BL_F32 ? Y_F32 : Y_BF16, dev.num_sms,
                                             as_stream(stream)));
@@ -790,13 +809,19 @@ bl_status bitlinear_device_status(void* stream) {
 }
 
 bl_status bitlinear_set_decode_engine(int engine) {
-    if (engine != BL_ENGINE_AUTO && engine != BL_ENGINE_CUDA_CORES && engine != BL_ENGINE_TENSOR_CORES)
+    if (engine != BL_ENGINE_AUTO && engine != BL_ENGINE_CUDA_CORES && engine != BL_ENGINE_TENSOR_CORES &&
+        engine != BL_ENGINE_CUDA_CORES_GENERAL)
         return BL_ERR_SHAPE;
     g_engine.store(engine, std::memory_order_relaxed);
     return BL_OK;
 }
 
 int bitlinear_get_decode_engine(void) { return g_engine.load(std::memory_order_relaxed); }
+
+bl_status bitlinear_test_expire_next_wait(int enable) {
+    g_expire_next_wait.store(enable ? 1 : 0, std::memory_order_relaxed);
+    return BL_OK;
+}
 
 int bitlinear_num_sms(void) {
     DevInfo dev;

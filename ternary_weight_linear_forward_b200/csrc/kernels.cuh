@@ -64,6 +64,16 @@ int gemv_group_max();
 cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
                                     const DevInfo& dev, cudaStream_t st);
 
+// k_gemv1.cu  (one token, up to eight problems, CUDA cores, weight stream
+// prefetched under the preceding kernel); x_dtype as above
+bool gemv1_ok(const GemvProblem* probs, int count, int M, const DevInfo& dev);
+cudaError_t launch_gemv1(const GemvProblem* probs, int count, int x_dtype, YMode mode, const DevInfo& dev,
+                         cudaStream_t st);
+
+// api.cu: true once after bitlinear_test_expire_next_wait(1) (test hook of
+// the bounded waits; consumed by the next one-token decode launch)
+bool take_wait_expiry_request();
+
 // k_decode_tc.cu  (M <= 16, tcgen05 int8 tensor cores)
 int decode_tc_max_m();
 bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev);
@@ -73,6 +83,10 @@ cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_d
 // process-wide engine choice
 enum DecodePath : int { PATH_CUDA = 0, PATH_TC = 1, PATH_GEMM = 2 };
 DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo& dev);
+// api.cu: the CUDA-core kernel for a problem set (the one-token streaming
+// kernel where it applies and the engine allows it, else the small-M kernels)
+cudaError_t launch_decode_cuda(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
+                               const DevInfo& dev, cudaStream_t st);
 
 // k_gemm.cu  (M > 64, tcgen05 int8 tensor cores); wbits 2 (trits) or 1 (signs)
 size_t gemm_ws_bytes(long long M, long long N, long long K);

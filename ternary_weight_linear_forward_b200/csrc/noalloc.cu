@@ -101,7 +101,7 @@ extern "C" bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* g
     if (path == PATH_TC)
         e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, d->info, st);
     else if (path == PATH_CUDA)
-        e = launch_gemv(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->info, st);
+        e = launch_decode_cuda(&prob, 1, (int)M, BL_I8, mode, d->info, st);
     else
         e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->scratch, d->info, st);
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;

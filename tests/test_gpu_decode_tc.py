@@ -205,7 +205,8 @@ def test_tc_engine_is_the_one_that_runs(dev):
     # the tensor-core kernel is what runs for a supported shape (kernel names from the profiler)
     xt, W_p, beta, _ = prep(dev, 1, 4096, 2048, seed=3)
     from kernel_trace import kernel_names
-    for engine, name in (("tensor_cores", "decode_tc_kernel"), ("cuda_cores", "gemv_small_kernel")):
+    for engine, name in (("tensor_cores", "decode_tc_kernel"), ("cuda_cores", "gemv1_kernel"),
+                         ("cuda_cores_general", "gemv_small_kernel")):
         with bl.decode_engine(engine):
             names = kernel_names(lambda: bl.forward_fp(xt, W_p, beta))
         if not names:

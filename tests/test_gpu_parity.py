@@ -86,13 +86,59 @@ def test_quantize_special_matrices(dev):
     assert beta.item() == 1.0
     np.testing.assert_array_equal(W_t.cpu().numpy(), oracle.ternarize(W, 1.0, 0.0))
     np.testing.assert_array_equal(W_t.cpu().numpy()[0, :4], [0, 0, 1, -1])
-    # wide dynamic range (no element below 2^-38 of the max, so the sum is exact)
+    # wide dynamic range
     g = np.random.default_rng(5)
     W = (g.standard_normal((64, 256)) * np.exp(g.uniform(-20, 20, (64, 256)))).astype(np.float32)
     W_t, beta, _ = gpu_prep(W, dev)
     oW_t, obeta = oracle.quantize_weights(W)
     assert beta.item() == float(obeta)
     np.testing.assert_array_equal(W_t.cpu().numpy(), oW_t)
+
+
+def _wide_range_matrices():
+    """Matrices whose |W| spans the whole binary32 range: the mean must be
+    the exact one whatever the ratio of an element to the largest."""
+    g = np.random.default_rng(55)
+    base = g.standard_normal((96, 512)).astype(np.float32)
+    out = {}
+    W = base * np.float32(0.02)
+    W[0, :200] = g.standard_normal(200) * 2.0 ** -45 * 0.02      # 2^-45 .. 2^-60 of the max
+    W[1, :200] = g.standard_normal(200) * 2.0 ** -60 * 0.02
+    W[2, :64] = g.standard_normal(64) * 1e-42                      # subnormals
+    W[3, :8] = [1e-45, -1e-45, 2e-45, 3e-44, -7e-40, 1.1754942e-38, -1.1754944e-38, 5.877472e-39]
+    out["gaussian_with_tiny_tail"] = W.astype(np.float32)
+    out["every_exponent"] = (base * np.exp2(g.integers(-149, 120, base.shape))).astype(np.float32)
+    out["subnormal_only"] = (base * 1e-41).astype(np.float32)
+    W = np.zeros((64, 128), np.float32)
+    W[5, 7] = 3.0e38                                               # one huge element, the rest tiny
+    W[6, :] = g.standard_normal(128) * 1e-40
+    out["one_huge"] = W
+    # many small elements whose total reaches the big ones' scale: a sum
+    # that truncation below 2^-38 of the max would change
+    W = np.full((128, 1024), np.float32(2.0 ** -40) * np.float32(1.0000001), np.float32)
+    W[0, 0] = 1.0
+    out["small_mass"] = W
+    # a mean one tiny step above a binary32 tie: 2^16, 2^-9 and 16384 copies
+    # of 2^-23 (1 + 2^-23) among 65536 elements sum to 2^16 + 2^-8 + 2^-32, so
+    # the mean is 1 + 2^-24 + 2^-48 and rounds up to 1 + 2^-23; dropping the
+    # copies' lowest bit (anything coarser than exact) leaves the tie 1 + 2^-24,
+    # which rounds to even, 1
+    W = np.zeros((64, 1024), np.float32)
+    W.flat[0] = 2.0 ** 16
+    W.flat[1] = 2.0 ** -9
+    W.flat[2:2 + 16384] = np.float32(2.0 ** -23) * np.float32(1.0000001)
+    out["above_a_tie"] = W
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(_wide_range_matrices()))
+def test_quantize_exact_over_the_whole_binary32_range(dev, name):
+    W = _wide_range_matrices()[name]
+    W_t, beta, W_p = gpu_prep(W, dev)
+    oW_t, obeta = oracle.quantize_weights(W)
+    assert beta.item() == float(obeta), (beta.item(), float(obeta))
+    np.testing.assert_array_equal(W_t.cpu().numpy(), oW_t)
+    np.testing.assert_array_equal(W_p.cpu().numpy().view(np.uint32), oracle.pack(oW_t))
 
 
 def test_pack_of_arbitrary_trits(dev):
@@ -163,7 +209,7 @@ def run_case(dev, M, K, N, seed, x_dtype="f32", y_dtype="f32", outliers=False):
     return ref
 
 
-@pytest.mark.parametrize("engine", ["cuda_cores", "tensor_cores"])
+@pytest.mark.parametrize("engine", ["cuda_cores", "tensor_cores", "cuda_cores_general"])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 16, 33, 64])
 @pytest.mark.parametrize("K,N", [(64, 5), (1024, 148), (1024, 149), (2560, 1000), (6912, 300)])
 def test_gemv_parity_sweep(dev, M, K, N, engine):
