@@ -218,6 +218,28 @@ def ternary_acc(x_q: np.ndarray, W_t: np.ndarray) -> np.ndarray:
     return acc
 
 
+_lib_omp = None
+
+
+def ternary_acc_all_cores(x_q: np.ndarray, W_t: np.ndarray) -> np.ndarray:
+    """:func:`ternary_acc` computed by the -fopenmp build of the same C source,
+    whose only difference is that the (m, n) pairs are shared among the
+    host's cores: the same integers, in time for full-size checks."""
+    global _lib_omp
+    if _lib_omp is None:
+        L = ctypes.CDLL(_build.build_omp())
+        L.orc_ternary_acc.argtypes = [_i8p, _i64, _i64, _i8p, _i64, _i32p]
+        _lib_omp = L
+    x_q = _c(x_q, np.int8)
+    W_t = _c(W_t, np.int8)
+    M, K = x_q.shape
+    N = W_t.shape[0]
+    assert W_t.shape[1] == K
+    acc = np.empty((M, N), np.int32)
+    _lib_omp.orc_ternary_acc(x_q, M, K, W_t, N, acc)
+    return acc
+
+
 def rescale_f32(acc, beta, gamma) -> np.ndarray:
     """unite.ai eq. 3 "BitLinear-Betrieb": y = acc * (beta * gamma / 127),
     binary32 with f = (beta * gamma) / 127 formed first."""

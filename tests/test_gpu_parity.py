@@ -379,6 +379,36 @@ def _sampled_rows_check(dev, shape, n_rows=48):
     assert_bf16_ok(y[rows], ref["y64"])
 
 
+@pytest.mark.parametrize("M,K,N", [(1024, 512, 11008), (700, 1024, 18000)])
+def test_gemm_multi_wave_full_output(dev, M, K, N):
+    # more 128 x 256 tiles than SMs (344 and 216): every CTA walks several
+    # tiles, alternating its two TMEM accumulators; every output is compared
+    run_case(dev, M, K, N, seed=M + K + N, y_dtype="bf16", outliers=True)
+    run_case(dev, M, K, N, seed=M + K + N + 1)
+
+
+@pytest.mark.parametrize("shape", workloads.W4.shapes, ids=lambda s: s.name)
+def test_workload_prefill_full_output(dev, shape):
+    # full-size prefill (M = 2048) in the launch configuration the benchmark
+    # times, every output against the oracle (its all-core build of the
+    # integer contraction)
+    W = shape.weights()
+    x = shape.inputs()
+    W_t, beta, W_p = gpu_prep(W, dev)
+    x_q, gamma = bl.quant_act(T(x, dev))
+    acc = bl.forward_acc(x_q, W_p).cpu().numpy()
+    y = bl.forward(x_q, gamma, W_p, beta, out_dtype=torch.bfloat16).cpu().view(torch.int16).numpy().view(np.uint16)
+    oW_t, obeta = oracle.quantize_weights(W)
+    assert beta.item() == float(obeta)
+    ox_q, ogamma = oracle.quant_act(x)
+    np.testing.assert_array_equal(x_q.cpu().numpy(), ox_q)
+    np.testing.assert_array_equal(gamma.cpu().numpy(), ogamma)
+    oacc = oracle.ternary_acc_all_cores(ox_q, oW_t)
+    np.testing.assert_array_equal(acc, oacc)
+    assert_bf16_ok(y, oracle.rescale_f64(oacc, obeta, ogamma))
+    np.testing.assert_array_equal(y, oracle.to_bf16(oracle.rescale_f32(oacc, obeta, ogamma)))
+
+
 @pytest.mark.parametrize("shape", workloads.W4.shapes, ids=lambda s: s.name)
 def test_workload_prefill_sampled_rows(dev, shape):
     # full-size prefill (M = 2048) in the launch configuration the benchmark

@@ -266,6 +266,17 @@ def test_acc_matches_int64_matmul_and_bounds():
     assert acc[0, 0] == 127 * K
 
 
+def test_all_core_build_gives_the_same_accumulators():
+    # the -fopenmp build of the same source (used for full-size checks) must
+    # give the plain build's integers, which the int64 matmul pins
+    g = np.random.default_rng(13)
+    x_q = g.integers(-127, 128, size=(33, 2048)).astype(np.int8)
+    W_t = g.integers(-1, 2, size=(301, 2048)).astype(np.int8)
+    acc = oracle.ternary_acc_all_cores(x_q, W_t)
+    np.testing.assert_array_equal(acc, oracle.ternary_acc(x_q, W_t))
+    np.testing.assert_array_equal(acc, x_q.astype(np.int64) @ W_t.T.astype(np.int64))
+
+
 # --------------------------------------------------------------------------
 # Rescale and bf16
 # --------------------------------------------------------------------------
