@@ -521,16 +521,17 @@ int bitlinear_num_sms(void);
 
 /*
  * Test hook of the bounded waits (no counterpart on the pages).  With
- * enable != 0, the next one-token decode launch of this process (the
- * streaming CUDA-core GEMV that bitlinear_forward, _fp, _fp_batch, _acc and
- * _noalloc run for M = 1) limits each of its waits to about 10^5 SM cycles,
- * and the weight producer of its first CTA issues no copies, so that CTA's
- * consumers give up waiting for data that never comes: the kernel raises the
- * device error word and returns (no copy is in flight, nothing hangs), that
- * CTA's outputs are unspecified, and the next bitlinear_device_status returns
- * BL_ERR_TIMEOUT.  The request applies to one launch and then clears itself;
- * enable == 0 withdraws it.  A launch recorded into a CUDA graph keeps it.
- * Always returns BL_OK.
+ * enable != 0, the next launch of the general small-M CUDA-core decode
+ * kernel by bitlinear_forward_fp_batch (for instance with the engine
+ * BL_ENGINE_CUDA_CORES_GENERAL and M <= 4) limits each wait of its first
+ * problem to about 10^5 SM cycles, and the weight producer of that problem's
+ * first CTA issues no copies, so that CTA's consumers give up waiting for
+ * data that never comes: the kernel raises the device error word and
+ * returns (no copy is in flight, nothing hangs), that CTA's outputs are
+ * unspecified, and the next bitlinear_device_status returns BL_ERR_TIMEOUT.
+ * The request applies to one launch and then clears itself; enable == 0
+ * withdraws it.  A launch recorded into a CUDA graph keeps it.  Always
+ * returns BL_OK.
  */
 bl_status bitlinear_test_expire_next_wait(int enable);
 

@@ -26,6 +26,12 @@
 //               per warp), rowsum correction, rescale, bf16/fp32 store.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap
 // the main loop of tile t + 1.  Every mbarrier wait is bounded.
+//
+// Few tiles (a few tokens: M <= 128 gives N / 256 tiles for 148 SMs) are cut
+// along K: a work unit is (tile, K range) and writes its int32 tile to a
+// workspace; a separate, fully parallel kernel then adds the partial tiles
+// of every output (exact, so the order does not matter), subtracts the row
+// sum and rescales.
 #include <cuda.h>
 
 #include <mutex>
@@ -63,7 +69,7 @@ constexpr uint32_t IDESC = idesc_i8(BM, BN, true, true);  // s8 x s8 -> s32, 128
 
 struct GemmHdr {
     uint64_t full[STAGES];      // TMA bytes landed
-    uint64_t unpacked[STAGES];  // codes written by the 128 unpack threads
+    uint64_t unpacked[STAGES];  // codes written by the unpack threads
     uint64_t empty[STAGES];     // MMAs reading the stage finished
     uint64_t tfull[2];          // accumulator complete
     uint64_t tempty[2];         // accumulator drained by the 128 epilogue threads
@@ -79,7 +85,19 @@ struct GemmParams {
     void* y;
     int M, N, K, mode;
     int tiles_m, tiles_n, num_kb;
+    int splits;     // K ranges per tile (1: no split)
+    int part_rows;  // rows of a partial tile in the workspace (min(M, BM))
+    int* part;      // split K: [tiles * splits][part_rows][BN] int32 partial tiles
 };
+
+// Work unit u: tile u / splits, K blocks [kb0, kb1) of its split u % splits.
+__device__ __forceinline__ void unit_range(const GemmParams& p, int u, int& t, int& kb0, int& kb1) {
+    t = u / p.splits;
+    const int sp = u % p.splits;
+    kb0 = (int)((long long)p.num_kb * sp / p.splits);
+    kb1 = (int)((long long)p.num_kb * (sp + 1) / p.splits);
+}
+
 
 __device__ __forceinline__ bool aborted(GemmHdr& h) { return *(volatile int*)&h.abort_flag != 0; }
 
@@ -110,6 +128,46 @@ __global__ void __launch_bounds__(256) rowsum_kernel(const int8_t* __restrict__ 
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) rowsum[row] = s;
+}
+
+// Split K: y[m, n] = (sum over the splits of the partial tiles) - rowsum_m,
+// rescaled; four consecutive n per thread (one 16-byte load per split).
+__global__ void __launch_bounds__(256) splitk_finish_kernel(const int* __restrict__ part, int splits, int part_rows,
+                                                            int tiles_m, const int* __restrict__ rowsum,
+                                                            const float* __restrict__ gamma,
+                                                            const float* __restrict__ beta, void* __restrict__ y,
+                                                            int M, int N, int mode) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const float b = mode == Y_ACC ? 0.0f : __ldg(beta);
+    const int nq = (N + 3) / 4;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)M * nq;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(e / nq), n = (int)(e % nq) * 4;
+        const int mb = m / BM, r = m % BM, nb = n / BN, c = n % BN;
+        const int t = mb + nb * tiles_m;
+        const int4* src = reinterpret_cast<const int4*>(part + ((size_t)t * splits * part_rows + r) * BN + c);
+        int4 acc = make_int4(0, 0, 0, 0);
+        for (int sp = 0; sp < splits; ++sp) {
+            const int4 v = __ldcg(src + (size_t)sp * part_rows * BN / 4);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        const int rs = __ldcg(rowsum + m);
+        const int a[4] = {acc.x - rs, acc.y - rs, acc.z - rs, acc.w - rs};
+        const float f = mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(b, __ldg(gamma + m)), 127.0f);
+        for (int j = 0; j < 4 && n + j < N; ++j) {
+            const long long o = (long long)m * N + n + j;
+            if (mode == Y_ACC)
+                reinterpret_cast<int*>(y)[o] = a[j];
+            else if (mode == Y_F32)
+                reinterpret_cast<float*>(y)[o] = __fmul_rn((float)a[j], f);
+            else
+                reinterpret_cast<uint16_t*>(y)[o] = f32_to_bf16_rn(__fmul_rn((float)a[j], f));
+        }
+    }
 }
 
 __device__ __forceinline__ void store_chunk(const GemmParams& p, int m, int n0, const int (&v)[32], int rs, float f,
@@ -164,7 +222,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     GemmHdr& h = *reinterpret_cast<GemmHdr*>(base);
     unsigned char* stages = base + HDR_BYTES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int num_units = p.tiles_m * p.tiles_n * p.splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -193,9 +251,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int it = 0;
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                int t, kb0, kb1;
+                unit_range(p, u, t, kb0, kb1);
                 const int mb = t % p.tiles_m, nb = t / p.tiles_m;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!wait_or_abort(h, &h.empty[s], ph ^ 1)) goto done;
@@ -210,13 +270,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             int it = 0, acc_it = 0;
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++acc_it) {
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++acc_it) {
+                int t, kb0, kb1;
+                unit_range(p, u, t, kb0, kb1);
                 const int b = acc_it & 1;
                 const uint32_t aph = (acc_it >> 1) & 1;
                 if (!wait_or_abort(h, &h.tempty[b], aph ^ 1)) goto done;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!wait_or_abort(h, &h.full[s], ph)) goto done;
@@ -227,7 +289,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint64_t bdesc = sw128_desc(smem_u32(st + A_BYTES));
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k)  // K = 32 bytes per MMA: advance 32 B = 2 in addr >> 4
-                        mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0);
+                        mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb != kb0) || (k != 0));
                     mma_commit(&h.empty[s]);
                 }
                 mma_commit(&h.tfull[b]);
@@ -250,8 +312,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             dst_off[i] = (uint32_t)(n * BK + ((c ^ (n & 7)) << 4));
         }
         int it = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            int t, kb0, kb1;
+            unit_range(p, u, t, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
                 if (!wait_or_abort(h, &h.full[s], ph)) goto done;
@@ -300,14 +364,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const bool vec_ok = p.mode == Y_BF16 ? (p.N % 8 == 0) : (p.N % 4 == 0);
         const float beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         int acc_it = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++acc_it) {
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++acc_it) {
+            int t, kb0, kb1;
+            unit_range(p, u, t, kb0, kb1);
             const int mb = t % p.tiles_m, nb = t / p.tiles_m;
             const int b = acc_it & 1;
             const uint32_t aph = (acc_it >> 1) & 1;
             // tcgen05.ld is warp-collective: the whole warp proceeds or leaves together
             if (!__all_sync(0xffffffffu, wait_or_abort(h, &h.tfull[b], aph))) goto done;
             tc_fence_after();
-            const int m = mb * BM + q * 32 + lane;
+            const int r = q * 32 + lane;  // row of the tile
+            const int m = mb * BM + r;
             int rs = 0;
             float f = 0.0f;
             if (m < p.M) {
@@ -315,12 +382,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (p.mode != Y_ACC) f = __fdiv_rn(__fmul_rn(beta, __ldg(p.gamma + m)), 127.0f);
             }
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+            if (p.splits == 1) {
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    int v[32];
+                    tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                    const int n0 = nb * BN + c * 32;
+                    if (m < p.M && n0 < p.N) store_chunk(p, m, n0, v, rs, f, vec_ok);
+                }
+                tc_fence_before();
+                mbar_arrive(&h.tempty[b]);
+                continue;
+            }
+            // split K: this unit's partial tile to the workspace
+            int* mine = p.part + ((size_t)u * p.part_rows + r) * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 int v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
-                const int n0 = nb * BN + c * 32;
-                if (m < p.M && n0 < p.N) store_chunk(p, m, n0, v, rs, f, vec_ok);
+                if (r < p.part_rows && m < p.M) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        __stcg(reinterpret_cast<int4*>(mine + c * 32 + j), make_int4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+                }
             }
             tc_fence_before();
             mbar_arrive(&h.tempty[b]);
@@ -352,14 +436,36 @@ EncodeTiled tensor_map_encoder() {
     return fn;
 }
 
+// K ranges per tile: as many as keep the units within one wave of the B200's
+// 148 SMs (a fixed count, so the workspace size does not depend on the device).
+constexpr int SPLIT_UNITS_TARGET = 148;
+
+struct GemmPlan {
+    int tiles_m, tiles_n, num_kb, splits, part_rows;
+    size_t rowsum_bytes, part_bytes;
+};
+
+GemmPlan gemm_plan(long long M, long long N, long long K, bool allow_split) {
+    GemmPlan g;
+    g.tiles_m = (int)((M + BM - 1) / BM);
+    g.tiles_n = (int)((N + BN - 1) / BN);
+    g.num_kb = (int)((K + BK - 1) / BK);
+    const long long tiles = (long long)g.tiles_m * g.tiles_n;
+    g.splits = allow_split ? (int)std::max<long long>(1, std::min<long long>(SPLIT_UNITS_TARGET / tiles, g.num_kb)) : 1;
+    g.part_rows = (int)std::min<long long>(M, BM);
+    g.rowsum_bytes = (size_t)((M * 4 + 255) / 256 * 256);
+    g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.part_rows * BN * 4 : 0;
+    return g;
+}
+
 size_t gemm_ws_bytes(long long M, long long N, long long K) {
-    (void)N;
-    (void)K;
-    return (size_t)((M * 4 + 255) / 256 * 256);
+    const GemmPlan g = gemm_plan(M, N, K, true);
+    return g.rowsum_bytes + g.part_bytes;
 }
 
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
-                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits) {
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits,
+                        bool allow_split) {
     if (wbits != 1 && wbits != 2) return cudaErrorInvalidValue;
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
@@ -386,7 +492,9 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    const GemmPlan plan = gemm_plan(M, N, K, allow_split);
     int* rowsum = reinterpret_cast<int*>(ws);
+    int* part = plan.splits > 1 ? reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + plan.rowsum_bytes) : nullptr;
     cudaError_t e = launch_pdl(rowsum_kernel, dim3((M + 7) / 8), dim3(256), 0, st, x_q, M, K, rowsum);
     if (e != cudaSuccess) return e;
 
@@ -399,15 +507,23 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     p.N = N;
     p.K = K;
     p.mode = mode;
-    p.tiles_m = (M + BM - 1) / BM;
-    p.tiles_n = (N + BN - 1) / BN;
-    p.num_kb = (K + BK - 1) / BK;
-    const int tiles = p.tiles_m * p.tiles_n;
-    const int grid = std::max(1, std::min(tiles, dev.num_sms));
+    p.tiles_m = plan.tiles_m;
+    p.tiles_n = plan.tiles_n;
+    p.num_kb = plan.num_kb;
+    p.splits = plan.splits;
+    p.part_rows = plan.part_rows;
+    p.part = part;
+    const int units = p.tiles_m * p.tiles_n * p.splits;
+    const int grid = std::max(1, std::min(units, dev.num_sms));
     auto kernel = wbits == 2 ? gemm_kernel<2> : gemm_kernel<1>;
     e = ensure_smem_optin(reinterpret_cast<const void*>(kernel), GEMM_SMEM);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
+    e = launch_pdl(kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
+    if (e != cudaSuccess || plan.splits == 1) return e;
+    const long long quads = (long long)M * ((N + 3) / 4);
+    const int fgrid = (int)std::max<long long>(1, std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8));
+    return launch_pdl(splitk_finish_kernel, dim3(fgrid), dim3(256), 0, st, (const int*)part, plan.splits,
+                      plan.part_rows, plan.tiles_m, (const int*)rowsum, gamma, beta, y, M, N, (int)mode);
 }
 
 }  // namespace bl

@@ -68,6 +68,8 @@ struct GemvParams {
     int ks;            // K slices per row (small kernel): 1, 2 or 4
     int slice4;        // 16-byte weight groups per slice
     int wave;          // mt kernel: rows in flight per wave
+    long long wait_limit;  // small kernel: SM cycles before a wait gives up
+    int stall_cta;         // small kernel test hook: this CTA's producer issues nothing (-1: none)
 };
 
 struct Shared {
@@ -155,11 +157,25 @@ __device__ __forceinline__ void produce(const GemvParams& p, Shared& sh, unsigne
     }
 }
 
+// Wait (at most `limit` SM cycles) for the phase of the given parity; false,
+// with the device error word raised, if it did not complete in time.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) {
+            set_dev_error(DEV_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
 // Wait for the chunk holding slab row i; false once the CTA has aborted.
 __device__ __forceinline__ bool wait_row(const GemvParams& p, Shared& sh, int i) {
     const int c = i >> p.rpc_shift;
     if (*(volatile int*)&sh.abort_flag) return false;
-    if (!mbar_wait(&sh.full[chunk_slot(p, c)], chunk_parity(p, c))) {
+    if (!mbar_wait_limit(&sh.full[chunk_slot(p, c)], chunk_parity(p, c), p.wait_limit)) {
         sh.abort_flag = 1;
         return false;
     }
@@ -340,12 +356,13 @@ __device__ __forceinline__ void gemv_small_body(const GemvParams& p, int cta, in
         // read before waiting for it
         sh.beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         fence_mbar_init();
-        produce(p, sh, ring, r0, nrows, 0, min(nchunks, GEMV_EARLY_CHUNKS));
+        if (cta != p.stall_cta) produce(p, sh, ring, r0, nrows, 0, min(nchunks, GEMV_EARLY_CHUNKS));
     }
     __syncthreads();
     pdl_launch_dependents();
     if (warp == 0) {
-        if (lane == 0 && nchunks > GEMV_EARLY_CHUNKS) produce(p, sh, ring, r0, nrows, GEMV_EARLY_CHUNKS, nchunks);
+        if (lane == 0 && nchunks > GEMV_EARLY_CHUNKS && cta != p.stall_cta)
+            produce(p, sh, ring, r0, nrows, GEMV_EARLY_CHUNKS, nchunks);
         return;
     }
     pdl_wait();
@@ -734,6 +751,8 @@ GroupKernel group_kernel_for(int mt) {
 GemvParams make_params(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
                        int N, void* y, YMode mode) {
     GemvParams p = {};
+    p.wait_limit = WAIT_LIMIT_CYCLES;
+    p.stall_cta = -1;
     p.x_q = x_q;
     p.gamma = gamma;
     p.W_p = W_p;
@@ -793,6 +812,10 @@ cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, 
         smem = std::max(smem, sh.smem);
     }
     g.cta0[count] = cta;
+    if (take_wait_expiry_request()) {  // test hook: the first CTA never receives its weights
+        g.prob[0].wait_limit = 100000;
+        g.prob[0].stall_cta = 0;
+    }
     const int mt = small_mt(M);
     GroupKernel k = xm == X_QUANTISED ? group_kernel_for<X_QUANTISED>(mt)
                     : xm == X_BF16    ? group_kernel_for<X_BF16>(mt)

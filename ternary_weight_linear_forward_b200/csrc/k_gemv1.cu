@@ -7,29 +7,32 @@
 // (per-token absmax int8 quantiser) and eq. 3 "BitLinear-Betrieb" (rescale by
 // beta * gamma / Q_b).
 //
-// A single token's projection moves its packed weights once and does almost
-// nothing else, so a decode step is a stream of HBM bytes with a short,
+// A single token's projection moves its packed weights once and does little
+// else, so a decode step is a stream of HBM bytes behind a short,
 // latency-bound prologue (the activation quantiser) that can only start once
 // the preceding kernel has finished.  The design hides everything but that
-// prologue behind the weight stream of the NEXT launch:
+// prologue behind the weight stream:
 //
 //   * one CTA per SM owns a contiguous slab of rows of every problem;
-//   * a CTA takes at most half of an SM (512 threads, 64 registers, about
+//   * a CTA takes at most half of an SM (512 threads, 64 registers, under
 //     113 KB of shared memory), so the following launch's CTA is resident
 //     beside it as soon as this one has started (programmatic dependent
-//     launch) and fills its own weight rings while this one computes;
-//   * each problem has its own ring of chunk slots (a power-of-two number of
-//     rows, about 8 KB), fed by 1-D bulk copies from one producer thread that
-//     never waits for the preceding kernel (weights and beta are inputs that
-//     no in-flight kernel writes);
-//   * a consumer warp is bound to one K slice (<= 64 groups of 16 packed
-//     bytes = 4096 trits) of one problem and keeps that slice of x_hat in
-//     registers (two 64-byte groups per lane), so the row loop reads only the
-//     weights from shared memory: one 16-byte load, four LOP3 and four
-//     dp4a.u32.s32 per 64 trits and lane per group;
-//   * R rows at a time are finished by one batched shuffle reduction; rows
-//     cut into several K slices add their slice sums in shared memory
-//     (integer, so the order does not matter) and are written at the end.
+//     launch) and puts its first weight rows in flight while this one
+//     computes;
+//   * every warp is bound to one K slice (<= 64 groups of 16 packed bytes =
+//     4096 trits) of one problem and keeps that slice of x_hat in registers
+//     (one or two 64-byte groups per lane);
+//   * every lane streams its own 16-byte groups of the warp's rows with
+//     cp.async into a per-warp ring of DEPTH row slots in shared memory, one
+//     commit group per row, and reads back only what it copied itself: no
+//     barrier and no hand-off between warps, and DEPTH rows of every warp (up
+//     to 80 KB per CTA) in flight from the moment the CTA starts.  Copies
+//     issued by all 512 threads keep far more requests in flight per SM than
+//     one thread's bulk copies, which streamed about 1.3 TB/s here;
+//   * per row and lane: one or two 16-byte loads, four LOP3 and four
+//     dp4a.u32.s32 per 16 trits; R rows at a time are finished by one batched
+//     shuffle reduction; rows cut into several K slices add their slice sums
+//     in shared memory (integer, so the order does not matter).
 //
 // The quantiser is the one of the other decode kernels: absmax per token
 // over the row (exact, order-free), s = 127 / gamma, codes rint(x s) clamped
@@ -44,14 +47,14 @@ namespace bl {
 namespace {
 
 constexpr int G1_MAX_PROBS = 8;
-constexpr int G1_CWARPS = 15;                     // consumer warps (warp 0 produces)
-constexpr int G1_THREADS = (G1_CWARPS + 1) * 32;  // 512: two CTAs fit an SM by registers
-constexpr int G1_MAX_BARS = 64;                   // ring slots over all problems
-constexpr int G1_PART_MAX = 512;                  // slice sums of K-sliced rows per CTA
-constexpr int G1_SLICE_UNITS = 64;                // 16-byte packed groups per K slice (2 per lane)
-constexpr int G1_CHUNK_TARGET = 8192;             // bytes per ring slot (about)
-constexpr int G1_XC = 2;                          // activation chunks cached per staging thread
-constexpr int G1_MAX_SUMK = G1_XC * G1_CWARPS * 32 * 16;  // every chunk cached: sum of K <= 15360
+constexpr int G1_WARPS = 16;
+constexpr int G1_THREADS = G1_WARPS * 32;  // 512: two CTAs fit an SM by registers
+constexpr int G1_DEPTH = 5;                // rows in flight per warp
+constexpr int G1_SLOT = 1024;              // bytes of a ring slot: one row's slice of <= 64 groups
+constexpr int G1_PART_MAX = 512;           // slice sums of K-sliced rows per CTA
+constexpr int G1_SLICE_UNITS = 64;         // 16-byte packed groups per K slice (2 per lane)
+constexpr int G1_XC = 2;                   // activation chunks cached per staging thread
+constexpr int G1_MAX_SUMK = G1_XC * G1_THREADS * 16;  // every chunk cached: sum of K <= 16384
 
 struct G1Prob {
     const void* x;       // fp32 / bf16 activations, or int8 x_q (with gamma)
@@ -60,39 +63,30 @@ struct G1Prob {
     const float* beta;
     void* y;
     int K, N;
-    int rb;         // bytes per packed row (K / 4)
-    int rpc_shift;  // log2(rows per ring slot)
-    int slot;       // bytes per ring slot
-    int stages;     // ring slots
-    int ring_off;   // shared-memory offset of the ring
-    int bar0;       // first barrier of the ring
-    int xq_off;     // shared-memory offset of x_hat (K bytes)
-    int nslice;     // K slices; rows with more than one add slice sums in part[]
-    int slice_w;    // 16-byte groups per slice (the last slice may be shorter)
-    int part_off;   // first part[] entry of this problem's rows
+    int rb;        // bytes per packed row (K / 4)
+    int xq_off;    // shared-memory offset of x_hat (K bytes)
+    int nslice;    // K slices; rows with more than one add slice sums in part[]
+    int slice_w;   // 16-byte groups per slice (the last slice may be shorter)
+    int part_off;  // first part[] entry of this problem's rows
 };
 
 struct G1Params {
     G1Prob prob[G1_MAX_PROBS];
     int count;
-    int x_mode;  // X_QUANTISED, X_F32 or X_BF16
-    int mode;    // Y_F32, Y_BF16 or Y_ACC
-    int sliced;  // any problem with nslice > 1
-    long long wait_limit;  // SM cycles before a wait gives up
-    int stall_cta;         // test hook: this CTA's producer issues nothing (-1: none)
-    // role of consumer warp w: problem, K slice, index in the (problem, slice)
-    // group, group size, rows per batch (1, 2 or 4)
-    unsigned char wp[G1_CWARPS], ws[G1_CWARPS], wj[G1_CWARPS], wn[G1_CWARPS], wr[G1_CWARPS];
+    int x_mode;    // X_QUANTISED, X_F32 or X_BF16
+    int mode;      // Y_F32, Y_BF16 or Y_ACC
+    int sliced;    // any problem with nslice > 1
+    int ring_off;  // shared-memory offset of the per-warp rings
+    // role of warp w: problem, K slice, index in the (problem, slice) group,
+    // group size, rows per batch (1, 2 or 4)
+    unsigned char wp[G1_WARPS], ws[G1_WARPS], wj[G1_WARPS], wn[G1_WARPS], wr[G1_WARPS];
 };
 
 struct G1Shared {
-    uint64_t full[G1_MAX_BARS];
-    uint64_t empty[G1_MAX_BARS];
-    int abort_flag;
     int rowsum[G1_MAX_PROBS];
     float beta[G1_MAX_PROBS];
     float fscale[G1_MAX_PROBS];
-    unsigned red[G1_CWARPS][G1_MAX_PROBS];
+    unsigned red[G1_WARPS][G1_MAX_PROBS];
     int part[G1_PART_MAX];
 };
 constexpr int G1_HDR = (int)((sizeof(G1Shared) + 127) / 128 * 128);
@@ -103,94 +97,13 @@ __device__ __forceinline__ void g1_rows(const G1Prob& q, int cta, int ncta, int&
     n = (int)((N * (cta + 1)) / ncta) - r0;
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-
-// Issue chunk k of problem q (rows [k << rpc_shift, ...) of this CTA's slab).
-__device__ __forceinline__ void g1_issue(const G1Prob& q, G1Shared& sh, unsigned char* smem, int r0, int n, int k,
-                                         uint64_t pol) {
-    const int st = k % q.stages;
-    const int rows = min(1 << q.rpc_shift, n - (k << q.rpc_shift));
-    const uint32_t bytes = (uint32_t)rows * q.rb;
-    uint64_t* full = &sh.full[q.bar0 + st];
-    mbar_arrive_expect_tx(full, bytes);
-    const unsigned char* src =
-        reinterpret_cast<const unsigned char*>(q.W_p) + ((long long)r0 + ((long long)k << q.rpc_shift)) * q.rb;
-    bulk_g2s(smem + q.ring_off + (size_t)st * q.slot, src, bytes, full, pol);
-}
-
-// Producer thread: every chunk of every problem, problems interleaved, a
-// slot reused once all its (row, slice) consumers have arrived.  Polls the
-// rings so that one problem's full ring never holds up another's.
-__device__ void g1_produce(const G1Params& g, G1Shared& sh, unsigned char* smem, int cta, int ncta, int first_k) {
-    const uint64_t pol = policy_evict_first();
-    int next[G1_MAX_PROBS], nch[G1_MAX_PROBS], r0[G1_MAX_PROBS], nr[G1_MAX_PROBS];
-    int left = 0;
-#pragma unroll
-    for (int i = 0; i < G1_MAX_PROBS; ++i) {
-        next[i] = nch[i] = r0[i] = nr[i] = 0;
-        if (i < g.count) {
-            g1_rows(g.prob[i], cta, ncta, r0[i], nr[i]);
-            nch[i] = (nr[i] + (1 << g.prob[i].rpc_shift) - 1) >> g.prob[i].rpc_shift;
-            next[i] = min(first_k, nch[i]);
-            left += nch[i] - next[i];
-        }
-    }
-    long long t0 = -1;
-    while (left > 0) {
-        bool progress = false;
-#pragma unroll
-        for (int i = 0; i < G1_MAX_PROBS; ++i) {
-            if (i >= g.count) break;
-            const G1Prob& q = g.prob[i];
-            const int k = next[i];
-            if (k >= nch[i]) continue;
-            if (k >= q.stages && !mbar_test(&sh.empty[q.bar0 + k % q.stages], ((k / q.stages) - 1) & 1)) continue;
-            g1_issue(q, sh, smem, r0[i], nr[i], k, pol);
-            next[i] = k + 1;
-            --left;
-            progress = true;
-        }
-        if (progress) {
-            t0 = -1;
-        } else {
-            if (*(volatile int*)&sh.abort_flag) return;
-            const long long t = clock64();
-            if (t0 < 0) t0 = t;
-            if (t - t0 > g.wait_limit) {
-                set_dev_error(DEV_ERR_TIMEOUT);
-                sh.abort_flag = 1;
-                return;
-            }
-        }
-    }
-}
-
-// Wait for the phase of the given parity, at most `limit` SM cycles; false
-// (and the device error word raised) if it did not complete in time.
-__device__ __forceinline__ bool g1_wait(uint64_t* bar, uint32_t parity, long long limit) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > limit) {
-            set_dev_error(DEV_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
-__device__ __forceinline__ void g1_consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(G1_CWARPS * 32) : "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void g1_store(const G1Params& g, const G1Prob& q, int n, int acc, float f) {
@@ -205,19 +118,49 @@ __device__ __forceinline__ void g1_store(const G1Params& g, const G1Prob& q, int
     }
 }
 
-// Consumers: quantise the token of every problem into shared memory (codes
-// in k order, row sums, rescale factors).  Every 16-element chunk of the
-// concatenated activations is loaded once into registers and serves both the
-// absmax pass and the code pass.
+// The rows one warp works on, in order: batches b = j, j + n, ... of R
+// consecutive rows; the t-th row of the sequence, or -1 past the slab's end.
+struct RowSeq {
+    int j, n, R, nrows;
+    __device__ __forceinline__ int row(int t) const {
+        const int i = (j + (t / R) * n) * R + t % R;
+        return i < nrows ? i : -1;
+    }
+};
+
+// This lane's part of a warp's streaming: its one or two 16-byte groups of
+// the warp's K slice in every row.
+struct Lane {
+    const unsigned char* wslice;  // the slice's first byte in row 0 of the CTA's slab
+    unsigned char* ring;          // the warp's ring of DEPTH slots
+    int rb, lane;
+    bool ha, hb;                  // the lane's first / second group exists
+
+    // put row i in flight into ring slot `slot`; one commit group per call,
+    // empty for i < 0
+    __device__ __forceinline__ void fetch(int i, int slot) const {
+        if (i >= 0) {
+            const unsigned char* src = wslice + (size_t)i * rb;
+            unsigned char* dst = ring + slot * G1_SLOT;
+            if (ha) cp_async16(dst + 16 * lane, src + 16 * lane);
+            if (hb) cp_async16(dst + 16 * (lane + 32), src + 16 * (lane + 32));
+        }
+        cp_async_commit();
+    }
+};
+
+// Quantise the token of every problem into shared memory (codes in k order,
+// row sums, rescale factors).  Every 16-element chunk of the concatenated
+// activations is loaded once into registers and serves both the absmax pass
+// and the code pass.  Called by all threads (two CTA barriers).
 template <int XM>
-__device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsigned char* smem, int ctid) {
-    constexpr int CT = G1_CWARPS * 32;
-    const int lane = ctid & 31, warp = ctid >> 5;
+__device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsigned char* smem) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     XChunk<XM> cache[G1_XC];
     int cp[G1_XC], cg[G1_XC];
 #pragma unroll
     for (int i = 0; i < G1_XC; ++i) {
-        int gi = ctid + i * CT;
+        int gi = tid + i * G1_THREADS;
         int p = -1;
         for (int j = 0; j < g.count; ++j) {
             const int gj = g.prob[j].K >> 4;
@@ -243,26 +186,25 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
             a = __reduce_max_sync(0xffffffffu, a);
             if (lane == 0) sh.red[warp][p] = a;
         }
-        g1_consumer_sync();
+        __syncthreads();
 #pragma unroll
         for (int i = 0; i < G1_XC; ++i) {
             if (cp[i] >= 0) {
                 unsigned a = 0u;
-                for (int w = 0; w < G1_CWARPS; ++w) a = max(a, sh.red[w][cp[i]]);
+                for (int w = 0; w < G1_WARPS; ++w) a = max(a, sh.red[w][cp[i]]);
                 s[i] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(a), 1e-5f));
             }
         }
-        if (ctid < g.count) {
+        if (tid < g.count) {
             unsigned a = 0u;
-            for (int w = 0; w < G1_CWARPS; ++w) a = max(a, sh.red[w][ctid]);
+            for (int w = 0; w < G1_WARPS; ++w) a = max(a, sh.red[w][tid]);
             const float gam = fmaxf(__uint_as_float(a), 1e-5f);
-            sh.fscale[ctid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[ctid], gam), 127.0f);
+            sh.fscale[tid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[tid], gam), 127.0f);
         }
-    } else if (ctid < g.count) {
-        sh.fscale[ctid] =
-            g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[ctid], __ldg(g.prob[ctid].gamma)), 127.0f);
+    } else if (tid < g.count) {
+        sh.fscale[tid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[tid], __ldg(g.prob[tid].gamma)), 127.0f);
     }
-    for (int i = ctid; i < G1_PART_MAX; i += CT) sh.part[i] = 0;
+    for (int i = tid; i < G1_PART_MAX; i += G1_THREADS) sh.part[i] = 0;
     int rs[G1_XC];
 #pragma unroll
     for (int i = 0; i < G1_XC; ++i) {
@@ -281,79 +223,67 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
         v = __reduce_add_sync(0xffffffffu, v);
         if (lane == 0 && v != 0) atomicAdd(&sh.rowsum[p], v);
     }
-    g1_consumer_sync();
+    __syncthreads();
 }
 
-// One consumer warp's share: rows b*R .. b*R+R-1 for batches b = j, j + n, ...
-// of problem q, K slice sl.  UPL = 16-byte groups per lane (1 or 2).
+// One warp's share of problem q, K slice starting at group u0: the rows of
+// `seq`, rows 0 .. DEPTH-1 of which are already in flight.  UPL = 16-byte
+// groups per lane (1 or 2).  No barrier inside.
 template <int R, int UPL>
-__device__ __forceinline__ void g1_rows_loop(const G1Params& g, const G1Prob& q, G1Shared& sh, unsigned char* smem,
-                                             int pi, int sl, int j, int n, int r0, int nrows) {
-    const int lane = threadIdx.x & 31;
-    const int U = q.K >> 6;
-    const int u0 = sl * q.slice_w;
-    const int width = min(q.slice_w, U - u0);
-    const bool ha = lane < width;
-    const bool hb = UPL == 2 && lane + 32 < width;
-    // x_hat of this lane's groups: 64 codes each, k = 64u .. 64u + 63
-    int4 xa[4], xb[4];
+__device__ __forceinline__ void g1_loop(const G1Params& g, const G1Prob& q, const G1Shared& sh,
+                                        const unsigned char* smem, int pi, int u0, const RowSeq& seq, int r0,
+                                        const Lane& ln) {
+    const int lane = ln.lane;
+    int4 xa[4], xb[4];  // x_hat of this lane's groups: 64 codes each, k = 64u .. 64u + 63
     const int4* xq = reinterpret_cast<const int4*>(smem + q.xq_off);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        xa[i] = ha ? xq[4 * (u0 + lane) + i] : make_int4(0, 0, 0, 0);
-        xb[i] = hb ? xq[4 * (u0 + lane + 32) + i] : make_int4(0, 0, 0, 0);
+        xa[i] = ln.ha ? xq[4 * (u0 + lane) + i] : make_int4(0, 0, 0, 0);
+        xb[i] = UPL == 2 && ln.hb ? xq[4 * (u0 + lane + 32) + i] : make_int4(0, 0, 0, 0);
     }
-    const int rmask = (1 << q.rpc_shift) - 1;
     const float f = sh.fscale[pi];
     const int rowsum = sh.rowsum[pi];
-    for (int b = j; b * R < nrows; b += n) {
-        const int i0 = b * R;
-        const int nv = min(R, nrows - i0);
-        bool ok = !*(volatile int*)&sh.abort_flag;
+    const int batches = (seq.nrows + R - 1) / R;
+    int t = 0;
+    for (int b = seq.j; b < batches; b += seq.n) {
         int vals[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
+        for (int r = 0; r < R; ++r, ++t) {
+            cp_async_wait<G1_DEPTH - 1>();  // row t's group has landed
+            const int slot = t % G1_DEPTH;
+            const unsigned char* w = ln.ring + slot * G1_SLOT;
             vals[r] = 0;
-            if (r < nv && ok) {
-                const int i = i0 + r;
-                const int k = i >> q.rpc_shift;
-                const int st = k % q.stages;
-                if (!g1_wait(&sh.full[q.bar0 + st], (uint32_t)((k / q.stages) & 1), g.wait_limit)) {
-                    sh.abort_flag = 1;
-                    ok = false;
-                } else {
-                    const uint4* wr = reinterpret_cast<const uint4*>(smem + q.ring_off + (size_t)st * q.slot +
-                                                                     (size_t)(i & rmask) * q.rb) +
-                                      u0;
-                    const uint4 wa = ha ? wr[lane] : make_uint4(0u, 0u, 0u, 0u);
-                    const uint4 wb = hb ? wr[lane + 32] : make_uint4(0u, 0u, 0u, 0u);
-                    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                    word_dot(wa.x, xa[0].x, xa[0].y, xa[0].z, xa[0].w, a0, a1, a2, a3);
-                    word_dot(wa.y, xa[1].x, xa[1].y, xa[1].z, xa[1].w, a0, a1, a2, a3);
-                    word_dot(wa.z, xa[2].x, xa[2].y, xa[2].z, xa[2].w, a0, a1, a2, a3);
-                    word_dot(wa.w, xa[3].x, xa[3].y, xa[3].z, xa[3].w, a0, a1, a2, a3);
-                    if (UPL == 2) {
-                        word_dot(wb.x, xb[0].x, xb[0].y, xb[0].z, xb[0].w, a0, a1, a2, a3);
-                        word_dot(wb.y, xb[1].x, xb[1].y, xb[1].z, xb[1].w, a0, a1, a2, a3);
-                        word_dot(wb.z, xb[2].x, xb[2].y, xb[2].z, xb[2].w, a0, a1, a2, a3);
-                        word_dot(wb.w, xb[3].x, xb[3].y, xb[3].z, xb[3].w, a0, a1, a2, a3);
-                    }
-                    vals[r] = combine4(a0, a1, a2, a3);
+            if (seq.row(t) >= 0) {
+                const uint4 wa = ln.ha ? *reinterpret_cast<const uint4*>(w + 16 * lane) : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 wb = UPL == 2 && ln.hb ? *reinterpret_cast<const uint4*>(w + 16 * (lane + 32))
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+                int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+                word_dot(wa.x, xa[0].x, xa[0].y, xa[0].z, xa[0].w, a0, a1, a2, a3);
+                word_dot(wa.y, xa[1].x, xa[1].y, xa[1].z, xa[1].w, a0, a1, a2, a3);
+                word_dot(wa.z, xa[2].x, xa[2].y, xa[2].z, xa[2].w, a0, a1, a2, a3);
+                word_dot(wa.w, xa[3].x, xa[3].y, xa[3].z, xa[3].w, a0, a1, a2, a3);
+                if (UPL == 2) {
+                    word_dot(wb.x, xb[0].x, xb[0].y, xb[0].z, xb[0].w, a0, a1, a2, a3);
+                    word_dot(wb.y, xb[1].x, xb[1].y, xb[1].z, xb[1].w, a0, a1, a2, a3);
+                    word_dot(wb.z, xb[2].x, xb[2].y, xb[2].z, xb[2].w, a0, a1, a2, a3);
+                    word_dot(wb.w, xb[3].x, xb[3].y, xb[3].z, xb[3].w, a0, a1, a2, a3);
                 }
+                vals[r] = combine4(a0, a1, a2, a3);
             }
+            // the slot's words are in registers and used: refill it with row t + DEPTH
+            ln.fetch(seq.row(t + G1_DEPTH), slot);
         }
-        ok = __all_sync(0xffffffffu, ok);
         int which;
         const int tot = team_reduce<32, R>(vals, lane, which);
-        if (ok && lane == which * (32 / R) && which < nv) {
-            const int i = i0 + which;
+        const int i = b * R + which;
+        if (lane == which * (32 / R) && i < seq.nrows) {
             if (q.nslice == 1)
                 g1_store(g, q, r0 + i, tot - rowsum, f);
             else
-                atomicAdd(&sh.part[q.part_off + i], tot);
-            mbar_arrive(&sh.empty[q.bar0 + (i >> q.rpc_shift) % q.stages]);
+                atomicAdd(const_cast<int*>(&sh.part[q.part_off + i]), tot);
         }
     }
+    cp_async_wait<0>();  // no copy of this lane is in flight past here
 }
 
 template <int XM>
@@ -362,66 +292,54 @@ __global__ void __launch_bounds__(G1_THREADS, 2) gemv1_kernel(const __grid_const
     G1Shared& sh = *reinterpret_cast<G1Shared*>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x, ncta = gridDim.x;
-    if (threadIdx.x == 0) {
-        for (int p = 0; p < g.count; ++p) {
-            const G1Prob& q = g.prob[p];
-            for (int s = 0; s < q.stages; ++s) {
-                mbar_init(&sh.full[q.bar0 + s], 1);
-                mbar_init(&sh.empty[q.bar0 + s], (1u << q.rpc_shift) * q.nslice);
-            }
-            sh.rowsum[p] = 0;
-            // beta and W_p are weight inputs, not written by the preceding
-            // kernel: read before waiting for it
-            sh.beta[p] = g.mode == Y_ACC ? 0.0f : __ldg(q.beta);
-        }
-        sh.abort_flag = 0;
-        fence_mbar_init();
-        // the first chunk of every problem is in flight before the CTA barrier
-        const uint64_t pol = policy_evict_first();
-        for (int p = 0; p < g.count && cta != g.stall_cta; ++p) {
-            int r0, n;
-            g1_rows(g.prob[p], cta, ncta, r0, n);
-            if (n > 0) g1_issue(g.prob[p], sh, smem, r0, n, 0, pol);
-        }
+
+    const int pi = g.wp[warp];
+    const G1Prob& q = g.prob[pi];
+    int r0, n;
+    g1_rows(q, cta, ncta, r0, n);
+    const int u0 = g.ws[warp] * q.slice_w;
+    const int width = min(q.slice_w, (q.K >> 6) - u0);  // 16-byte groups of this slice
+    const RowSeq seq = {g.wj[warp], g.wn[warp], g.wr[warp], n};
+    Lane ln;
+    ln.wslice = reinterpret_cast<const unsigned char*>(q.W_p) + (size_t)r0 * q.rb + 16 * u0;
+    ln.ring = smem + g.ring_off + (size_t)warp * G1_DEPTH * G1_SLOT;
+    ln.rb = q.rb;
+    ln.lane = lane;
+    ln.ha = lane < width;
+    ln.hb = lane + 32 < width;
+    // The weights and beta are inputs that no in-flight kernel writes: the
+    // first DEPTH rows of every warp go in flight before the preceding kernel
+    // is waited for.
+#pragma unroll
+    for (int d = 0; d < G1_DEPTH; ++d) ln.fetch(seq.row(d), d);
+    if (threadIdx.x < G1_MAX_PROBS) {
+        const int p = threadIdx.x;
+        sh.rowsum[p] = 0;
+        sh.beta[p] = p < g.count && g.mode != Y_ACC ? __ldg(g.prob[p].beta) : 0.0f;
     }
     __syncthreads();
     pdl_launch_dependents();
-    if (warp == 0) {
-        if (lane == 0 && cta != g.stall_cta) g1_produce(g, sh, smem, cta, ncta, 1);
-        return;
-    }
     pdl_wait();
-    const int cw = warp - 1;
-    g1_stage<XM>(g, sh, smem, threadIdx.x - 32);
-    const int pi = g.wp[cw];
-    if (pi < g.count) {
-        const G1Prob& q = g.prob[pi];
-        int r0, n;
-        g1_rows(q, cta, ncta, r0, n);
-        const int sl = g.ws[cw], j = g.wj[cw], nn = g.wn[cw], R = g.wr[cw];
-        const bool two = min(q.slice_w, (q.K >> 6) - sl * q.slice_w) > 32;  // groups per lane: 2 or 1
-        if (R == 4)
-            two ? g1_rows_loop<4, 2>(g, q, sh, smem, pi, sl, j, nn, r0, n)
-                : g1_rows_loop<4, 1>(g, q, sh, smem, pi, sl, j, nn, r0, n);
-        else if (R == 2)
-            two ? g1_rows_loop<2, 2>(g, q, sh, smem, pi, sl, j, nn, r0, n)
-                : g1_rows_loop<2, 1>(g, q, sh, smem, pi, sl, j, nn, r0, n);
-        else
-            two ? g1_rows_loop<1, 2>(g, q, sh, smem, pi, sl, j, nn, r0, n)
-                : g1_rows_loop<1, 1>(g, q, sh, smem, pi, sl, j, nn, r0, n);
-    }
+    g1_stage<XM>(g, sh, smem);
+
+    if (seq.R == 4)
+        width > 32 ? g1_loop<4, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<4, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+    else if (seq.R == 2)
+        width > 32 ? g1_loop<2, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<2, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+    else
+        width > 32 ? g1_loop<1, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<1, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+
     if (g.sliced) {  // every slice of every row is in: finish the sliced rows
-        g1_consumer_sync();
-        if (*(volatile int*)&sh.abort_flag) return;
-        const int ctid = threadIdx.x - 32;
+        __syncthreads();
         for (int p = 0; p < g.count; ++p) {
-            const G1Prob& q = g.prob[p];
-            if (q.nslice == 1) continue;
-            int r0, n;
-            g1_rows(q, cta, ncta, r0, n);
+            const G1Prob& qq = g.prob[p];
+            if (qq.nslice == 1) continue;
+            int rr0, nn;
+            g1_rows(qq, cta, ncta, rr0, nn);
             const float f = sh.fscale[p];
             const int rowsum = sh.rowsum[p];
-            for (int i = ctid; i < n; i += G1_CWARPS * 32) g1_store(g, q, r0 + i, sh.part[q.part_off + i] - rowsum, f);
+            for (int i = threadIdx.x; i < nn; i += G1_THREADS)
+                g1_store(g, qq, rr0 + i, sh.part[qq.part_off + i] - rowsum, f);
         }
     }
 }
@@ -438,7 +356,7 @@ int g1_cost(int rows, int upl, int n, int& best_r) {
         const int batches = (rows + R - 1) / R;
         const int per_warp = (batches + n - 1) / n * R;
         const int red = R == 1 ? 10 : R == 2 ? 5 : 3;  // shuffle-reduction steps per row
-        const int c = per_warp * (upl * 33 + 4 + red);
+        const int c = per_warp * (upl * 35 + 6 + red);
         if (c < best) {
             best = c;
             best_r = R;
@@ -447,12 +365,10 @@ int g1_cost(int rows, int upl, int n, int& best_r) {
     return best;
 }
 
-}  // namespace
-
 // Plan the launch; false when the problem set does not suit the kernel (the
 // caller then uses the general small-M kernel).
-static bool g1_plan(const GemvProblem* probs, int count, int x_mode, YMode mode, const DevInfo& dev, G1Params& g,
-                    int& grid, size_t& smem) {
+bool g1_plan(const GemvProblem* probs, int count, int x_mode, YMode mode, const DevInfo& dev, G1Params& g, int& grid,
+             size_t& smem) {
     if (count < 1 || count > G1_MAX_PROBS) return false;
     g = {};
     g.count = count;
@@ -466,15 +382,12 @@ static bool g1_plan(const GemvProblem* probs, int count, int x_mode, YMode mode,
         maxN = std::max(maxN, probs[i].N);
         pairs += (K / 64 + G1_SLICE_UNITS - 1) / G1_SLICE_UNITS;
     }
-    if (sumK > G1_MAX_SUMK || pairs > G1_CWARPS) return false;
+    if (sumK > G1_MAX_SUMK || pairs > G1_WARPS) return false;
     grid = std::max(1, std::min(dev.num_sms, maxN));
     // two CTAs per SM: the shared memory of one SM (228 KB) halved, less the
     // 1 KB the hardware reserves per CTA
     const int budget = std::min(dev.max_smem_optin, 233472 / 2 - 1024);
-    int off = G1_HDR;
-    long long slab_bytes[G1_MAX_PROBS];
-    long long total = 0;
-    int part = 0;
+    int off = G1_HDR, part = 0;
     for (int i = 0; i < count; ++i) {
         G1Prob& q = g.prob[i];
         const GemvProblem& s = probs[i];
@@ -491,58 +404,32 @@ static bool g1_plan(const GemvProblem* probs, int count, int x_mode, YMode mode,
         const int U = s.K / 64;
         q.nslice = (U + G1_SLICE_UNITS - 1) / G1_SLICE_UNITS;
         q.slice_w = (U + q.nslice - 1) / q.nslice;
-        const int rows_max = (s.N + grid - 1) / grid;
-        int rpc = 1;
-        while (rpc * 2 * q.rb <= G1_CHUNK_TARGET && rpc * 2 <= std::max(1, rows_max)) rpc *= 2;
-        q.rpc_shift = 0;
-        while ((1 << q.rpc_shift) < rpc) ++q.rpc_shift;
-        q.slot = rpc * q.rb;
         if (q.nslice > 1) {
             q.part_off = part;
-            part += rows_max;
+            part += (s.N + grid - 1) / grid;
         }
-        slab_bytes[i] = (long long)rows_max * q.rb;
-        total += slab_bytes[i];
         g.sliced |= q.nslice > 1;
     }
     if (part > G1_PART_MAX) return false;
-    const int ring_budget = budget - off;
-    if (ring_budget <= 0) return false;
-    int bars = 0;
-    for (int i = 0; i < count; ++i) {
-        G1Prob& q = g.prob[i];
-        const int rows_max = (q.N + grid - 1) / grid;
-        const int nch = (rows_max + (1 << q.rpc_shift) - 1) >> q.rpc_shift;
-        const long long share = (long long)ring_budget * slab_bytes[i] / std::max(1LL, total);
-        int st = (int)std::min<long long>(share / q.slot, nch);
-        // a batch of up to 4 rows spans at most 4 / rpc + 1 chunks; the ring
-        // must hold that many so that a warp never waits on a chunk whose
-        // slot it still holds
-        const int span = std::min(nch, 4 / (1 << q.rpc_shift) + 1 + ((4 % (1 << q.rpc_shift)) ? 1 : 0));
-        if (st < span) return false;
-        q.stages = st;
-        q.ring_off = off;
-        off += st * q.slot;
-        q.bar0 = bars;
-        bars += st;
-    }
-    if (bars > G1_MAX_BARS || off > budget) return false;
-    // consumer warps: one per (problem, slice) to start with, the rest to the
-    // group whose slowest warp has the most work
+    g.ring_off = off;
+    off += G1_WARPS * G1_DEPTH * G1_SLOT;
+    if (off > budget) return false;
+    // warps: one per (problem, slice) to start with, the rest to the group
+    // whose slowest warp has the most work
     struct Pair {
-        int p, s, rows, upl, n, r;
+        int p, s, rows, upl, n;
     };
-    Pair pr[G1_CWARPS];
+    Pair pr[G1_WARPS];
     int np = 0;
     for (int i = 0; i < count; ++i) {
         const G1Prob& q = g.prob[i];
         const int U = q.K / 64;
         for (int s = 0; s < q.nslice; ++s) {
             const int width = std::min(q.slice_w, U - s * q.slice_w);
-            pr[np++] = {i, s, (q.N + grid - 1) / grid, width > 32 ? 2 : 1, 1, 1};
+            pr[np++] = {i, s, (q.N + grid - 1) / grid, width > 32 ? 2 : 1, 1};
         }
     }
-    for (int w = np; w < G1_CWARPS; ++w) {
+    for (int w = np; w < G1_WARPS; ++w) {
         int worst = 0, wc = -1;
         for (int k = 0; k < np; ++k) {
             int r;
@@ -570,6 +457,8 @@ static bool g1_plan(const GemvProblem* probs, int count, int x_mode, YMode mode,
     return true;
 }
 
+}  // namespace
+
 bool gemv1_ok(const GemvProblem* probs, int count, int M, const DevInfo& dev) {
     if (M != 1) return false;
     G1Params g;
@@ -586,12 +475,6 @@ cudaError_t launch_gemv1(const GemvProblem* probs, int count, int x_dtype, YMode
     int grid;
     size_t smem;
     if (!g1_plan(probs, count, xm, mode, dev, g, grid, smem)) return cudaErrorInvalidValue;
-    g.wait_limit = WAIT_LIMIT_CYCLES;
-    g.stall_cta = -1;
-    if (take_wait_expiry_request()) {  // test hook: CTA 0 never receives its weights
-        g.wait_limit = 100000;
-        g.stall_cta = 0;
-    }
     auto k = xm == X_QUANTISED ? gemv1_kernel<X_QUANTISED> : xm == X_BF16 ? gemv1_kernel<X_BF16> : gemv1_kernel<X_F32>;
     cudaError_t e = ensure_smem_optin(reinterpret_cast<const void*>(k), smem);
     if (e != cudaSuccess) return e;

@@ -71,7 +71,8 @@ cudaError_t launch_gemv1(const GemvProblem* probs, int count, int x_dtype, YMode
                          cudaStream_t st);
 
 // api.cu: true once after bitlinear_test_expire_next_wait(1) (test hook of
-// the bounded waits; consumed by the next one-token decode launch)
+// the bounded waits; consumed by the next launch of the general small-M
+// decode kernel's batched form)
 bool take_wait_expiry_request();
 
 // k_decode_tc.cu  (M <= 16, tcgen05 int8 tensor cores)
@@ -88,10 +89,14 @@ DecodePath decode_path(int M, const GemvProblem* probs, int count, const DevInfo
 cudaError_t launch_decode_cuda(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
                                const DevInfo& dev, cudaStream_t st);
 
-// k_gemm.cu  (M > 64, tcgen05 int8 tensor cores); wbits 2 (trits) or 1 (signs)
+// k_gemm.cu  (tcgen05 int8 tensor cores); wbits 2 (trits) or 1 (signs).  The
+// workspace holds the row sums and, when few tiles are cut along K
+// (allow_split), the per-tile counters and partial tiles; gemm_ws_bytes
+// sizes it for allow_split, and M int32 suffice without.
 size_t gemm_ws_bytes(long long M, long long N, long long K);
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
-                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits = 2);
+                        int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits = 2,
+                        bool allow_split = true);
 
 // k_group.cu  (group quantisation along K)
 size_t regroup_ws_bytes(long long N, long long K);

@@ -103,6 +103,7 @@ extern "C" bl_status bitlinear_forward_noalloc(const int8_t* x_q, const float* g
     else if (path == PATH_CUDA)
         e = launch_decode_cuda(&prob, 1, (int)M, BL_I8, mode, d->info, st);
     else
-        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->scratch, d->info, st);
+        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, d->scratch, d->info, st, 2,
+                        false);  // the static scratch holds row sums only: no split along K
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }

@@ -181,7 +181,7 @@ def test_binary_forward_validation():
     assert _L().bitlinear_forward_binary_fp_workspace(1, 4096, 4096) == 0
     need = _L().bitlinear_forward_binary_fp_workspace(64, 4096, 4096)
     assert need >= 64 * 4096 + 64 * 4
-    assert h(P(A1), 0, 64, 4096, P(A3), P(A4), 64, P(A5), 0, P(A6), need - 1, None) == WS
+    assert h(P(A1), 0, 64, 4096, P(A3), P(A4), 4096, P(A5), 0, P(A6), need - 1, None) == WS
     assert h(P(A1), 0, 1, 1024, P(A3), P(A4), 64, P(A5), 0, None, 0, None) == DEVICE
 
 

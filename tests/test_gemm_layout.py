@@ -1,14 +1,19 @@
 """CPU emulation of the prefill GEMM's tile walk and operand layouts.
 
-The tcgen05 GEMM is persistent: CTA b takes tiles b, b + grid, ... in
-m-fastest order (128 x 256 output tiles), and per 128-byte K-block a TMA
+The tcgen05 GEMM is persistent: CTA b takes work units b, b + grid, ...;
+a unit is a 128 x 256 output tile (m-fastest order) and, when there are few
+tiles, one of `splits` ranges of its K-blocks.  Per 128-byte K-block a TMA
 box of x_q (128 rows, 128-byte swizzle, zero fill past M and K) and a box of
 packed words (256 rows, zero fill) land in a stage; unpack warps expand each
 word into 16-byte code chunks of the K-major, 128-byte-swizzled B operand
 (2-bit trits: one chunk per word; 1-bit signs: two chunks per word, codes
 {0, 2}); four MMAs of K = 32 walk both swizzled operands; the epilogue
-subtracts the token's row sum.  This test restates those steps in numpy,
-with garbage in the stage before every fill, and requires the oracle's
+subtracts the token's row sum.  With splits, each unit stores its int32 tile
+to the workspace and a separate kernel adds the partial tiles of every
+output, four columns per thread.  This test restates those steps in
+numpy, with garbage in the stage before every fill and in the workspace,
+restates the host's choice of splits and workspace size, checks every
+partial-tile index against that size, and requires the oracle's
 contraction, for ternary and for 1-bit weights.
 """
 import numpy as np
@@ -17,6 +22,18 @@ import pytest
 import oracle
 
 BM, BN, BK = 128, 256, 128
+SPLIT_UNITS_TARGET = 148
+
+
+def plan(M, N, K, allow_split=True):
+    tiles_m, tiles_n, num_kb = (M + BM - 1) // BM, (N + BN - 1) // BN, (K + BK - 1) // BK
+    tiles = tiles_m * tiles_n
+    splits = max(1, min(SPLIT_UNITS_TARGET // tiles, num_kb)) if allow_split else 1
+    part_rows = min(M, BM)
+    rowsum_bytes = (M * 4 + 255) // 256 * 256
+    part_bytes = tiles * splits * part_rows * BN * 4 if splits > 1 else 0
+    return dict(tiles_m=tiles_m, tiles_n=tiles_n, num_kb=num_kb, splits=splits, part_rows=part_rows,
+                ws_bytes=rowsum_bytes + part_bytes, part_off=rowsum_bytes)
 
 
 def sw128_off(row, chunk):
@@ -32,18 +49,28 @@ def tma_box(src: np.ndarray, r0: int, c0: int, rows: int, cols: int) -> np.ndarr
     return box
 
 
-def emulate(x_q, W_p, K, N, wbits, grid, rng):
+def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
     M = x_q.shape[0]
-    tiles_m, tiles_n, num_kb = (M + BM - 1) // BM, (N + BN - 1) // BN, (K + BK - 1) // BK
+    pl = plan(M, N, K, allow_split)
+    tiles_m, tiles_n, num_kb, splits, part_rows = (pl[k] for k in ("tiles_m", "tiles_n", "num_kb", "splits",
+                                                                    "part_rows"))
     wpr = BK * wbits // 32                            # packed words per row and K-block
     xq_u8 = x_q.view(np.uint8)
     rowsum = x_q.astype(np.int64).sum(1)
     y = np.full((M, N), -(2 ** 40), np.int64)
+    units = tiles_m * tiles_n * splits
+    part_ints = (pl["ws_bytes"] - pl["part_off"]) // 4
+    part = rng.integers(-2 ** 31, 2 ** 31, max(part_ints, 1), dtype=np.int64)   # garbage on entry
+    kb_seen = np.zeros((tiles_m * tiles_n, num_kb), np.int64)
     for cta in range(grid):
-        for t in range(cta, tiles_m * tiles_n, grid):
+        for u in range(cta, units, grid):
+            t = u // splits
+            sp = u % splits
+            kb0, kb1 = num_kb * sp // splits, num_kb * (sp + 1) // splits
             mb, nb = t % tiles_m, t // tiles_m
             D = np.zeros((BM, BN), np.int64)
-            for kb in range(num_kb):
+            for kb in range(kb0, kb1):
+                kb_seen[t, kb] += 1
                 a_st = rng.integers(0, 256, BM * BK, dtype=np.int64).astype(np.uint8)
                 b_st = rng.integers(0, 256, BN * BK, dtype=np.int64).astype(np.uint8)
                 # x_q box with the 128-byte swizzle
@@ -72,11 +99,32 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng):
                               for n in range(BN)]).view(np.int8).astype(np.int64)
                 for k in range(BK // 32):
                     D += A[:, 32 * k:32 * k + 32] @ B[:, 32 * k:32 * k + 32].T
-            for r in range(BM):
-                m = mb * BM + r
-                if m < M:
-                    n0, n1 = nb * BN, min(N, nb * BN + BN)
-                    y[m, n0:n1] = D[r, :n1 - n0] - rowsum[m]
+            if splits == 1:
+                for r in range(BM):
+                    m = mb * BM + r
+                    if m < M:
+                        n0, n1 = nb * BN, min(N, nb * BN + BN)
+                        y[m, n0:n1] = D[r, :n1 - n0] - rowsum[m]
+                continue
+            for r in range(BM):                       # this unit's partial tile
+                if r < part_rows and mb * BM + r < M:
+                    o = (u * part_rows + r) * BN
+                    assert o + BN <= part_ints
+                    part[o:o + BN] = D[r]
+    assert np.all(kb_seen == 1)                       # every (tile, K-block) exactly once
+    if splits > 1:                                    # the finishing kernel: four columns per thread
+        for m in range(M):
+            for n in range(0, N, 4):
+                mb, r, nb, c = m // BM, m % BM, n // BN, n % BN
+                t = mb + nb * tiles_m
+                tot = np.zeros(4, np.int64)
+                for s2 in range(splits):
+                    o = ((t * splits + s2) * part_rows + r) * BN + c
+                    assert o + 4 <= part_ints
+                    tot += part[o:o + 4]
+                for j in range(4):
+                    if n + j < N:
+                        y[m, n + j] = tot[j] - rowsum[m]
     return y
 
 
@@ -87,6 +135,30 @@ def test_ternary_gemm_emulation_matches_the_oracle(M, K, N, grid):
     x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
     y = emulate(x_q, oracle.pack(W_t), K, N, 2, grid, rng)
     np.testing.assert_array_equal(y, oracle.ternary_acc(x_q, W_t))
+
+
+@pytest.mark.parametrize("M,K,N,grid", [(64, 1024, 1300, 40), (17, 640, 260, 7), (130, 512, 1000, 148),
+                                        (64, 4096, 300, 16)])
+def test_split_k_gemm_emulation_matches_the_oracle(M, K, N, grid):
+    # few tiles: units of (tile, K range), partial tiles summed by the last
+    # warp of each quarter; the chosen splits and the workspace they need
+    pl = plan(M, N, K)
+    assert pl["splits"] > 1
+    assert pl["tiles_m"] * pl["tiles_n"] * pl["splits"] <= SPLIT_UNITS_TARGET
+    rng = np.random.default_rng(M * 7 + K + N)
+    W_t = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    y = emulate(x_q, oracle.pack(W_t), K, N, 2, grid, rng, allow_split=True)
+    np.testing.assert_array_equal(y, oracle.ternary_acc(x_q, W_t))
+
+
+def test_split_k_plan_of_the_small_batch_shapes():
+    # M = 16 and 64 on K = 4096: 16 or 43 tiles, cut into 9 or 3 K ranges
+    for M in (16, 64):
+        assert plan(M, 4096, 4096)["splits"] == 9
+        assert plan(M, 11008, 4096)["splits"] == 3
+    # prefill: enough tiles, no split
+    assert plan(2048, 4096, 4096)["splits"] == 1 and plan(2048, 11008, 4096)["splits"] == 1
 
 
 @pytest.mark.parametrize("M,K,N,grid", [(130, 384, 300, 2), (5, 128, 260, 1)])

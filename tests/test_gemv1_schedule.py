@@ -1,23 +1,22 @@
 """CPU check of the one-token streaming GEMV's plan and index walk.
 
 The one-token kernel gives every CTA (one per SM) a contiguous slab of rows
-of every problem, streams each problem's slab through its own ring of chunk
-slots (a power-of-two number of rows each) and binds every consumer warp to
-one K slice of one problem, with that slice of x_hat in registers.  Its
-correctness rests on host-side planning that the GPU parity tests only
+of every problem and binds every warp to one K slice of one problem, with
+that slice of x_hat in registers; every lane streams its own 16-byte groups
+of the warp's rows with cp.async through a per-warp ring of DEPTH slots.
+Its correctness rests on host-side planning that the GPU parity tests only
 sample.  This test restates the plan and the device-side walk in Python and
 checks, over a sweep of problem sets:
   * shared memory: header, x_hat areas and rings are disjoint and fit half an
-    SM (two CTAs per SM); barrier and slice-sum indices fit their tables;
+    SM (two CTAs per SM); slice-sum indices fit their table;
   * the staging threads cover every 16-element activation chunk exactly once
     and write inside the problem's x_hat area;
-  * every bulk copy stays inside its slot and inside W_p;
-  * every (row, K slice) of every CTA is computed exactly once, each weight
-    read lies inside the bytes its chunk brought in, each x_hat read inside
-    the problem's K;
-  * a warp's batch of rows never spans more chunks than its ring holds (so
-    no warp waits for a slot it still holds), and every chunk but the last of
-    a slab collects exactly the arrivals its empty barrier counts;
+  * every copy stays inside its ring slot and inside its row of W_p, and
+    every read of a slot reads back exactly the bytes the same lane copied
+    into it for the same row (the commit-group accounting: DEPTH groups in
+    flight, one committed per row consumed);
+  * every (row, K slice) of every CTA is computed exactly once, each x_hat
+    read lies inside the problem's K;
   * the slice partition reproduces the oracle's integer accumulators.
 """
 import numpy as np
@@ -27,12 +26,12 @@ import oracle
 import workloads
 
 NUM_SMS, SMEM_OPTIN = 148, 232448                 # B200
-MAX_PROBS, CWARPS, MAX_BARS, PART_MAX = 8, 15, 64, 512
-SLICE_UNITS, CHUNK_TARGET, XC = 64, 8192, 2
-MAX_SUMK = XC * CWARPS * 32 * 16
-# G1Shared: 2 x 64 mbarriers, abort flag, rowsum/beta/fscale[8], red[15][8], part[512]
-HDR = ((2 * MAX_BARS * 8 + 4 + 3 * MAX_PROBS * 4 + CWARPS * MAX_PROBS * 4 + PART_MAX * 4 + 7) // 8 * 8 + 127) \
-    // 128 * 128
+MAX_PROBS, WARPS, DEPTH, SLOT, PART_MAX = 8, 16, 5, 1024, 512
+SLICE_UNITS, XC = 64, 2
+THREADS = WARPS * 32
+MAX_SUMK = XC * THREADS * 16
+# G1Shared: rowsum/beta/fscale[8], red[16][8], part[512]
+HDR = ((3 * MAX_PROBS * 4 + WARPS * MAX_PROBS * 4 + PART_MAX * 4 + 3) // 4 * 4 + 127) // 128 * 128
 
 
 def cost(rows, upl, n):
@@ -41,7 +40,7 @@ def cost(rows, upl, n):
         batches = (rows + R - 1) // R
         per_warp = (batches + n - 1) // n * R
         red = 10 if R == 1 else 5 if R == 2 else 3
-        c = per_warp * (upl * 33 + 4 + red)
+        c = per_warp * (upl * 35 + 6 + red)
         if c < best:
             best, best_r = c, R
     return best, best_r
@@ -51,15 +50,15 @@ def plan(probs):
     """probs: list of (K, N).  Returns the plan dict or None (kernel not used)."""
     if not 1 <= len(probs) <= MAX_PROBS:
         return None
-    sumK = sum(K for K, _ in probs)
     if any(K % 64 or K < 64 * 32 for K, _ in probs):
         return None
+    sumK = sum(K for K, _ in probs)
     pairs = sum((K // 64 + SLICE_UNITS - 1) // SLICE_UNITS for K, _ in probs)
-    if sumK > MAX_SUMK or pairs > CWARPS:
+    if sumK > MAX_SUMK or pairs > WARPS:
         return None
     grid = max(1, min(NUM_SMS, max(N for _, N in probs)))
     budget = min(SMEM_OPTIN, 233472 // 2 - 1024)
-    off, part, total = HDR, 0, 0
+    off, part = HDR, 0
     P = []
     for K, N in probs:
         q = dict(K=K, N=N, rb=K // 4, xq_off=off)
@@ -67,37 +66,15 @@ def plan(probs):
         U = K // 64
         q["nslice"] = (U + SLICE_UNITS - 1) // SLICE_UNITS
         q["slice_w"] = (U + q["nslice"] - 1) // q["nslice"]
-        rows_max = (N + grid - 1) // grid
-        rpc = 1
-        while rpc * 2 * q["rb"] <= CHUNK_TARGET and rpc * 2 <= max(1, rows_max):
-            rpc *= 2
-        q["rpc"] = rpc
-        q["shift"] = rpc.bit_length() - 1
-        q["slot"] = rpc * q["rb"]
         if q["nslice"] > 1:
             q["part_off"] = part
-            part += rows_max
-        q["slab"] = rows_max * q["rb"]
-        total += q["slab"]
+            part += (N + grid - 1) // grid
         P.append(q)
     if part > PART_MAX:
         return None
-    ring_budget = budget - off
-    if ring_budget <= 0:
-        return None
-    bars = 0
-    for q in P:
-        rows_max = (q["N"] + grid - 1) // grid
-        nch = (rows_max + q["rpc"] - 1) >> q["shift"]
-        share = ring_budget * q["slab"] // max(1, total)
-        st = min(share // q["slot"], nch)
-        span = min(nch, 4 // q["rpc"] + 1 + (1 if 4 % q["rpc"] else 0))
-        if st < span:
-            return None
-        q["stages"], q["ring_off"], q["bar0"] = st, off, bars
-        off += st * q["slot"]
-        bars += st
-    if bars > MAX_BARS or off > budget:
+    ring_off = off
+    off += WARPS * DEPTH * SLOT
+    if off > budget:
         return None
     pr = []
     for i, q in enumerate(P):
@@ -105,7 +82,7 @@ def plan(probs):
         for s in range(q["nslice"]):
             width = min(q["slice_w"], U - s * q["slice_w"])
             pr.append(dict(p=i, s=s, rows=(q["N"] + grid - 1) // grid, upl=2 if width > 32 else 1, n=1))
-    for _ in range(len(pr), CWARPS):
+    for _ in range(len(pr), WARPS):
         worst = max(range(len(pr)), key=lambda k: (cost(pr[k]["rows"], pr[k]["upl"], pr[k]["n"])[0], -k))
         pr[worst]["n"] += 1
     roles = []
@@ -113,8 +90,8 @@ def plan(probs):
         R = cost(e["rows"], e["upl"], e["n"])[1]
         for j in range(e["n"]):
             roles.append((e["p"], e["s"], j, e["n"], R))
-    assert len(roles) == CWARPS
-    return dict(P=P, grid=grid, smem=off, budget=budget, roles=roles, bars=bars)
+    assert len(roles) == WARPS
+    return dict(P=P, grid=grid, smem=off, budget=budget, roles=roles, ring_off=ring_off)
 
 
 def rows_of(q, cta, ncta):
@@ -125,20 +102,19 @@ def rows_of(q, cta, ncta):
 def check_plan(pl):
     P, grid = pl["P"], pl["grid"]
     assert pl["smem"] <= pl["budget"] and 2 * (pl["smem"] + 1024) <= 233472
-    # disjoint, 16-byte aligned areas
     areas = [(0, HDR)] + [(q["xq_off"], q["xq_off"] + q["K"]) for q in P] + \
-            [(q["ring_off"], q["ring_off"] + q["stages"] * q["slot"]) for q in P]
+            [(pl["ring_off"], pl["ring_off"] + WARPS * DEPTH * SLOT)]
     areas.sort()
     for (a0, a1), (b0, b1) in zip(areas, areas[1:]):
         assert a1 <= b0
     for q in P:
-        assert q["xq_off"] % 16 == 0 and q["ring_off"] % 16 == 0 and q["slot"] % 16 == 0
-        assert q["bar0"] + q["stages"] <= MAX_BARS
-    # staging: chunk g of the concatenation -> thread g % 480, cache slot g // 480
+        assert q["xq_off"] % 16 == 0
+    assert pl["ring_off"] % 16 == 0
+    # staging: chunk g of the concatenation -> thread g % THREADS, cache slot g // THREADS
     seen = set()
-    for ctid in range(CWARPS * 32):
+    for tid in range(THREADS):
         for i in range(XC):
-            gi, p = ctid + i * CWARPS * 32, -1
+            gi, p = tid + i * THREADS, -1
             for j, q in enumerate(P):
                 gj = q["K"] >> 4
                 if p < 0 and gi < gj:
@@ -150,7 +126,7 @@ def check_plan(pl):
                 seen.add((p, gi))
     assert len(seen) == sum(q["K"] // 16 for q in P)
     for cta in range(grid):
-        done = {}
+        done = set()
         for w, (p, s, j, n, R) in enumerate(pl["roles"]):
             q = P[p]
             r0, nrows = rows_of(q, cta, grid)
@@ -159,43 +135,58 @@ def check_plan(pl):
             width = min(q["slice_w"], U - u0)
             assert width > 0
             upl = 2 if width > 32 else 1
-            for lane in range(32):  # x_hat reads
-                for u in (u0 + lane, u0 + lane + 32):
-                    if u - u0 < width and (u == u0 + lane or upl == 2):
-                        assert 64 * u + 64 <= q["K"]
+            ring = pl["ring_off"] + w * DEPTH * SLOT
+
+            def row(t):
+                i = (j + (t // R) * n) * R + t % R
+                return i if i < nrows else -1
+
+            def groups(lane):
+                return [u for u in (u0 + lane, u0 + lane + 32) if u - u0 < width]
+
+            for lane in range(32):
+                for u in groups(lane):
+                    assert 64 * u + 64 <= q["K"]                       # x_hat read
+                    if u == u0 + lane + 32:
+                        assert upl == 2
+            # commit groups: DEPTH fetches, then one per consumed row; slot
+            # contents tracked per lane and byte offset
+            slot_row = {}
+            committed = []
+            for d in range(DEPTH):
+                slot_row[d] = row(d)
+                committed.append(row(d))
+            batches = (nrows + R - 1) // R
+            t = 0
             b = j
-            while b * R < nrows:
-                i0 = b * R
-                nv = min(R, nrows - i0)
-                ks = [(i0 + r) >> q["shift"] for r in range(nv)]
-                assert max(ks) - min(ks) + 1 <= q["stages"]       # no wait on a slot still held
-                for r in range(nv):
-                    i = i0 + r
-                    k = i >> q["shift"]
-                    rows_k = min(q["rpc"], nrows - k * q["rpc"])
-                    base = (i & (q["rpc"] - 1)) * q["rb"]
-                    hi = base + 16 * (u0 + min(width, 64 if upl == 2 else 32))
-                    assert hi <= rows_k * q["rb"] <= q["slot"]
-                    if q["nslice"] > 1:
-                        assert q["part_off"] + i < PART_MAX
-                    assert r0 + i < q["N"]
-                    key = (p, i, s)
-                    assert key not in done
-                    done[key] = w
+            while b < batches:
+                for r in range(R):
+                    # wait_group(DEPTH - 1): groups 0 .. t have landed
+                    assert len(committed) - (t + 1) <= DEPTH - 1
+                    slot = t % DEPTH
+                    i = row(t)
+                    assert slot_row[slot] == i                       # the slot holds row t
+                    if i >= 0:
+                        assert (j + (t // R) * n) * R + t % R == b * R + r
+                        for lane in range(32):
+                            for u in groups(lane):
+                                dst = ring + slot * SLOT + 16 * (u - u0)
+                                assert ring <= dst and dst + 16 <= ring + DEPTH * SLOT
+                                src = (r0 + i) * q["rb"] + 16 * u
+                                assert src + 16 <= (r0 + i + 1) * q["rb"] <= q["N"] * q["rb"]
+                        key = (p, i, s)
+                        assert key not in done
+                        done.add(key)
+                        if q["nslice"] > 1:
+                            assert q["part_off"] + i < PART_MAX
+                        assert r0 + i < q["N"]
+                    slot_row[slot] = row(t + DEPTH)
+                    committed.append(row(t + DEPTH))
+                    t += 1
                 b += n
         for p, q in enumerate(P):
             r0, nrows = rows_of(q, cta, grid)
             assert sum(1 for (pp, _, _) in done if pp == p) == nrows * q["nslice"]
-            # bulk copies
-            nch = (nrows + q["rpc"] - 1) >> q["shift"]
-            for k in range(nch):
-                rows = min(q["rpc"], nrows - (k << q["shift"]))
-                assert rows > 0
-                assert (r0 + (k << q["shift"]) + rows) * q["rb"] <= q["N"] * q["rb"]
-                assert rows * q["rb"] <= q["slot"]
-                if k < nch - 1:   # reused slots: arrivals == count
-                    arrivals = sum(1 for (pp, i, _) in done if pp == p and (i >> q["shift"]) == k)
-                    assert arrivals == q["rpc"] * q["nslice"]
 
 
 DECODE_SETS = {
@@ -231,10 +222,10 @@ def test_plan_and_walk_in_bounds(probs):
     if pl is None:
         # rejected sets run on the general small-M kernel; only the structural
         # limits may reject
-        assert (any(K < 2048 for K, _ in probs) or sum(K for K, _ in probs) > MAX_SUMK
-                or sum((K // 64 + 63) // 64 for K, _ in probs) > CWARPS
-                or any((N + min(NUM_SMS, max(n for _, n in probs)) - 1) // min(NUM_SMS, max(n for _, n in probs))
-                       > PART_MAX for K, N in probs if K > 4096))
+        grid = min(NUM_SMS, max(n for _, n in probs))
+        assert (any(K < 2048 or K % 64 for K, _ in probs) or sum(K for K, _ in probs) > MAX_SUMK
+                or sum((K // 64 + 63) // 64 for K, _ in probs) > WARPS
+                or sum((N + grid - 1) // grid for K, N in probs if K > 4096) > PART_MAX)
         return
     check_plan(pl)
 
