@@ -522,10 +522,10 @@ int bitlinear_num_sms(void);
 /*
  * Test hook of the bounded waits (no counterpart on the pages).  With
  * enable != 0, the next launch of the general small-M CUDA-core decode
- * kernel by bitlinear_forward_fp_batch (for instance with the engine
- * BL_ENGINE_CUDA_CORES_GENERAL and M <= 4) limits each wait of its first
- * problem to about 10^5 SM cycles, and the weight producer of that problem's
- * first CTA issues no copies, so that CTA's consumers give up waiting for
+ * kernel (M <= 4 tokens; with the engine BL_ENGINE_CUDA_CORES_GENERAL it
+ * also runs one token) limits each wait of its first problem to about 10^5
+ * SM cycles, and the weight producer of that problem's first CTA issues no
+ * copies, so that CTA's consumers give up waiting for
  * data that never comes: the kernel raises the device error word and
  * returns (no copy is in flight, nothing hangs), that CTA's outputs are
  * unspecified, and the next bitlinear_device_status returns BL_ERR_TIMEOUT.

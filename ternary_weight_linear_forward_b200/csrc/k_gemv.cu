@@ -723,6 +723,10 @@ cudaError_t launch_gemv_impl(GemvParams& p, const DevInfo& dev, cudaStream_t st)
     const int M = p.M, N = p.N;
     if (small_ok(M, p.K)) {
         const SmallShape sh = configure_small(p, dev, GEMV_CO_RESIDENT);
+        if (take_wait_expiry_request()) {  // test hook: the first CTA never receives its weights
+            p.wait_limit = 100000;
+            p.stall_cta = 0;
+        }
         const int mt = small_mt(M);
         GemvKernel k = small_kernel_for_mode<2>(p.x_mode, sh.lpr, mt, sh.r);
         return launch_with_smem(k, sh.grid, (sh.cwarps + 1) * 32, sh.smem, st, p);

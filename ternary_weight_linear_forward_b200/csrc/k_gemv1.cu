@@ -83,6 +83,7 @@ struct G1Params {
 };
 
 struct G1Shared {
+    G1Prob prob[G1_MAX_PROBS];  // the problem descriptors, copied from the parameters
     int rowsum[G1_MAX_PROBS];
     float beta[G1_MAX_PROBS];
     float fscale[G1_MAX_PROBS];
@@ -106,15 +107,15 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void g1_store(const G1Params& g, const G1Prob& q, int n, int acc, float f) {
-    if (g.mode == Y_ACC) {
-        reinterpret_cast<int*>(q.y)[n] = acc;
+__device__ __forceinline__ void g1_store(int mode, void* y, int n, int acc, float f) {
+    if (mode == Y_ACC) {
+        reinterpret_cast<int*>(y)[n] = acc;
     } else {
         const float v = __fmul_rn((float)acc, f);
-        if (g.mode == Y_F32)
-            reinterpret_cast<float*>(q.y)[n] = v;
+        if (mode == Y_F32)
+            reinterpret_cast<float*>(y)[n] = v;
         else
-            reinterpret_cast<uint16_t*>(q.y)[n] = f32_to_bf16_rn(v);
+            reinterpret_cast<uint16_t*>(y)[n] = f32_to_bf16_rn(v);
     }
 }
 
@@ -155,6 +156,7 @@ struct Lane {
 // and the code pass.  Called by all threads (two CTA barriers).
 template <int XM>
 __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsigned char* smem) {
+    const G1Prob* prob = sh.prob;  // the shared copy: indexed at run time without reloading parameters
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     XChunk<XM> cache[G1_XC];
     int cp[G1_XC], cg[G1_XC];
@@ -163,13 +165,13 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
         int gi = tid + i * G1_THREADS;
         int p = -1;
         for (int j = 0; j < g.count; ++j) {
-            const int gj = g.prob[j].K >> 4;
+            const int gj = prob[j].K >> 4;
             if (p < 0 && gi < gj) p = j;
             if (p < 0) gi -= gj;
         }
         cp[i] = p;
         cg[i] = gi;
-        if (p >= 0) ld_chunk<XM>(g.prob[p].x, gi, cache[i]);
+        if (p >= 0) ld_chunk<XM>(prob[p].x, gi, cache[i]);
     }
     float s[G1_XC];
 #pragma unroll
@@ -202,7 +204,7 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
             sh.fscale[tid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[tid], gam), 127.0f);
         }
     } else if (tid < g.count) {
-        sh.fscale[tid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[tid], __ldg(g.prob[tid].gamma)), 127.0f);
+        sh.fscale[tid] = g.mode == Y_ACC ? 0.0f : __fdiv_rn(__fmul_rn(sh.beta[tid], __ldg(prob[tid].gamma)), 127.0f);
     }
     for (int i = tid; i < G1_PART_MAX; i += G1_THREADS) sh.part[i] = 0;
     int rs[G1_XC];
@@ -212,7 +214,7 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
         if (cp[i] >= 0) {
             const int4 q = chunk_codes<XM>(cache[i], s[i]);
             rs[i] = bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
-            *reinterpret_cast<int4*>(smem + g.prob[cp[i]].xq_off + 16 * cg[i]) = q;
+            *reinterpret_cast<int4*>(smem + prob[cp[i]].xq_off + 16 * cg[i]) = q;
         }
     }
     for (int p = 0; p < g.count; ++p) {
@@ -227,13 +229,20 @@ __device__ __forceinline__ void g1_stage(const G1Params& g, G1Shared& sh, unsign
 }
 
 // One warp's share of problem q, K slice starting at group u0: the rows of
-// `seq`, rows 0 .. DEPTH-1 of which are already in flight.  UPL = 16-byte
-// groups per lane (1 or 2).  No barrier inside.
+// `seq`, rows 0 .. DEPTH-1 of which are already in flight.  A batch of R
+// rows is waited for at once, its words loaded at once and its R dot
+// products interleaved (independent chains), then its slots are refilled.
+// UPL = 16-byte groups per lane (1 or 2).  No barrier inside.
 template <int R, int UPL>
-__device__ __forceinline__ void g1_loop(const G1Params& g, const G1Prob& q, const G1Shared& sh,
+__device__ __forceinline__ void g1_loop(const int mode, const G1Prob& q, const G1Shared& sh,
                                         const unsigned char* smem, int pi, int u0, const RowSeq& seq, int r0,
                                         const Lane& ln) {
+    static_assert(R <= G1_DEPTH, "a batch must fit the ring");
     const int lane = ln.lane;
+    // loop invariants, read once (q is the shared-memory copy)
+    void* const y = q.y;
+    const int sliced = q.nslice > 1;
+    int* const part = const_cast<int*>(sh.part) + q.part_off;
     int4 xa[4], xb[4];  // x_hat of this lane's groups: 64 codes each, k = 64u .. 64u + 63
     const int4* xq = reinterpret_cast<const int4*>(smem + q.xq_off);
 #pragma unroll
@@ -244,43 +253,55 @@ __device__ __forceinline__ void g1_loop(const G1Params& g, const G1Prob& q, cons
     const float f = sh.fscale[pi];
     const int rowsum = sh.rowsum[pi];
     const int batches = (seq.nrows + R - 1) / R;
-    int t = 0;
-    for (int b = seq.j; b < batches; b += seq.n) {
+    int t = 0;  // rows of the sequence consumed so far
+    for (int b = seq.j; b < batches; b += seq.n, t += R) {
+        // rows t .. t+R-1 have landed once at most DEPTH - R groups are pending
+        cp_async_wait<G1_DEPTH - R>();
+        uint4 wa[R], wb[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const unsigned char* w = ln.ring + ((t + r) % G1_DEPTH) * G1_SLOT;
+            const bool live = b * R + r < seq.nrows;
+            wa[r] = live && ln.ha ? *reinterpret_cast<const uint4*>(w + 16 * lane) : make_uint4(0u, 0u, 0u, 0u);
+            wb[r] = UPL == 2 && live && ln.hb ? *reinterpret_cast<const uint4*>(w + 16 * (lane + 32))
+                                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+        int a[R][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) word_dot(wa[r].x, xa[0].x, xa[0].y, xa[0].z, xa[0].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+        for (int r = 0; r < R; ++r) word_dot(wa[r].y, xa[1].x, xa[1].y, xa[1].z, xa[1].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+        for (int r = 0; r < R; ++r) word_dot(wa[r].z, xa[2].x, xa[2].y, xa[2].z, xa[2].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+        for (int r = 0; r < R; ++r) word_dot(wa[r].w, xa[3].x, xa[3].y, xa[3].z, xa[3].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+        if (UPL == 2) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) word_dot(wb[r].x, xb[0].x, xb[0].y, xb[0].z, xb[0].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+            for (int r = 0; r < R; ++r) word_dot(wb[r].y, xb[1].x, xb[1].y, xb[1].z, xb[1].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+            for (int r = 0; r < R; ++r) word_dot(wb[r].z, xb[2].x, xb[2].y, xb[2].z, xb[2].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+#pragma unroll
+            for (int r = 0; r < R; ++r) word_dot(wb[r].w, xb[3].x, xb[3].y, xb[3].z, xb[3].w, a[r][0], a[r][1], a[r][2], a[r][3]);
+        }
         int vals[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r, ++t) {
-            cp_async_wait<G1_DEPTH - 1>();  // row t's group has landed
-            const int slot = t % G1_DEPTH;
-            const unsigned char* w = ln.ring + slot * G1_SLOT;
-            vals[r] = 0;
-            if (seq.row(t) >= 0) {
-                const uint4 wa = ln.ha ? *reinterpret_cast<const uint4*>(w + 16 * lane) : make_uint4(0u, 0u, 0u, 0u);
-                const uint4 wb = UPL == 2 && ln.hb ? *reinterpret_cast<const uint4*>(w + 16 * (lane + 32))
-                                                   : make_uint4(0u, 0u, 0u, 0u);
-                int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                word_dot(wa.x, xa[0].x, xa[0].y, xa[0].z, xa[0].w, a0, a1, a2, a3);
-                word_dot(wa.y, xa[1].x, xa[1].y, xa[1].z, xa[1].w, a0, a1, a2, a3);
-                word_dot(wa.z, xa[2].x, xa[2].y, xa[2].z, xa[2].w, a0, a1, a2, a3);
-                word_dot(wa.w, xa[3].x, xa[3].y, xa[3].z, xa[3].w, a0, a1, a2, a3);
-                if (UPL == 2) {
-                    word_dot(wb.x, xb[0].x, xb[0].y, xb[0].z, xb[0].w, a0, a1, a2, a3);
-                    word_dot(wb.y, xb[1].x, xb[1].y, xb[1].z, xb[1].w, a0, a1, a2, a3);
-                    word_dot(wb.z, xb[2].x, xb[2].y, xb[2].z, xb[2].w, a0, a1, a2, a3);
-                    word_dot(wb.w, xb[3].x, xb[3].y, xb[3].z, xb[3].w, a0, a1, a2, a3);
-                }
-                vals[r] = combine4(a0, a1, a2, a3);
-            }
-            // the slot's words are in registers and used: refill it with row t + DEPTH
-            ln.fetch(seq.row(t + G1_DEPTH), slot);
-        }
+        for (int r = 0; r < R; ++r) vals[r] = combine4(a[r][0], a[r][1], a[r][2], a[r][3]);
+        // the batch's words are in registers and used: refill its slots with
+        // rows t+DEPTH .. t+DEPTH+R-1
+#pragma unroll
+        for (int r = 0; r < R; ++r) ln.fetch(seq.row(t + r + G1_DEPTH), (t + r) % G1_DEPTH);
         int which;
         const int tot = team_reduce<32, R>(vals, lane, which);
         const int i = b * R + which;
         if (lane == which * (32 / R) && i < seq.nrows) {
-            if (q.nslice == 1)
-                g1_store(g, q, r0 + i, tot - rowsum, f);
+            if (!sliced)
+                g1_store(mode, y, r0 + i, tot - rowsum, f);
             else
-                atomicAdd(const_cast<int*>(&sh.part[q.part_off + i]), tot);
+                atomicAdd(part + i, tot);
         }
     }
     cp_async_wait<0>();  // no copy of this lane is in flight past here
@@ -294,16 +315,18 @@ __global__ void __launch_bounds__(G1_THREADS, 2) gemv1_kernel(const __grid_const
     const int cta = blockIdx.x, ncta = gridDim.x;
 
     const int pi = g.wp[warp];
-    const G1Prob& q = g.prob[pi];
-    int r0, n;
-    g1_rows(q, cta, ncta, r0, n);
-    const int u0 = g.ws[warp] * q.slice_w;
-    const int width = min(q.slice_w, (q.K >> 6) - u0);  // 16-byte groups of this slice
-    const RowSeq seq = {g.wj[warp], g.wn[warp], g.wr[warp], n};
+    int r0, n, u0, width;
     Lane ln;
-    ln.wslice = reinterpret_cast<const unsigned char*>(q.W_p) + (size_t)r0 * q.rb + 16 * u0;
+    {
+        const G1Prob& qp = g.prob[pi];  // read once, before the shared copy exists
+        g1_rows(qp, cta, ncta, r0, n);
+        u0 = g.ws[warp] * qp.slice_w;
+        width = min(qp.slice_w, (qp.K >> 6) - u0);  // 16-byte groups of this slice
+        ln.wslice = reinterpret_cast<const unsigned char*>(qp.W_p) + (size_t)r0 * qp.rb + 16 * u0;
+        ln.rb = qp.rb;
+    }
+    const RowSeq seq = {g.wj[warp], g.wn[warp], g.wr[warp], n};
     ln.ring = smem + g.ring_off + (size_t)warp * G1_DEPTH * G1_SLOT;
-    ln.rb = q.rb;
     ln.lane = lane;
     ln.ha = lane < width;
     ln.hb = lane + 32 < width;
@@ -312,6 +335,12 @@ __global__ void __launch_bounds__(G1_THREADS, 2) gemv1_kernel(const __grid_const
     // is waited for.
 #pragma unroll
     for (int d = 0; d < G1_DEPTH; ++d) ln.fetch(seq.row(d), d);
+    {  // the descriptors to shared memory, one 4-byte word per thread
+        constexpr int WORDS = (int)(sizeof(G1Prob) / 4) * G1_MAX_PROBS;
+        static_assert(WORDS <= G1_THREADS, "descriptor copy: one word per thread");
+        if (threadIdx.x < WORDS)
+            reinterpret_cast<int*>(sh.prob)[threadIdx.x] = reinterpret_cast<const int*>(g.prob)[threadIdx.x];
+    }
     if (threadIdx.x < G1_MAX_PROBS) {
         const int p = threadIdx.x;
         sh.rowsum[p] = 0;
@@ -322,41 +351,50 @@ __global__ void __launch_bounds__(G1_THREADS, 2) gemv1_kernel(const __grid_const
     pdl_wait();
     g1_stage<XM>(g, sh, smem);
 
+    const G1Prob& q = sh.prob[pi];
+    const int mode = g.mode;
+    // (R = 4 with two groups per lane would not fit 64 registers; the plan
+    // never chooses it)
     if (seq.R == 4)
-        width > 32 ? g1_loop<4, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<4, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+        g1_loop<4, 1>(mode, q, sh, smem, pi, u0, seq, r0, ln);
     else if (seq.R == 2)
-        width > 32 ? g1_loop<2, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<2, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+        width > 32 ? g1_loop<2, 2>(mode, q, sh, smem, pi, u0, seq, r0, ln)
+                   : g1_loop<2, 1>(mode, q, sh, smem, pi, u0, seq, r0, ln);
     else
-        width > 32 ? g1_loop<1, 2>(g, q, sh, smem, pi, u0, seq, r0, ln) : g1_loop<1, 1>(g, q, sh, smem, pi, u0, seq, r0, ln);
+        width > 32 ? g1_loop<1, 2>(mode, q, sh, smem, pi, u0, seq, r0, ln)
+                   : g1_loop<1, 1>(mode, q, sh, smem, pi, u0, seq, r0, ln);
 
     if (g.sliced) {  // every slice of every row is in: finish the sliced rows
         __syncthreads();
         for (int p = 0; p < g.count; ++p) {
-            const G1Prob& qq = g.prob[p];
+            const G1Prob& qq = sh.prob[p];
             if (qq.nslice == 1) continue;
             int rr0, nn;
             g1_rows(qq, cta, ncta, rr0, nn);
             const float f = sh.fscale[p];
             const int rowsum = sh.rowsum[p];
-            for (int i = threadIdx.x; i < nn; i += G1_THREADS)
-                g1_store(g, qq, rr0 + i, sh.part[qq.part_off + i] - rowsum, f);
+            void* const y = qq.y;
+            const int* const part = sh.part + qq.part_off;
+            for (int i = threadIdx.x; i < nn; i += G1_THREADS) g1_store(mode, y, rr0 + i, part[i] - rowsum, f);
         }
     }
 }
 
 // ------------------------------------------------------------------- host
 
-// Estimated issue slots of one warp of a (problem, slice) group of n warps
-// working on `rows` rows with `upl` groups per lane, and the batch size that
-// minimises it.
+// Estimated cycles of one warp of a (problem, slice) group of n warps
+// working on `rows` rows with `upl` groups per lane, and the batch size R
+// that minimises it.  A batch costs a fixed latency (shared-memory loads,
+// shuffle reduction, dependent arithmetic) plus its issue slots, so larger
+// batches hide more latency until the rows run out.
 int g1_cost(int rows, int upl, int n, int& best_r) {
     int best = 1 << 30;
     best_r = 1;
     for (int R : {4, 2, 1}) {
+        if (R * upl > 4) continue;  // registers: at most four 16-byte groups of a batch per lane
         const int batches = (rows + R - 1) / R;
-        const int per_warp = (batches + n - 1) / n * R;
-        const int red = R == 1 ? 10 : R == 2 ? 5 : 3;  // shuffle-reduction steps per row
-        const int c = per_warp * (upl * 35 + 6 + red);
+        const int per_warp = (batches + n - 1) / n;
+        const int c = per_warp * (300 + R * (upl * 35 + 10));
         if (c < best) {
             best = c;
             best_r = R;

@@ -72,7 +72,7 @@ cudaError_t launch_gemv1(const GemvProblem* probs, int count, int x_dtype, YMode
 
 // api.cu: true once after bitlinear_test_expire_next_wait(1) (test hook of
 // the bounded waits; consumed by the next launch of the general small-M
-// decode kernel's batched form)
+// decode kernel)
 bool take_wait_expiry_request();
 
 // k_decode_tc.cu  (M <= 16, tcgen05 int8 tensor cores)

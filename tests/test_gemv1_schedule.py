@@ -37,10 +37,11 @@ HDR = ((3 * MAX_PROBS * 4 + WARPS * MAX_PROBS * 4 + PART_MAX * 4 + 3) // 4 * 4 +
 def cost(rows, upl, n):
     best, best_r = 1 << 30, 1
     for R in (4, 2, 1):
+        if R * upl > 4:
+            continue
         batches = (rows + R - 1) // R
-        per_warp = (batches + n - 1) // n * R
-        red = 10 if R == 1 else 5 if R == 2 else 3
-        c = per_warp * (upl * 35 + 6 + red)
+        per_warp = (batches + n - 1) // n
+        c = per_warp * (300 + R * (upl * 35 + 10))
         if c < best:
             best, best_r = c, R
     return best, best_r
@@ -135,6 +136,7 @@ def check_plan(pl):
             width = min(q["slice_w"], U - u0)
             assert width > 0
             upl = 2 if width > 32 else 1
+            assert R * upl <= 4
             ring = pl["ring_off"] + w * DEPTH * SLOT
 
             def row(t):
@@ -160,14 +162,15 @@ def check_plan(pl):
             t = 0
             b = j
             while b < batches:
+                # wait_group(DEPTH - R): rows t .. t+R-1 have landed
+                assert R <= DEPTH
+                assert len(committed) - (t + R) <= DEPTH - R
                 for r in range(R):
-                    # wait_group(DEPTH - 1): groups 0 .. t have landed
-                    assert len(committed) - (t + 1) <= DEPTH - 1
-                    slot = t % DEPTH
-                    i = row(t)
-                    assert slot_row[slot] == i                       # the slot holds row t
+                    slot = (t + r) % DEPTH
+                    i = row(t + r)
+                    assert slot_row[slot] == i                       # the slot holds row t + r
+                    assert (i == b * R + r) if b * R + r < nrows else (i == -1)
                     if i >= 0:
-                        assert (j + (t // R) * n) * R + t % R == b * R + r
                         for lane in range(32):
                             for u in groups(lane):
                                 dst = ring + slot * SLOT + 16 * (u - u0)
@@ -180,9 +183,10 @@ def check_plan(pl):
                         if q["nslice"] > 1:
                             assert q["part_off"] + i < PART_MAX
                         assert r0 + i < q["N"]
-                    slot_row[slot] = row(t + DEPTH)
-                    committed.append(row(t + DEPTH))
-                    t += 1
+                for r in range(R):                                   # refills after the batch
+                    slot_row[(t + r) % DEPTH] = row(t + r + DEPTH)
+                    committed.append(row(t + r + DEPTH))
+                t += R
                 b += n
         for p, q in enumerate(P):
             r0, nrows = rows_of(q, cta, grid)
