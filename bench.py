@@ -46,6 +46,37 @@ METRIC = "BitLinear W1.58A8 GEMV GB/s (frac of HBM peak); prefill GEMM int8 TOPS
 WORKLOAD = workloads.W2
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : bf16 tensor ratio
+
+# Compute-side bounds of the small-batch paths, from rates measured on B200
+# with single-SM probes: a tcgen05.mma kind::i8 of 128 x N x 32 takes ~186
+# cycles for every N <= 256; dp4a alone issues 64 lanes per cycle per SM, and
+# an even mix of dp4a and LOP3 85.  At the nominal maximum SM clock.
+MMA_CYCLES = 186
+DP4A_LANES_PER_CLK = 64
+MIXED_LANES_PER_CLK = 85
+NOMINAL_SM_HZ = 1.965e9
+
+
+def small_batch_bound(M, K, N, nbytes, hbm_gbs, sms):
+    """Lower bounds (us) of one small-batch call on the path it takes: HBM
+    time of its algorithmic bytes, and the compute time of the path's own
+    instruction stream spread evenly over the SMs -- dp4a + mask per 4 trits
+    on CUDA cores (M <= 4), 128 weight rows x 32 k per MMA for the swap-AB
+    kernel (M <= 16), 128 tokens x 256 weight rows x 32 k per MMA for the
+    GEMM.  The bound is the larger."""
+    hbm_us = nbytes / (hbm_gbs * 1e3)
+    if M <= 4:
+        dp4a, lop3 = N * K / 16 * 4 * M, N * K / 16 * 4
+        clk = max(dp4a / DP4A_LANES_PER_CLK, (dp4a + lop3) / MIXED_LANES_PER_CLK) / sms
+        comp_us, kind = clk / NOMINAL_SM_HZ * 1e6, "alu (dp4a + mask)"
+    elif M <= 16:
+        mmas = N * K / (128 * 32)
+        comp_us, kind = mmas / sms * MMA_CYCLES / NOMINAL_SM_HZ * 1e6, "tensor (swap-AB, 128 rows x 32 k per MMA)"
+    else:
+        mmas = -(-M // 128) * -(-N // 256) * K / 32
+        comp_us, kind = mmas / sms * MMA_CYCLES / NOMINAL_SM_HZ * 1e6, "tensor (GEMM, 128 x 256 x 32 per MMA)"
+    return {"hbm_us": hbm_us, "compute_us": comp_us, "compute": kind, "bound_us": max(hbm_us, comp_us),
+            "bound": "hbm" if hbm_us >= comp_us else kind.split()[0]}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_decode_m1_traffic.json")
 
 
@@ -63,13 +94,13 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of what defines the decode GEMV's device code: its source, the two
+    """Hash of what defines the decode GEMV's device code: its source, the
     device headers it includes, and the output-mode enum it reads (the rest of
     kernels.cuh declares host launchers)."""
     import re
     csrc = os.path.join(ROOT, "ternary_weight_linear_forward_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("k_gemv.cu", "act_inl.cuh", "common.cuh"):
+    for name in ("k_gemv.cu", "gemv_inl.cuh", "act_inl.cuh", "common.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     with open(os.path.join(csrc, "kernels.cuh")) as f:
@@ -326,6 +357,24 @@ def reference_arm(args):
 # our arm
 # ---------------------------------------------------------------------------
 
+class PartRanges:
+    """NVTX push/pop ranges around the parts of the run (decode, e2e, prefill,
+    small, ...), so that a profiler can select the launches of one part, e.g.
+    ``ncu --nvtx --nvtx-include "small/" ...``.  Calling it with a name closes
+    the open range and opens the named one; with None it only closes."""
+
+    def __init__(self):
+        self.open = False
+
+    def __call__(self, name):
+        import torch
+        if self.open:
+            torch.cuda.nvtx.range_pop()
+        self.open = name is not None
+        if name is not None:
+            torch.cuda.nvtx.range_push(name)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -438,6 +487,8 @@ def main():
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / 1e3
 
+    part = PartRanges()
+    part("decode")
     # SM clocks are sampled over the whole measured part of the run (the timed
     # decode region alone is far shorter than one sampling period)
     clk = ClockSampler(local).__enter__()
@@ -475,6 +526,7 @@ def main():
                 "bytes_per_launch": step_bytes(), "us_per_launch": t_step / args.steps * 1e6,
                 "alone_per_shape": per_shape}
 
+    part("e2e")
     # ---- end to end through the public API with pinned host buffers ----
     # The step's inputs (both projections' x) sit in one pinned host buffer and
     # its outputs in one device / one pinned host buffer, so a step is one H2D
@@ -603,6 +655,7 @@ def main():
                      "path": "the same three operations issued from the host every step on one stream, "
                              "no graph, no overlap"}}
 
+    part("prefill")
     # ---- prefill GEMM (M = 2048): int8 tensor-core TOPS ----
     prefill = None
     if "prefill" in sections:
@@ -637,6 +690,7 @@ def main():
         prefill["int8_peak_source"] = (f"{peak_kind} bf16_tflops {peaks['bf16_tflops']} x nominal int8/bf16 ratio "
                                        f"{INT8_OVER_BF16}")
 
+    part("small")
     # ---- small-batch decode (M = 4, 16, 64; K = 4096; N = 4096, 11008) ----
     small = None
     if "small" in sections:
@@ -663,11 +717,16 @@ def main():
             g.replay()
             t = timed_run([g])
             gbs = s.algorithmic_bytes * reps / t / 1e9
-            small[s.name] = {"us_per_call": t / reps * 1e6, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+            us = t / reps * 1e6
+            rl = small_batch_bound(s.M, s.K, s.N, s.algorithmic_bytes, peaks["hbm_gbs"], props.multi_processor_count)
+            rl["frac_of_bound"] = rl["bound_us"] / us
+            small[s.name] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                             "roofline": rl,
                              "path": "CUDA-core GEMV" if s.M <= 4 else
                                      ("tcgen05 swap-AB decode" if s.M <= 16 else "tcgen05 GEMM")}
             del g, W_ps, W_p0, x, y, ws
 
+    part("block")
     # ---- decoder block at batch-1 decode (hidden 2560, intermediate 6912) ----
     block = None
     if "block" in sections:
@@ -695,6 +754,7 @@ def main():
                  "copies": nblk}
         del g, blocks
 
+    part("binary")
     # ---- 1-bit weights (Sign(W - mean W)): decode GEMV and prefill GEMM ----
     binary = None
     if "binary" in sections:
@@ -750,6 +810,7 @@ def main():
                                            "path": "tcgen05 GEMM, 1-bit unpack"}
             del g, W_p, x_q, y, ws
 
+    part("grouped")
     # ---- group quantisation along K (G = 4): decode M = 1 on the FFN shapes ----
     grouped = None
     if "grouped" in sections:
@@ -784,6 +845,7 @@ def main():
                                                       "written, + the ordered sum of the terms"}
             del g, W_ps, W_p0, xb, y, ws
 
+    part("glu")
     # ---- MatMul-free GLU channel mixer (hidden 2560, intermediate 6912) ----
     glu = None
     if "glu" in sections:
@@ -827,6 +889,7 @@ def main():
         del base
 
     clk.__exit__()
+    part(None)
     clocks = clk.summary()
     clocks["window"] = "whole GPU part of the run (decode warm-up and timed steps, roofline, e2e and sections)"
 

@@ -85,10 +85,11 @@ struct DtcHdr {
     uint64_t drain;                  // every MMA issued by this CTA finished
     uint32_t tmem_base;
     int abort_flag;
-    int rowsum[DTC_MAX_M];
+    int rowsum[DTC_MAX_M];           // sum of x_hat per token (zeroed at CTA start)
+    int amax[DTC_MAX_M];             // max |x| per token as float bits (zeroed at CTA start)
+    float gam[DTC_MAX_M];
+    float xscale[DTC_MAX_M];         // 127 / gamma
     float fscale[DTC_MAX_M];
-    unsigned red_u[DTC_UNPACK_WARPS][DTC_MAX_M];
-    int red_i[DTC_UNPACK_WARPS][DTC_MAX_M];
 };
 static_assert(sizeof(DtcHdr) <= DTC_HDR, "decode header too large");
 
@@ -190,113 +191,126 @@ __device__ __forceinline__ int produce(const DtcParams& p, DtcHdr& h, unsigned c
     return u1;
 }
 
+// Total of v over the lanes of the warp that hold the same key (maximum if
+// MAX, else sum), for keys that are non-decreasing in lane order, so that
+// equal keys form contiguous runs.  The first lane of every run returns true
+// and holds the run's total.
+template <bool MAX>
+__device__ __forceinline__ bool run_total(int key, int& v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_down_sync(0xffffffffu, v, off);
+        const int ko = __shfl_down_sync(0xffffffffu, key, off);
+        if (lane + off < 32 && ko == key) v = MAX ? max(v, o) : v + o;
+    }
+    const int kp = __shfl_up_sync(0xffffffffu, key, 1);
+    return lane == 0 || kp != key;
+}
+
 // Build B (x_hat in S column blocks of MP tokens x G groups, zero outside each
 // slice, each group and for padded tokens), the per-token row sums of x_hat
 // and the rescale factors.  Runs on the unpack warps after the wait for the
-// preceding kernel.
+// preceding kernel.  The (token, chunk) pairs of each pass are dealt to the
+// threads as one flat range and loaded NB per thread at a time, so that the
+// loads of all tokens are in flight together; per-token totals are reduced
+// over runs of lanes and added to shared memory with one atomic per run.
 template <int MP, int G, int XM>
 __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part, unsigned char* Bs) {
+    constexpr int NT = DTC_UNPACK_THREADS;
+    constexpr int NB = XM == X_QUANTISED ? 4 : 1;  // <= 16 registers of chunks in flight
     const int ctid = threadIdx.x;
-    const int lane = ctid & 31, warp = ctid >> 5;
-    const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : 4);
-    float s[MP], gam[MP];
-#pragma unroll
-    for (int m = 0; m < MP; ++m) s[m] = gam[m] = 0.0f;
+    const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : XM == X_F32 ? 4 : 1);
+    const char* xbase = XM == X_QUANTISED ? reinterpret_cast<const char*>(p.x_q) : reinterpret_cast<const char*>(p.x);
     if (XM != X_QUANTISED) {
         // pass 1: max |x| of every token (exact, order-free)
+        const int GK = p.K / 16;
+        const int total = p.M * GK;
+        for (int e0 = 0; e0 < total; e0 += NB * NT) {
+            XChunk<XM> c[NB];
 #pragma unroll
-        for (int m = 0; m < MP; ++m) {
-            unsigned a = 0u;
-            if (m < p.M) {
-                const char* xr = reinterpret_cast<const char*>(p.x) + (size_t)m * xrow;
-                for (int g = ctid; g < p.K / 16; g += DTC_UNPACK_THREADS) {
-                    float v[16];
-                    load16<XM>(xr, g, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) a = max(a, __float_as_uint(fabsf(v[i])));
-                }
+            for (int b = 0; b < NB; ++b) {
+                const int e = e0 + b * NT + ctid;
+                if (e < total) ld_chunk<XM>(xbase + (size_t)(e / GK) * xrow, e % GK, c[b]);
             }
-            a = __reduce_max_sync(0xffffffffu, a);
-            if (lane == 0) h.red_u[warp][m] = a;
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int e = e0 + b * NT + ctid;
+                const int key = e < total ? e / GK : MP;
+                int a = e < total ? (int)chunk_absmax<XM>(c[b], 0u) : 0;
+                if (run_total<true>(key, a) && key < MP) atomicMax(&h.amax[key], a);
+            }
         }
         unpack_sync();
-#pragma unroll
-        for (int m = 0; m < MP; ++m) {
-            unsigned a = 0u;
-            for (int w = 0; w < DTC_UNPACK_WARPS; ++w) a = max(a, h.red_u[w][m]);
-            gam[m] = fmaxf(__uint_as_float(a), 1e-5f);
-            s[m] = __fdiv_rn(127.0f, gam[m]);
+        if (ctid < MP) {
+            const float g = fmaxf(__int_as_float(h.amax[ctid]), 1e-5f);
+            h.gam[ctid] = g;
+            h.xscale[ctid] = __fdiv_rn(127.0f, g);
         }
+        unpack_sync();
     }
-    for (int i = ctid; i < p.Rt * MP; i += DTC_UNPACK_THREADS) part[i] = 0;
+    for (int i = ctid; i < p.Rt * MP; i += NT) part[i] = 0;
     // pass 2: 16-byte chunks of x_hat into B.  Row j = (q * MP + m) * G + s of
     // K-block kb holds group s of x_hat[m, q * Lfull + 128 kb ...]; chunk c of
     // a row sits at c ^ (j % 8).
     const uint32_t bs = smem_u32(Bs);
     const int KC = p.T * (DTC_STAGE_K / 16);  // chunks per B row
-    int rs[MP];
+    const int per_tok = p.S * KC;
+    const int total = MP * per_tok;
+    for (int e0 = 0; e0 < total; e0 += NB * NT) {
+        XChunk<XM> c[NB];
 #pragma unroll
-    for (int m = 0; m < MP; ++m) {
-        rs[m] = 0;
-        for (int idx = ctid; idx < p.S * KC; idx += DTC_UNPACK_THREADS) {
-            const int q = idx / KC, kc = idx - q * KC;
-            const int kl = kc * 16;
-            const int ls = min(p.Lfull, p.K - q * p.Lfull);
-            int4 v = make_int4(0, 0, 0, 0);
-            if (m < p.M && kl < ls) {
-                const int k = q * p.Lfull + kl;
-                if (XM == X_QUANTISED) {
-                    v = __ldg(reinterpret_cast<const int4*>(p.x_q + (size_t)m * p.K + k));
-                } else {
-                    const char* xr = reinterpret_cast<const char*>(p.x) + (size_t)m * xrow;
-                    float f[16];
-                    load16<XM>(xr, k / 16, f);
-                    v.x = (int)pack4(q8(f[0], s[m]), q8(f[1], s[m]), q8(f[2], s[m]), q8(f[3], s[m]));
-                    v.y = (int)pack4(q8(f[4], s[m]), q8(f[5], s[m]), q8(f[6], s[m]), q8(f[7], s[m]));
-                    v.z = (int)pack4(q8(f[8], s[m]), q8(f[9], s[m]), q8(f[10], s[m]), q8(f[11], s[m]));
-                    v.w = (int)pack4(q8(f[12], s[m]), q8(f[13], s[m]), q8(f[14], s[m]), q8(f[15], s[m]));
-                }
-                rs[m] += bytesum_s8(v.x) + bytesum_s8(v.y) + bytesum_s8(v.z) + bytesum_s8(v.w);
-            }
-            const uint32_t kb_off = (uint32_t)((kc >> 3) * p.brow * 128);
-            if (G == 1) {
-                const int j = q * MP + m;
-                sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), v);
-            } else {
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int j = (q * MP + m) * 4 + g;
-                    const int4 vg = make_int4(g == 0 ? v.x : 0, g == 1 ? v.y : 0, g == 2 ? v.z : 0, g == 3 ? v.w : 0);
-                    sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), vg);
-                }
+        for (int b = 0; b < NB; ++b) {
+            const int e = e0 + b * NT + ctid;
+            if (e < total) {
+                const int m = e / per_tok, r = e - m * per_tok;
+                const int q = r / KC, kl = (r - q * KC) * 16;
+                if (m < p.M && kl < min(p.Lfull, p.K - q * p.Lfull))
+                    ld_chunk<XM>(xbase + (size_t)m * xrow, (q * p.Lfull + kl) / 16, c[b]);
             }
         }
-    }
 #pragma unroll
-    for (int m = 0; m < MP; ++m) {
-        int v = rs[m];
+        for (int b = 0; b < NB; ++b) {
+            const int e = e0 + b * NT + ctid;
+            int key = MP, rs = 0;
+            if (e < total) {
+                const int m = e / per_tok, r = e - m * per_tok;
+                const int q = r / KC, kc = r - q * KC;
+                const int kl = kc * 16;
+                int4 v = make_int4(0, 0, 0, 0);
+                if (m < p.M && kl < min(p.Lfull, p.K - q * p.Lfull)) {
+                    v = chunk_codes<XM>(c[b], XM == X_QUANTISED ? 0.0f : h.xscale[m]);
+                    rs = bytesum_s8(v.x) + bytesum_s8(v.y) + bytesum_s8(v.z) + bytesum_s8(v.w);
+                }
+                key = m;
+                const uint32_t kb_off = (uint32_t)((kc >> 3) * p.brow * 128);
+                if (G == 1) {
+                    const int j = q * MP + m;
+                    sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), v);
+                } else {
 #pragma unroll
-        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) h.red_i[warp][m] = v;
+                    for (int g = 0; g < 4; ++g) {
+                        const int j = (q * MP + m) * 4 + g;
+                        const int4 vg =
+                            make_int4(g == 0 ? v.x : 0, g == 1 ? v.y : 0, g == 2 ? v.z : 0, g == 3 ? v.w : 0);
+                        sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), vg);
+                    }
+                }
+            }
+            if (run_total<false>(key, rs) && key < MP && rs != 0) atomicAdd(&h.rowsum[key], rs);
+        }
     }
+    fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
     unpack_sync();
     if (ctid < MP) {
         const int m = ctid;
-        int t = 0;
-        for (int w = 0; w < DTC_UNPACK_WARPS; ++w) t += h.red_i[w][m];
-        h.rowsum[m] = t;
         float f = 0.0f;
         if (p.mode != Y_ACC && m < p.M) {
-            float g = 0.0f;
-#pragma unroll
-            for (int i = 0; i < MP; ++i)
-                if (i == m) g = gam[i];
-            if (XM == X_QUANTISED) g = __ldg(p.gamma + m);
+            const float g = XM == X_QUANTISED ? __ldg(p.gamma + m) : h.gam[m];
             f = __fdiv_rn(__fmul_rn(__ldg(p.beta), g), 127.0f);
         }
         h.fscale[m] = f;
     }
-    fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
     unpack_sync();
     if (ctid == 0) mbar_arrive(&h.b_ready);
 }
@@ -470,6 +484,7 @@ __device__ __forceinline__ void dtc_body(const DtcParams& p, int cta) {
         mbar_init(&h.d_empty, 4);
         mbar_init(&h.drain, 1);
         h.abort_flag = 0;
+        for (int m = 0; m < DTC_MAX_M; ++m) h.rowsum[m] = h.amax[m] = 0;
         fence_mbar_init();
         prefetch_tmap(&p.tmap);
         produce(p, h, ring, r0, 0, 1, pol);
@@ -543,27 +558,28 @@ int pow2_at_least(int v) {
 
 int round_up(int v, int a) { return (v + a - 1) / a * a; }
 
-// K slices and row tiles for M tokens (padded to mp) and R rows per CTA.
+// K slices and row tiles for M tokens (padded to mp) and R rows per CTA.  A
+// tile holds up to 128 / S rows, each split into S K-slices placed in
+// different TMEM subpartitions; every tile costs Lfull / 32 MMAs, whatever
+// the number of its rows, so the split with the fewest tiles x Lfull wins
+// (ties: fewer tiles).
 bool dtc_split(int mp, int K, int R, int& S, int& Lfull, int& ntiles, int& Rt) {
-    S = 1;
-    Lfull = 0;
-    ntiles = 1;
-    Rt = R;
-    if (R > 128) {
-        ntiles = (R + 127) / 128;
-        Rt = (R + ntiles - 1) / ntiles;
-        Lfull = round_up(K, DTC_STAGE_K);
-        return mp <= DTC_MAX_NMMA;
-    }
-    for (int s : {4, 2, 1}) {
-        if (R * s > 128 || s * mp > DTC_MAX_NMMA) continue;
+    long long best = -1;
+    for (int s : {1, 2, 4}) {
+        if (s * mp > DTC_MAX_NMMA) continue;
         const int lf = round_up((K + s - 1) / s, DTC_STAGE_K);
         if ((s - 1) * lf >= K) continue;  // every slice must hold data
-        S = s;
-        Lfull = lf;
-        return true;
+        const int nt = (R + 128 / s - 1) / (128 / s);
+        const long long cost = (long long)nt * lf;
+        if (best < 0 || cost < best) {
+            best = cost;
+            S = s;
+            Lfull = lf;
+            ntiles = nt;
+            Rt = (R + nt - 1) / nt;
+        }
     }
-    return false;
+    return best >= 0;
 }
 
 // Shape and shared-memory layout of one problem with G column groups for a

@@ -19,10 +19,11 @@
 //               packed weight tile (256 rows x 8 words) per K-block, no multicast;
 //   warp 1      TMEM allocation and the single-thread tcgen05.mma issuer
 //               (4 MMAs of K = 32 per K-block), tcgen05.commit to free stages;
-//   warps 2-5   unpack: packed word -> four registers of codes (w >> 2s) &
-//               0x03030303, i.e. 16 consecutive-k bytes, stored as one 16-byte
-//               chunk into the 128-byte-swizzled K-major operand layout;
-//   warps 6-9   epilogue: tcgen05.ld of the int32 accumulators (32 TMEM lanes
+//   warps 2-9   unpack (UNPACK_WARPS = 8): packed word -> four registers of
+//               codes (w >> 2s) & 0x03030303, i.e. 16 consecutive-k bytes,
+//               stored as one 16-byte chunk into the 128-byte-swizzled
+//               K-major operand layout;
+//   warps 10-13 epilogue: tcgen05.ld of the int32 accumulators (32 TMEM lanes
 //               per warp), rowsum correction, rescale, bf16/fp32 store.
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap
 // the main loop of tile t + 1.  Every mbarrier wait is bounded.

@@ -234,6 +234,7 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
     const int lane = ctid & 31, warp = ctid >> 5;
     constexpr int XC = XM == X_F32 ? (MT <= 2 ? 2 / MT : 0) : 4 / MT;  // <= 32 registers of cache
     constexpr int XCA = XC > 0 ? XC : 1;
+    constexpr int TB = XM == X_F32 ? (MT < 2 ? MT : 2) : MT;            // tokens loaded together past the cache
     const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : XM == X_F32 ? 4 : 1);
     const char* xbase = XM == X_QUANTISED ? reinterpret_cast<const char*>(p.x_q) : reinterpret_cast<const char*>(p.x);
     XChunk<XM> cache[MT][XCA];
@@ -250,21 +251,32 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
 #pragma unroll
     for (int m = 0; m < MT; ++m) s[m] = gam[m] = 0.0f;
     if (XM != X_QUANTISED) {
-        // pass 1: per-token absmax over the row (exact, order-free)
+        // pass 1: per-token absmax over the row (exact, order-free); chunks
+        // beyond the cache are loaded TB tokens at a time, so that their
+        // loads are in flight together
+        unsigned amax[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            unsigned a = 0u;
-            if (m < p.M) {
+            amax[m] = 0u;
 #pragma unroll
-                for (int i = 0; i < XC; ++i)
-                    if (ctid + i * cthreads < G) a = chunk_absmax<XM>(cache[m][i], a);
-                for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
-                    XChunk<XM> c;
-                    ld_chunk<XM>(xbase + (size_t)m * xrow, g, c);
-                    a = chunk_absmax<XM>(c, a);
-                }
+            for (int i = 0; i < XC; ++i)
+                if (m < p.M && ctid + i * cthreads < G) amax[m] = chunk_absmax<XM>(cache[m][i], amax[m]);
+        }
+#pragma unroll
+        for (int m0 = 0; m0 < MT; m0 += TB) {
+            for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
+                XChunk<XM> c[TB];
+#pragma unroll
+                for (int t = 0; t < TB; ++t)
+                    if (m0 + t < p.M) ld_chunk<XM>(xbase + (size_t)(m0 + t) * xrow, g, c[t]);
+#pragma unroll
+                for (int t = 0; t < TB; ++t)
+                    if (m0 + t < p.M) amax[m0 + t] = chunk_absmax<XM>(c[t], amax[m0 + t]);
             }
-            a = __reduce_max_sync(0xffffffffu, a);
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const unsigned a = __reduce_max_sync(0xffffffffu, amax[m]);
             if (lane == 0) sh.red_u[warp][m] = a;
         }
         consumer_sync(cthreads);
@@ -305,15 +317,24 @@ __device__ __forceinline__ void stage_activations(const GemvParams& p, Shared& s
                 dst[xq_slot<WB>(g)] = q;
             }
         }
+    }
+#pragma unroll
+    for (int m0 = 0; m0 < MT; m0 += TB) {
         for (int g = ctid + XC * cthreads; g < G; g += cthreads) {
-            int4 q = make_int4(0, 0, 0, 0);
-            if (m < p.M) {
-                XChunk<XM> c;
-                ld_chunk<XM>(xbase + (size_t)m * xrow, g, c);
-                q = chunk_codes<XM>(c, s[m]);
-                rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
+            XChunk<XM> c[TB];
+#pragma unroll
+            for (int t = 0; t < TB; ++t)
+                if (m0 + t < p.M) ld_chunk<XM>(xbase + (size_t)(m0 + t) * xrow, g, c[t]);
+#pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                const int m = m0 + t;
+                int4 q = make_int4(0, 0, 0, 0);
+                if (m < p.M) {
+                    q = chunk_codes<XM>(c[t], s[m]);
+                    rs[m] += bytesum_s8(q.x) + bytesum_s8(q.y) + bytesum_s8(q.z) + bytesum_s8(q.w);
+                }
+                xsm[(size_t)m * G + xq_slot<WB>(g)] = q;
             }
-            dst[xq_slot<WB>(g)] = q;
         }
     }
 #pragma unroll

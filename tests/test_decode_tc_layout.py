@@ -32,18 +32,19 @@ def pow2(v):
 
 
 def split(mp, K, R):
-    """Slices S (placed in different TMEM subpartitions) and row tiles."""
-    if R > 128:
-        ntiles = (R + 127) // 128
-        return dict(S=1, Lfull=ru(K, STAGE_K), ntiles=ntiles, Rt=(R + ntiles - 1) // ntiles), mp <= MAX_NMMA
-    for s in (4, 2, 1):
-        if R * s > 128 or s * mp > MAX_NMMA:
+    """Slices S (placed in different TMEM subpartitions) and row tiles: the
+    fewest tiles x slice length (MMAs per CTA), ties to fewer tiles."""
+    best = None
+    for s in (1, 2, 4):
+        if s * mp > MAX_NMMA:
             continue
         lf = ru((K + s - 1) // s, STAGE_K)
         if (s - 1) * lf >= K:
             continue
-        return dict(S=s, Lfull=lf, ntiles=1, Rt=R), True
-    return None, False
+        nt = (R + 128 // s - 1) // (128 // s)
+        if best is None or nt * lf < best[0]:
+            best = (nt * lf, dict(S=s, Lfull=lf, ntiles=nt, Rt=(R + nt - 1) // nt))
+    return (best[1], True) if best else (None, False)
 
 
 def layout(G, M, K, N, sms, budget):
@@ -86,6 +87,52 @@ def sw128(row, chunk):
     return (row // 8) * 1024 + (row % 8) * 128 + ((chunk ^ (row % 8)) << 4)
 
 
+NT, NB = 384, 4          # unpack threads; x_q chunks each thread loads at once
+
+
+def run_total(keys, vals, op):
+    """The warp's segmented reduction: five shuffle-down steps, each adding
+    (or taking the max of) the value `off` lanes down when that lane holds the
+    same key (a lane past the warp reads its own value).  Returns the values
+    and which lanes lead a run of equal keys."""
+    v = list(vals)
+    for off in (1, 2, 4, 8, 16):
+        o = [v[l + off] if l + off < 32 else v[l] for l in range(32)]
+        ko = [keys[l + off] if l + off < 32 else keys[l] for l in range(32)]
+        v = [op(v[l], o[l]) if (l + off < 32 and ko[l] == keys[l]) else v[l] for l in range(32)]
+    return v, [l == 0 or keys[l - 1] != keys[l] for l in range(32)]
+
+
+def flat_rowsum(x_q, M, K, mp, S, KC, Lfull):
+    """Row sums of x_hat as the staging pass forms them: (token, slice,
+    chunk) entries dealt to NT threads NB at a time, per-warp segmented sums,
+    one shared add per run leader."""
+    per_tok = S * KC
+    total = mp * per_tok
+    rows = [0] * mp
+    for e0 in range(0, total, NB * NT):
+        for b in range(NB):
+            for w in range(NT // 32):
+                keys, vals = [], []
+                for lane in range(32):
+                    e = e0 + b * NT + 32 * w + lane
+                    key, val = mp, 0
+                    if e < total:
+                        m, r = divmod(e, per_tok)
+                        q, kc = divmod(r, KC)
+                        kl = kc * 16
+                        key = m
+                        if m < M and kl < min(Lfull, K - q * Lfull):
+                            val = int(x_q[m, q * Lfull + kl:q * Lfull + kl + 16].astype(np.int64).sum())
+                    keys.append(key)
+                    vals.append(val)
+                tot, lead = run_total(keys, vals, lambda a, c: a + c)
+                for lane in range(32):
+                    if lead[lane] and keys[lane] < mp and tot[lane] != 0:
+                        rows[keys[lane]] += tot[lane]
+    return rows
+
+
 def emulate(p, Wbytes, x_q, rng):
     """acc [M, N] as the kernel computes it."""
     M, K, N, G, S, T, mp = p["M"], p["K"], p["N"], p["G"], p["S"], p["T"], p["mp"]
@@ -113,7 +160,7 @@ def emulate(p, Wbytes, x_q, rng):
                         vg[4 * g:4 * g + 4] = v[4 * g:4 * g + 4]
                     o = p["b_off"] + kb_off + j * 128 + (((kc & 7) ^ (j & 7)) << 4)
                     smem[o:o + 16] = vg.view(np.uint8)
-        rowsum = [int(x_q[m].astype(np.int64).sum()) if m < M else 0 for m in range(mp)]
+        rowsum = flat_rowsum(x_q, M, K, mp, S, KC, Lfull)
         part = np.zeros((Rt, mp), np.int64)
         u4 = 0
         for tile in range(p["ntiles"]):
@@ -203,6 +250,8 @@ CASES = [
     (1, 512, 2000, 4),
     (8, 1024, 9, 8),
     (1, 17 * 512, 65, 1),            # 17 stages through 4 ring slots
+    (16, 2048, 300, 4),              # 75 rows per CTA: 4 slices in 3 tiles
+    (2, 2048, 600, 4),               # 150 rows per CTA: 4 slices in 5 tiles
 ]
 
 
@@ -222,5 +271,37 @@ def test_emulated_cases_cover_the_kernel_shapes():
     assert {p["S"] for p in shapes} == {1, 2, 4}
     assert {p["G"] for p in shapes} == {1, 4}
     assert max(p["ntiles"] for p in shapes) > 1
+    assert any(p["ntiles"] > 1 and p["S"] > 1 for p in shapes)      # sliced tiles
     assert any(p["slots"] < p["ntiles"] * p["T"] for p in shapes)     # a recycled ring
     assert any(p["nmma"] > p["brow"] for p in shapes)                  # B read past its rows
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_segmented_warp_reduction(seed):
+    """Every run leader of the shuffle scan holds its run's sum and max, for
+    runs of every length from 1 to 32 and a trailing sentinel run."""
+    rng = np.random.default_rng(seed)
+    for _ in range(50):
+        lens, n = [], 0
+        while n < 32:
+            lens.append(int(min(32 - n, rng.integers(1, 33 if seed % 2 else 6))))
+            n += lens[-1]
+        keys = sum(([k] * l for k, l in enumerate(lens)), [])
+        vals = [int(v) for v in rng.integers(0, 1 << 20, 32)]
+        for op, ref in ((lambda a, c: a + c, sum), (max, max)):
+            tot, lead = run_total(keys, vals, op)
+            starts = np.cumsum([0] + lens[:-1])
+            assert [l for l in range(32) if lead[l]] == list(starts)
+            for k, (s0, l) in enumerate(zip(starts, lens)):
+                assert tot[s0] == ref(vals[s0:s0 + l])
+
+
+def test_flat_rowsum_matches_the_row_sums():
+    rng = np.random.default_rng(3)
+    for M, K, S in ((16, 4096, 4), (5, 1088, 2), (1, 640, 1), (9, 2048, 1)):
+        mp = pow2(M)
+        Lfull = ru(-(-K // S), STAGE_K)
+        T = Lfull // STAGE_K
+        x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        rows = flat_rowsum(x_q, M, K, mp, S, T * (STAGE_K // 16), Lfull)
+        assert rows == [int(x_q[m].astype(np.int64).sum()) if m < M else 0 for m in range(mp)]
