@@ -157,6 +157,12 @@ __device__ __forceinline__ void sts128(uint32_t addr, int4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void store_y(const DtcParams& p, int m, int n, int acc, float f) {
     const long long o = (long long)m * p.N + n;
     if (p.mode == Y_ACC) {
@@ -191,55 +197,44 @@ __device__ __forceinline__ int produce(const DtcParams& p, DtcHdr& h, unsigned c
     return u1;
 }
 
-// Total of v over the lanes of the warp that hold the same key (maximum if
-// MAX, else sum), for keys that are non-decreasing in lane order, so that
-// equal keys form contiguous runs.  The first lane of every run returns true
-// and holds the run's total.
-template <bool MAX>
-__device__ __forceinline__ bool run_total(int key, int& v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_down_sync(0xffffffffu, v, off);
-        const int ko = __shfl_down_sync(0xffffffffu, key, off);
-        if (lane + off < 32 && ko == key) v = MAX ? max(v, o) : v + o;
-    }
-    const int kp = __shfl_up_sync(0xffffffffu, key, 1);
-    return lane == 0 || kp != key;
-}
-
 // Build B (x_hat in S column blocks of MP tokens x G groups, zero outside each
 // slice, each group and for padded tokens), the per-token row sums of x_hat
 // and the rescale factors.  Runs on the unpack warps after the wait for the
-// preceding kernel.  The (token, chunk) pairs of each pass are dealt to the
-// threads as one flat range and loaded NB per thread at a time, so that the
-// loads of all tokens are in flight together; per-token totals are reduced
-// over runs of lanes and added to shared memory with one atomic per run.
+// preceding kernel.  Work is dealt by B row: row j = q * MP + m (slice q,
+// token m) goes to warp j % 12 and its KC = 32 T chunks to the lanes, so the
+// index arithmetic is shifts and masks and every row's total is one warp
+// reduction plus one shared-memory atomic.  Plain int8 x_hat is copied into
+// B by cp.async, all chunks in flight at once.
 template <int MP, int G, int XM>
 __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part, unsigned char* Bs) {
-    constexpr int NT = DTC_UNPACK_THREADS;
-    constexpr int NB = XM == X_QUANTISED ? 4 : 1;  // <= 16 registers of chunks in flight
-    const int ctid = threadIdx.x;
+    constexpr int NW = DTC_UNPACK_WARPS;
+    const int ctid = threadIdx.x, lane = ctid & 31, warp = ctid >> 5;
     const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : XM == X_F32 ? 4 : 1);
     const char* xbase = XM == X_QUANTISED ? reinterpret_cast<const char*>(p.x_q) : reinterpret_cast<const char*>(p.x);
+    const int rows = p.S * MP;                // B rows per K-block before the G expansion
+    const int KC = p.T * (DTC_STAGE_K / 16);  // chunks per B row
+    const uint32_t bs = smem_u32(Bs);
+    // chunk kc of row j: byte offset in B (G = 1), and whether it holds data
+    auto slot = [&](int j, int kc) -> uint32_t {
+        return (uint32_t)((kc >> 3) * p.brow * 128 + j * 128 + (((kc & 7) ^ (j & 7)) << 4));
+    };
     if (XM != X_QUANTISED) {
         // pass 1: max |x| of every token (exact, order-free)
-        const int GK = p.K / 16;
-        const int total = p.M * GK;
-        for (int e0 = 0; e0 < total; e0 += NB * NT) {
-            XChunk<XM> c[NB];
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int e = e0 + b * NT + ctid;
-                if (e < total) ld_chunk<XM>(xbase + (size_t)(e / GK) * xrow, e % GK, c[b]);
+        for (int j = warp; j < rows; j += NW) {
+            const int q = j / MP, m = j % MP;
+            unsigned a = 0u;
+            if (m < p.M) {
+                const int ls = min(p.Lfull, p.K - q * p.Lfull);
+                const char* xr = xbase + (size_t)m * xrow;
+#pragma unroll 2
+                for (int kc = lane; kc * 16 < ls; kc += 32) {
+                    XChunk<XM> c;
+                    ld_chunk<XM>(xr, (q * p.Lfull + kc * 16) / 16, c);
+                    a = chunk_absmax<XM>(c, a);
+                }
             }
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int e = e0 + b * NT + ctid;
-                const int key = e < total ? e / GK : MP;
-                int a = e < total ? (int)chunk_absmax<XM>(c[b], 0u) : 0;
-                if (run_total<true>(key, a) && key < MP) atomicMax(&h.amax[key], a);
-            }
+            a = __reduce_max_sync(0xffffffffu, a);
+            if (lane == 0 && a != 0u) atomicMax(&h.amax[m], (int)a);
         }
         unpack_sync();
         if (ctid < MP) {
@@ -249,55 +244,62 @@ __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part
         }
         unpack_sync();
     }
-    for (int i = ctid; i < p.Rt * MP; i += NT) part[i] = 0;
-    // pass 2: 16-byte chunks of x_hat into B.  Row j = (q * MP + m) * G + s of
+    for (int i = ctid; i < p.Rt * MP; i += DTC_UNPACK_THREADS) part[i] = 0;
+    // pass 2: 16-byte chunks of x_hat into B.  Row (q * MP + m) * G + s of
     // K-block kb holds group s of x_hat[m, q * Lfull + 128 kb ...]; chunk c of
-    // a row sits at c ^ (j % 8).
-    const uint32_t bs = smem_u32(Bs);
-    const int KC = p.T * (DTC_STAGE_K / 16);  // chunks per B row
-    const int per_tok = p.S * KC;
-    const int total = MP * per_tok;
-    for (int e0 = 0; e0 < total; e0 += NB * NT) {
-        XChunk<XM> c[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int e = e0 + b * NT + ctid;
-            if (e < total) {
-                const int m = e / per_tok, r = e - m * per_tok;
-                const int q = r / KC, kl = (r - q * KC) * 16;
-                if (m < p.M && kl < min(p.Lfull, p.K - q * p.Lfull))
-                    ld_chunk<XM>(xbase + (size_t)m * xrow, (q * p.Lfull + kl) / 16, c[b]);
+    // a row sits at c ^ (row % 8).
+    if constexpr (XM == X_QUANTISED && G == 1) {
+        for (int j = warp; j < rows; j += NW) {
+            const int q = j / MP, m = j % MP;
+            const int ls = m < p.M ? min(p.Lfull, p.K - q * p.Lfull) : 0;
+            const int8_t* xr = p.x_q + (size_t)m * p.K + q * p.Lfull;
+            for (int kc = lane; kc < KC; kc += 32) {
+                if (kc * 16 < ls)
+                    cp_async16(bs + slot(j, kc), xr + kc * 16);
+                else
+                    sts128(bs + slot(j, kc), make_int4(0, 0, 0, 0));
             }
         }
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int e = e0 + b * NT + ctid;
-            int key = MP, rs = 0;
-            if (e < total) {
-                const int m = e / per_tok, r = e - m * per_tok;
-                const int q = r / KC, kc = r - q * KC;
-                const int kl = kc * 16;
+        cp_async_wait_all();
+        for (int j = warp; j < rows; j += NW) {
+            const int m = j % MP;
+            int rs = 0;
+            for (int kc = lane; kc < KC; kc += 32) {
+                const uint4 v = lds128(bs + slot(j, kc));
+                rs += bytesum_s8((int)v.x) + bytesum_s8((int)v.y) + bytesum_s8((int)v.z) + bytesum_s8((int)v.w);
+            }
+            rs = __reduce_add_sync(0xffffffffu, rs);
+            if (lane == 0 && rs != 0) atomicAdd(&h.rowsum[m], rs);
+        }
+    } else {
+        for (int j = warp; j < rows; j += NW) {
+            const int q = j / MP, m = j % MP;
+            const int ls = m < p.M ? min(p.Lfull, p.K - q * p.Lfull) : 0;
+            const char* xr = xbase + (size_t)m * xrow;
+            const float sc = XM == X_QUANTISED ? 0.0f : h.xscale[m];
+            int rs = 0;
+#pragma unroll 2
+            for (int kc = lane; kc < KC; kc += 32) {
                 int4 v = make_int4(0, 0, 0, 0);
-                if (m < p.M && kl < min(p.Lfull, p.K - q * p.Lfull)) {
-                    v = chunk_codes<XM>(c[b], XM == X_QUANTISED ? 0.0f : h.xscale[m]);
-                    rs = bytesum_s8(v.x) + bytesum_s8(v.y) + bytesum_s8(v.z) + bytesum_s8(v.w);
+                if (kc * 16 < ls) {
+                    XChunk<XM> c;
+                    ld_chunk<XM>(xr, (q * p.Lfull + kc * 16) / 16, c);
+                    v = chunk_codes<XM>(c, sc);
+                    rs += bytesum_s8(v.x) + bytesum_s8(v.y) + bytesum_s8(v.z) + bytesum_s8(v.w);
                 }
-                key = m;
-                const uint32_t kb_off = (uint32_t)((kc >> 3) * p.brow * 128);
                 if (G == 1) {
-                    const int j = q * MP + m;
-                    sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), v);
+                    sts128(bs + slot(j, kc), v);
                 } else {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        const int j = (q * MP + m) * 4 + g;
                         const int4 vg =
                             make_int4(g == 0 ? v.x : 0, g == 1 ? v.y : 0, g == 2 ? v.z : 0, g == 3 ? v.w : 0);
-                        sts128(bs + kb_off + (uint32_t)(j * 128 + (((kc & 7) ^ (j & 7)) << 4)), vg);
+                        sts128(bs + slot(j * 4 + g, kc), vg);
                     }
                 }
             }
-            if (run_total<false>(key, rs) && key < MP && rs != 0) atomicAdd(&h.rowsum[key], rs);
+            rs = __reduce_add_sync(0xffffffffu, rs);
+            if (lane == 0 && rs != 0) atomicAdd(&h.rowsum[m], rs);
         }
     }
     fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
@@ -667,7 +669,20 @@ cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_d
     const int xm = x_dtype == 2 ? X_QUANTISED : x_dtype == 1 ? X_BF16 : X_F32;
     // the problems of a group share each SM; at least two CTAs fit an SM so the
     // next kernel can start its stream under this one's tail
-    const int budget = group_budget(dev, count);
+    int budget = group_budget(dev, count);
+    if (count == 1) {
+        // A lone problem whose ring cannot hold all of its stages at two CTAs
+        // per SM takes the whole SM instead: its weight stream is then never
+        // throttled by slot reuse (measured at M = 16, N = 11008: the stream
+        // of 2 slots ran 3 us per stage behind the tensor cores).
+        DtcParams t = {};
+        int gt = 0, grid;
+        size_t sm;
+        const int full = dev.max_smem_optin - 1024;
+        if (dtc_configure(t, gt, M, probs[0].K, probs[0].N, dev, budget, grid, sm) && t.slots < t.ntiles * t.T &&
+            dtc_configure(t, gt, M, probs[0].K, probs[0].N, dev, full, grid, sm))
+            budget = full;
+    }
     DtcGroup g;
     memset(&g, 0, sizeof(g));
     g.count = count;

@@ -87,49 +87,27 @@ def sw128(row, chunk):
     return (row // 8) * 1024 + (row % 8) * 128 + ((chunk ^ (row % 8)) << 4)
 
 
-NT, NB = 384, 4          # unpack threads; x_q chunks each thread loads at once
+NW = 12                  # unpack warps
 
 
-def run_total(keys, vals, op):
-    """The warp's segmented reduction: five shuffle-down steps, each adding
-    (or taking the max of) the value `off` lanes down when that lane holds the
-    same key (a lane past the warp reads its own value).  Returns the values
-    and which lanes lead a run of equal keys."""
-    v = list(vals)
-    for off in (1, 2, 4, 8, 16):
-        o = [v[l + off] if l + off < 32 else v[l] for l in range(32)]
-        ko = [keys[l + off] if l + off < 32 else keys[l] for l in range(32)]
-        v = [op(v[l], o[l]) if (l + off < 32 and ko[l] == keys[l]) else v[l] for l in range(32)]
-    return v, [l == 0 or keys[l - 1] != keys[l] for l in range(32)]
-
-
-def flat_rowsum(x_q, M, K, mp, S, KC, Lfull):
-    """Row sums of x_hat as the staging pass forms them: (token, slice,
-    chunk) entries dealt to NT threads NB at a time, per-warp segmented sums,
-    one shared add per run leader."""
-    per_tok = S * KC
-    total = mp * per_tok
+def row_rowsum(x_q, M, K, mp, S, KC, Lfull):
+    """Row sums of x_hat as the staging pass forms them: B row j = q * mp + m
+    (slice q, token m) to warp j % NW, its KC chunks to the lanes (lane l
+    takes chunks l, l + 32, ...), a warp sum per row and one shared add per
+    row into token m's total."""
     rows = [0] * mp
-    for e0 in range(0, total, NB * NT):
-        for b in range(NB):
-            for w in range(NT // 32):
-                keys, vals = [], []
-                for lane in range(32):
-                    e = e0 + b * NT + 32 * w + lane
-                    key, val = mp, 0
-                    if e < total:
-                        m, r = divmod(e, per_tok)
-                        q, kc = divmod(r, KC)
-                        kl = kc * 16
-                        key = m
-                        if m < M and kl < min(Lfull, K - q * Lfull):
-                            val = int(x_q[m, q * Lfull + kl:q * Lfull + kl + 16].astype(np.int64).sum())
-                    keys.append(key)
-                    vals.append(val)
-                tot, lead = run_total(keys, vals, lambda a, c: a + c)
-                for lane in range(32):
-                    if lead[lane] and keys[lane] < mp and tot[lane] != 0:
-                        rows[keys[lane]] += tot[lane]
+    for w in range(NW):
+        for j in range(w, S * mp, NW):
+            q, m = divmod(j, mp)
+            ls = min(Lfull, K - q * Lfull) if m < M else 0
+            lane_sums = [0] * 32
+            for lane in range(32):
+                for kc in range(lane, KC, 32):
+                    if kc * 16 < ls:
+                        k0 = q * Lfull + kc * 16
+                        lane_sums[lane] += int(x_q[m, k0:k0 + 16].astype(np.int64).sum())
+            if sum(lane_sums) != 0:
+                rows[m] += sum(lane_sums)
     return rows
 
 
@@ -160,7 +138,7 @@ def emulate(p, Wbytes, x_q, rng):
                         vg[4 * g:4 * g + 4] = v[4 * g:4 * g + 4]
                     o = p["b_off"] + kb_off + j * 128 + (((kc & 7) ^ (j & 7)) << 4)
                     smem[o:o + 16] = vg.view(np.uint8)
-        rowsum = flat_rowsum(x_q, M, K, mp, S, KC, Lfull)
+        rowsum = row_rowsum(x_q, M, K, mp, S, KC, Lfull)
         part = np.zeros((Rt, mp), np.int64)
         u4 = 0
         for tile in range(p["ntiles"]):
@@ -276,32 +254,12 @@ def test_emulated_cases_cover_the_kernel_shapes():
     assert any(p["nmma"] > p["brow"] for p in shapes)                  # B read past its rows
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_segmented_warp_reduction(seed):
-    """Every run leader of the shuffle scan holds its run's sum and max, for
-    runs of every length from 1 to 32 and a trailing sentinel run."""
-    rng = np.random.default_rng(seed)
-    for _ in range(50):
-        lens, n = [], 0
-        while n < 32:
-            lens.append(int(min(32 - n, rng.integers(1, 33 if seed % 2 else 6))))
-            n += lens[-1]
-        keys = sum(([k] * l for k, l in enumerate(lens)), [])
-        vals = [int(v) for v in rng.integers(0, 1 << 20, 32)]
-        for op, ref in ((lambda a, c: a + c, sum), (max, max)):
-            tot, lead = run_total(keys, vals, op)
-            starts = np.cumsum([0] + lens[:-1])
-            assert [l for l in range(32) if lead[l]] == list(starts)
-            for k, (s0, l) in enumerate(zip(starts, lens)):
-                assert tot[s0] == ref(vals[s0:s0 + l])
-
-
-def test_flat_rowsum_matches_the_row_sums():
+def test_staging_row_sums_match_the_token_sums():
     rng = np.random.default_rng(3)
     for M, K, S in ((16, 4096, 4), (5, 1088, 2), (1, 640, 1), (9, 2048, 1)):
         mp = pow2(M)
         Lfull = ru(-(-K // S), STAGE_K)
         T = Lfull // STAGE_K
         x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
-        rows = flat_rowsum(x_q, M, K, mp, S, T * (STAGE_K // 16), Lfull)
+        rows = row_rowsum(x_q, M, K, mp, S, T * (STAGE_K // 16), Lfull)
         assert rows == [int(x_q[m].astype(np.int64).sum()) if m < M else 0 for m in range(mp)]
