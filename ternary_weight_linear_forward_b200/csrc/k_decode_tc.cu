@@ -656,7 +656,7 @@ int decode_tc_max_m() { return DTC_MAX_M; }
 
 bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev) {
     DtcParams p = {};
-    int G, grid;
+    int G = 0, grid;
     size_t smem;
     return count >= 1 && count <= DTC_GROUP_MAX &&
            dtc_configure(p, G, M, K, N, dev, group_budget(dev, count), grid, smem);

@@ -45,35 +45,47 @@ namespace bl {
 
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 128;  // rows of one MMA (a sub-tile)
 constexpr int BN = 256;
 constexpr int BK = 128;  // bytes of K per stage
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK;           // 16 KiB
-constexpr int BC_BYTES = BN * BK;          // 32 KiB unpacked codes
+constexpr int A_SUB_BYTES = BM * BK;          // 16 KiB of x_q per sub-tile
+constexpr int BC_BYTES = BN * BK;             // 32 KiB unpacked codes
 constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words (2-bit; 1-bit uses half)
-constexpr int STAGE_BYTES = A_BYTES + BC_BYTES + BP_BYTES;
 constexpr int HDR_BYTES = 1024;
-constexpr int GEMM_SMEM = 1024 /* alignment slack */ + HDR_BYTES + STAGES * STAGE_BYTES;
+constexpr int MAX_STAGES = 4;
 constexpr int UNPACK_WARPS = 8;
 constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
-constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;               // epilogue warps EPI_WARP0 .. +3
-constexpr int GEMM_THREADS = (EPI_WARP0 + 4) * 32;
+constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;  // epilogue warps EPI_WARP0 .. EPI_WARP0 + 4 MT - 1
+
+// A tile is MT sub-tiles of 128 rows on the same 256 weight rows: MT = 2
+// issues two MMAs (two accumulators) per unpacked B block, halving the unpack
+// and the packed-weight traffic per output; its two accumulators fill tensor
+// memory, so they are not double-buffered.
+template <int MT> constexpr int tile_rows() { return BM * MT; }
+template <int MT> constexpr int a_bytes() { return A_SUB_BYTES * MT; }
+template <int MT> constexpr int stage_bytes() { return a_bytes<MT>() + BC_BYTES + BP_BYTES; }
+template <int MT> constexpr int num_stages() { return MT == 1 ? 4 : 3; }
+template <int MT> constexpr int gemm_smem() { return 1024 /* alignment slack */ + HDR_BYTES + num_stages<MT>() * stage_bytes<MT>(); }
+template <int MT> constexpr int gemm_threads() { return (EPI_WARP0 + 4 * MT) * 32; }
+template <int MT> constexpr int acc_sets() { return MT == 1 ? 2 : 1; }
+static_assert(gemm_smem<1>() <= 232448 && gemm_smem<2>() <= 232448, "GEMM stages exceed shared memory");
+static_assert(num_stages<1>() <= MAX_STAGES && num_stages<2>() <= MAX_STAGES, "stage count");
+static_assert(acc_sets<1>() * 1 * BN <= 512 && acc_sets<2>() * 2 * BN <= 512, "accumulators exceed TMEM");
 // packed words per row and K-block: 8 of 16 trits, or 4 of 32 signs
 template <int WB>
 constexpr int words_per_row() { return BK * WB / 32; }
 template <int WB>
 constexpr int words_per_thread() { return BN * words_per_row<WB>() / UNPACK_THREADS; }
-constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators
+constexpr int TMEM_COLS = 512;  // two 128 x 256 int32 accumulators (double buffer, or the two sub-tiles)
 
 constexpr uint32_t IDESC = idesc_i8(BM, BN, true, true);  // s8 x s8 -> s32, 128 x 256
 
 struct GemmHdr {
-    uint64_t full[STAGES];      // TMA bytes landed
-    uint64_t unpacked[STAGES];  // codes written by the unpack threads
-    uint64_t empty[STAGES];     // MMAs reading the stage finished
-    uint64_t tfull[2];          // accumulator complete
-    uint64_t tempty[2];         // accumulator drained by the 128 epilogue threads
+    uint64_t full[MAX_STAGES];      // TMA bytes landed
+    uint64_t unpacked[MAX_STAGES];  // codes written by the unpack threads
+    uint64_t empty[MAX_STAGES];     // MMAs reading the stage finished
+    uint64_t tfull[2];              // accumulator set complete
+    uint64_t tempty[2];             // accumulator set drained by the 128 MT epilogue threads
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -213,10 +225,14 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int m, int n0, 
     }
 }
 
-template <int WB>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <int WB, int MT>
+__global__ void __launch_bounds__(gemm_threads<MT>(), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
+    constexpr int STAGES = num_stages<MT>();
+    constexpr int STAGE_BYTES = stage_bytes<MT>();
+    constexpr int A_BYTES = a_bytes<MT>();
+    constexpr int SETS = acc_sets<MT>();
     extern __shared__ unsigned char smem_raw[];
     unsigned char* base =
         smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-byte aligned for the swizzle
@@ -231,9 +247,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&h.unpacked[s], UNPACK_THREADS);
             mbar_init(&h.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < SETS; ++b) {
             mbar_init(&h.tfull[b], 1);
-            mbar_init(&h.tempty[b], 128);
+            mbar_init(&h.tempty[b], 128 * MT);
         }
         h.abort_flag = 0;
         fence_mbar_init();
@@ -262,7 +278,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     if (!wait_or_abort(h, &h.empty[s], ph ^ 1)) goto done;
                     unsigned char* st = stages + (size_t)s * STAGE_BYTES;
                     mbar_arrive_expect_tx(&h.full[s], A_BYTES + BN * words_per_row<WB>() * 4);
-                    tma_load_2d(st, &tmap_a, kb * BK, mb * BM, &h.full[s]);
+                    tma_load_2d(st, &tmap_a, kb * BK, mb * tile_rows<MT>(), &h.full[s]);
                     tma_load_2d(st + A_BYTES + BC_BYTES, &tmap_b, kb * words_per_row<WB>(), nb * BN, &h.full[s]);
                 }
             }
@@ -274,11 +290,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++acc_it) {
                 int t, kb0, kb1;
                 unit_range(p, u, t, kb0, kb1);
-                const int b = acc_it & 1;
-                const uint32_t aph = (acc_it >> 1) & 1;
+                const int b = acc_it % SETS;
+                const uint32_t aph = (acc_it / SETS) & 1;
                 if (!wait_or_abort(h, &h.tempty[b], aph ^ 1)) goto done;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
+                const uint32_t d_tmem = tmem + (uint32_t)(b * MT * BN);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
@@ -286,11 +302,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     if (!wait_or_abort(h, &h.unpacked[s], ph)) goto done;
                     tc_fence_after();
                     unsigned char* st = stages + (size_t)s * STAGE_BYTES;
-                    const uint64_t adesc = sw128_desc(smem_u32(st));
                     const uint64_t bdesc = sw128_desc(smem_u32(st + A_BYTES));
 #pragma unroll
-                    for (int k = 0; k < BK / 32; ++k)  // K = 32 bytes per MMA: advance 32 B = 2 in addr >> 4
-                        mma_i8(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb != kb0) || (k != 0));
+                    for (int k = 0; k < BK / 32; ++k) {  // K = 32 bytes per MMA: advance 32 B = 2 in addr >> 4
+#pragma unroll
+                        for (int a = 0; a < MT; ++a)      // sub-tile a: x_q rows 128 a .., accumulator a
+                            mma_i8(d_tmem + (uint32_t)(a * BN), sw128_desc(smem_u32(st + a * A_SUB_BYTES)) + 2 * k,
+                                   bdesc + 2 * k, IDESC, (kb != kb0) || (k != 0));
+                    }
                     mma_commit(&h.empty[s]);
                 }
                 mma_commit(&h.tfull[b]);
@@ -361,7 +380,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lanes 32q .. 32q + 31
+        const int q = warp & 3;                  // TMEM lanes 32q .. 32q + 31
+        const int sub = (warp - EPI_WARP0) / 4;  // sub-tile (accumulator) of this warp
         const bool vec_ok = p.mode == Y_BF16 ? (p.N % 8 == 0) : (p.N % 4 == 0);
         const float beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         int acc_it = 0;
@@ -369,21 +389,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             int t, kb0, kb1;
             unit_range(p, u, t, kb0, kb1);
             const int mb = t % p.tiles_m, nb = t / p.tiles_m;
-            const int b = acc_it & 1;
-            const uint32_t aph = (acc_it >> 1) & 1;
+            const int b = acc_it % SETS;
+            const uint32_t aph = (acc_it / SETS) & 1;
             // tcgen05.ld is warp-collective: the whole warp proceeds or leaves together
             if (!__all_sync(0xffffffffu, wait_or_abort(h, &h.tfull[b], aph))) goto done;
             tc_fence_after();
-            const int r = q * 32 + lane;  // row of the tile
-            const int m = mb * BM + r;
+            const int r = sub * BM + q * 32 + lane;  // row of the tile
+            const int m = mb * tile_rows<MT>() + r;
             int rs = 0;
             float f = 0.0f;
             if (m < p.M) {
                 rs = __ldcg(p.rowsum + m);  // L2 only: written by the preceding kernel
                 if (p.mode != Y_ACC) f = __fdiv_rn(__fmul_rn(beta, __ldg(p.gamma + m)), 127.0f);
             }
-            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
-            if (p.splits == 1) {
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((b * MT + sub) * BN);
+            if (MT > 1 || p.splits == 1) {
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
                     int v[32];
@@ -441,18 +461,26 @@ EncodeTiled tensor_map_encoder() {
 // 148 SMs (a fixed count, so the workspace size does not depend on the device).
 constexpr int SPLIT_UNITS_TARGET = 148;
 
+// Two sub-tiles per tile from this many tokens on (when K is not cut).
+constexpr long long MT2_MIN_M = 256;
+
 struct GemmPlan {
-    int tiles_m, tiles_n, num_kb, splits, part_rows;
+    int mt, tiles_m, tiles_n, num_kb, splits, part_rows;
     size_t rowsum_bytes, part_bytes;
 };
 
 GemmPlan gemm_plan(long long M, long long N, long long K, bool allow_split) {
     GemmPlan g;
+    g.mt = 1;
     g.tiles_m = (int)((M + BM - 1) / BM);
     g.tiles_n = (int)((N + BN - 1) / BN);
     g.num_kb = (int)((K + BK - 1) / BK);
     const long long tiles = (long long)g.tiles_m * g.tiles_n;
     g.splits = allow_split ? (int)std::max<long long>(1, std::min<long long>(SPLIT_UNITS_TARGET / tiles, g.num_kb)) : 1;
+    if (g.splits == 1 && M >= MT2_MIN_M) {
+        g.mt = 2;
+        g.tiles_m = (int)((M + 2 * BM - 1) / (2 * BM));
+    }
     g.part_rows = (int)std::min<long long>(M, BM);
     g.rowsum_bytes = (size_t)((M * 4 + 255) / 256 * 256);
     g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.part_rows * BN * 4 : 0;
@@ -470,12 +498,14 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     if (wbits != 1 && wbits != 2) return cudaErrorInvalidValue;
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    if (dev.max_smem_optin < GEMM_SMEM) return cudaErrorNotSupported;
+    const GemmPlan plan = gemm_plan(M, N, K, allow_split);
+    const int smem = plan.mt == 1 ? gemm_smem<1>() : gemm_smem<2>();
+    if (dev.max_smem_optin < smem) return cudaErrorNotSupported;
     CUtensorMap ta, tb;
     {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t strides[1] = {(cuuint64_t)K};
-        const cuuint32_t box[2] = {BK, BM};
+        const cuuint32_t box[2] = {BK, (cuuint32_t)(plan.mt * BM)};
         const cuuint32_t estr[2] = {1, 1};
         if (enc(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(x_q), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -493,7 +523,6 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    const GemmPlan plan = gemm_plan(M, N, K, allow_split);
     int* rowsum = reinterpret_cast<int*>(ws);
     int* part = plan.splits > 1 ? reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + plan.rowsum_bytes) : nullptr;
     cudaError_t e = launch_pdl(rowsum_kernel, dim3((M + 7) / 8), dim3(256), 0, st, x_q, M, K, rowsum);
@@ -516,10 +545,12 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     p.part = part;
     const int units = p.tiles_m * p.tiles_n * p.splits;
     const int grid = std::max(1, std::min(units, dev.num_sms));
-    auto kernel = wbits == 2 ? gemm_kernel<2> : gemm_kernel<1>;
-    e = ensure_smem_optin(reinterpret_cast<const void*>(kernel), GEMM_SMEM);
+    auto kernel = plan.mt == 1 ? (wbits == 2 ? gemm_kernel<2, 1> : gemm_kernel<1, 1>)
+                               : (wbits == 2 ? gemm_kernel<2, 2> : gemm_kernel<1, 2>);
+    const int threads = plan.mt == 1 ? gemm_threads<1>() : gemm_threads<2>();
+    e = ensure_smem_optin(reinterpret_cast<const void*>(kernel), (size_t)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kernel, dim3(grid), dim3(GEMM_THREADS), (size_t)GEMM_SMEM, st, ta, tb, p);
+    e = launch_pdl(kernel, dim3(grid), dim3(threads), (size_t)smem, st, ta, tb, p);
     if (e != cudaSuccess || plan.splits == 1) return e;
     const long long quads = (long long)M * ((N + 3) / 4);
     const int fgrid = (int)std::max<long long>(1, std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8));

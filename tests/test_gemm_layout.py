@@ -1,8 +1,10 @@
 """CPU emulation of the prefill GEMM's tile walk and operand layouts.
 
 The tcgen05 GEMM is persistent: CTA b takes work units b, b + grid, ...;
-a unit is a 128 x 256 output tile (m-fastest order) and, when there are few
-tiles, one of `splits` ranges of its K-blocks.  Per 128-byte K-block a TMA
+a unit is a 128 MT x 256 output tile (m-fastest order) and, when there are few
+tiles, one of `splits` ranges of its K-blocks.  From 256 tokens on (and no
+split) a tile is two 128-row sub-tiles (MT = 2) whose two MMAs, into two
+accumulators, read the same unpacked B block.  Per 128-byte K-block a TMA
 box of x_q (128 rows, 128-byte swizzle, zero fill past M and K) and a box of
 packed words (256 rows, zero fill) land in a stage; unpack warps expand each
 word into 16-byte code chunks of the K-major, 128-byte-swizzled B operand
@@ -23,16 +25,20 @@ import oracle
 
 BM, BN, BK = 128, 256, 128
 SPLIT_UNITS_TARGET = 148
+MT2_MIN_M = 256
 
 
 def plan(M, N, K, allow_split=True):
     tiles_m, tiles_n, num_kb = (M + BM - 1) // BM, (N + BN - 1) // BN, (K + BK - 1) // BK
     tiles = tiles_m * tiles_n
     splits = max(1, min(SPLIT_UNITS_TARGET // tiles, num_kb)) if allow_split else 1
+    mt = 1
+    if splits == 1 and M >= MT2_MIN_M:
+        mt, tiles_m = 2, (M + 2 * BM - 1) // (2 * BM)
     part_rows = min(M, BM)
     rowsum_bytes = (M * 4 + 255) // 256 * 256
     part_bytes = tiles * splits * part_rows * BN * 4 if splits > 1 else 0
-    return dict(tiles_m=tiles_m, tiles_n=tiles_n, num_kb=num_kb, splits=splits, part_rows=part_rows,
+    return dict(mt=mt, tiles_m=tiles_m, tiles_n=tiles_n, num_kb=num_kb, splits=splits, part_rows=part_rows,
                 ws_bytes=rowsum_bytes + part_bytes, part_off=rowsum_bytes)
 
 
@@ -54,6 +60,7 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
     pl = plan(M, N, K, allow_split)
     tiles_m, tiles_n, num_kb, splits, part_rows = (pl[k] for k in ("tiles_m", "tiles_n", "num_kb", "splits",
                                                                     "part_rows"))
+    TBM = BM * pl["mt"]                               # rows of a tile: MT sub-tiles of 128
     wpr = BK * wbits // 32                            # packed words per row and K-block
     xq_u8 = x_q.view(np.uint8)
     rowsum = x_q.astype(np.int64).sum(1)
@@ -68,14 +75,14 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
             sp = u % splits
             kb0, kb1 = num_kb * sp // splits, num_kb * (sp + 1) // splits
             mb, nb = t % tiles_m, t // tiles_m
-            D = np.zeros((BM, BN), np.int64)
+            D = np.zeros((TBM, BN), np.int64)             # MT accumulators of 128 rows
             for kb in range(kb0, kb1):
                 kb_seen[t, kb] += 1
-                a_st = rng.integers(0, 256, BM * BK, dtype=np.int64).astype(np.uint8)
+                a_st = rng.integers(0, 256, TBM * BK, dtype=np.int64).astype(np.uint8)
                 b_st = rng.integers(0, 256, BN * BK, dtype=np.int64).astype(np.uint8)
                 # x_q box with the 128-byte swizzle
-                box = tma_box(xq_u8, mb * BM, kb * BK, BM, BK)
-                for r in range(BM):
+                box = tma_box(xq_u8, mb * TBM, kb * BK, TBM, BK)
+                for r in range(TBM):
                     for c in range(8):
                         a_st[sw128_off(r, c):sw128_off(r, c) + 16] = box[r, 16 * c:16 * c + 16]
                 # packed words (no swizzle), then the unpack into swizzled code chunks
@@ -92,16 +99,20 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
                         for c, ts in chunks.items():
                             o = sw128_off(n, c)
                             b_st[o:o + 16] = np.array(ts, np.uint32).view(np.uint8)
-                # four MMAs of K = 32 bytes: both operands read through the swizzle
-                A = np.stack([np.concatenate([a_st[sw128_off(r, c):sw128_off(r, c) + 16] for c in range(8)])
-                              for r in range(BM)]).view(np.int8).astype(np.int64)
+                # four MMAs of K = 32 bytes per sub-tile: sub-tile a's A operand starts
+                # 16 KiB into the stage, its rows read through the same swizzle
                 B = np.stack([np.concatenate([b_st[sw128_off(n, c):sw128_off(n, c) + 16] for c in range(8)])
                               for n in range(BN)]).view(np.int8).astype(np.int64)
-                for k in range(BK // 32):
-                    D += A[:, 32 * k:32 * k + 32] @ B[:, 32 * k:32 * k + 32].T
+                for a in range(pl["mt"]):
+                    base = a * BM * BK
+                    A = np.stack([np.concatenate([a_st[base + sw128_off(r, c):base + sw128_off(r, c) + 16]
+                                                  for c in range(8)])
+                                  for r in range(BM)]).view(np.int8).astype(np.int64)
+                    for k in range(BK // 32):
+                        D[a * BM:(a + 1) * BM] += A[:, 32 * k:32 * k + 32] @ B[:, 32 * k:32 * k + 32].T
             if splits == 1:
-                for r in range(BM):
-                    m = mb * BM + r
+                for r in range(TBM):                  # epilogue warp (sub-tile r // 128, lanes of r % 128)
+                    m = mb * TBM + r
                     if m < M:
                         n0, n1 = nb * BN, min(N, nb * BN + BN)
                         y[m, n0:n1] = D[r, :n1 - n0] - rowsum[m]
@@ -168,3 +179,29 @@ def test_one_bit_gemm_emulation_matches_the_oracle(M, K, N, grid):
     x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
     y = emulate(x_q, oracle.pack_bits(W_b), K, N, 1, grid, rng)
     np.testing.assert_array_equal(y, oracle.ternary_acc(x_q, W_b))
+
+
+@pytest.mark.parametrize("M,K,N,grid,wbits,split", [(300, 128, 520, 3, 2, True), (600, 128, 260, 2, 1, True),
+                                                     (256, 384, 300, 1, 2, False), (513, 256, 40, 2, 2, False)])
+def test_two_sub_tile_gemm_emulation_matches_the_oracle(M, K, N, grid, wbits, split):
+    # small shapes take two sub-tiles when K is not cut: one K-block, or no
+    # split allowed (the workspace-free entry point)
+    pl = plan(M, N, K, split)
+    assert pl["mt"] == 2 and pl["splits"] == 1
+    rng = np.random.default_rng(M * 5 + K + N + wbits)
+    if wbits == 2:
+        W = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        W_p = oracle.pack(W)
+    else:
+        W = np.where(rng.random((N, K)) < 0.5, 1, -1).astype(np.int8)
+        W_p = oracle.pack_bits(W)
+    x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    np.testing.assert_array_equal(emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=split),
+                                  oracle.ternary_acc(x_q, W))
+
+
+def test_sub_tiles_of_the_prefill_shapes():
+    for N in (4096, 11008):
+        pl = plan(2048, N, 4096)
+        assert pl["mt"] == 2 and pl["tiles_m"] == 8 and pl["splits"] == 1
+    assert plan(64, 4096, 4096)["mt"] == 1 and plan(200, 4096, 4096)["mt"] == 1
