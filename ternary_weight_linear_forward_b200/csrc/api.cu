@@ -109,8 +109,11 @@ DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& 
     return M <= AUTO_CUDA_MAX_M ? PATH_CUDA : PATH_GEMM;
 }
 
+// rowsum_ready: on the GEMM path, the quantiser has written the row sums of
+// x_q at the start of ws.
 bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
-                      const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes, void* stream) {
+                      const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes, void* stream,
+                      bool rowsum_ready = false) {
     const size_t need = bitlinear_forward_workspace(M, N, K);
     if (need && (!ws || ws_bytes < need)) return BL_ERR_WORKSPACE;
     if (need && !aligned16(ws)) return BL_ERR_ALIGN;
@@ -125,7 +128,8 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
     else if (path == PATH_CUDA)
         e = launch_decode_cuda(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
     else
-        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream));
+        e = launch_gemm(x_q, gamma, (int)M, (int)K, W_p, beta, (int)N, y, mode, ws, dev, as_stream(stream), 2, true,
+                        rowsum_ready);
     return from_cuda(e);
 }
 
@@ -415,10 +419,14 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
     int8_t* x_q = reinterpret_cast<int8_t*>(ws);
     float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
     char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * 4);
-    cudaError_t e = launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream));
+    // on the GEMM path the quantiser also writes the row sums the GEMM needs
+    // (at the start of its workspace), which saves the row-sum launch
+    const bool gemm = pick_path((int)M, &prob, 1, dev) == PATH_GEMM;
+    cudaError_t e = launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream),
+                                     gemm ? reinterpret_cast<int*>(fws) : nullptr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
     return run_forward(x_q, gamma, M, K, W_p, beta, N, y, mode, fws, ws_bytes - (fws - reinterpret_cast<char*>(ws)),
-                       stream);
+                       stream, gemm);
 }
 
 bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int64_t M, int x_dtype, int y_dtype,

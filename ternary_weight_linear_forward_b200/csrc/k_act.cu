@@ -57,13 +57,28 @@ __device__ __forceinline__ void load16(const void* row, int g, float (&v)[16]) {
     }
 }
 
-__device__ __forceinline__ void store16(int8_t* row_q, int g, const float (&v)[16], float s) {
+// Returns the sum of the 16 codes.
+__device__ __forceinline__ int store16(int8_t* row_q, int g, const float (&v)[16], float s) {
     uint4 o;
     o.x = pack4(q8(v[0], s), q8(v[1], s), q8(v[2], s), q8(v[3], s));
     o.y = pack4(q8(v[4], s), q8(v[5], s), q8(v[6], s), q8(v[7], s));
     o.z = pack4(q8(v[8], s), q8(v[9], s), q8(v[10], s), q8(v[11], s));
     o.w = pack4(q8(v[12], s), q8(v[13], s), q8(v[14], s), q8(v[15], s));
     reinterpret_cast<uint4*>(row_q)[g] = o;
+    return __dp4a((int)o.x, 0x01010101, 0) + __dp4a((int)o.y, 0x01010101, 0) + __dp4a((int)o.z, 0x01010101, 0) +
+           __dp4a((int)o.w, 0x01010101, 0);
+}
+
+// block-wide sum of ints
+__device__ __forceinline__ int block_sum_i32(int v, int* sm) {
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    int r = lane < ACT_THREADS / 32 ? sm[lane] : 0;
+    for (int off = 16; off; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+    __syncthreads();
+    return r;
 }
 
 // block-wide max of non-negative floats (compared as bit patterns)
@@ -90,9 +105,11 @@ __device__ __forceinline__ double block_sum_f64(double v, double* sm) {
 }
 
 // Quantise the n activations at xr (n % 16 == 0) with their own absmax:
-// codes to qr, the floored absmax to *gamma_out.  Called by whole CTAs.
+// codes to qr, the floored absmax to *gamma_out and, when rowsum_out is not
+// null, the sum of the codes to *rowsum_out.  Called by whole CTAs.
 template <bool BF16>
-__device__ __forceinline__ void quant_row(const char* xr, int n, int8_t* qr, float* gamma_out, unsigned* sm) {
+__device__ __forceinline__ void quant_row(const char* xr, int n, int8_t* qr, float* gamma_out, unsigned* sm,
+                                          int* rowsum_out = nullptr) {
     const int G = n / 16;
     float amax = 0.0f;
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
@@ -104,23 +121,29 @@ __device__ __forceinline__ void quant_row(const char* xr, int n, int8_t* qr, flo
     amax = block_max_nonneg(amax, sm);
     const float gm = fmaxf(amax, 1e-5f);
     const float s = __fdiv_rn(127.0f, gm);
+    int rs = 0;
     for (int g = threadIdx.x; g < G; g += ACT_THREADS) {
         float v[16];
         load16<BF16>(xr, g, v);
-        store16(qr, g, v, s);
+        rs += store16(qr, g, v, s);
+    }
+    if (rowsum_out) {  // uniform over the CTA
+        rs = block_sum_i32(rs, reinterpret_cast<int*>(sm));
+        if (threadIdx.x == 0) *rowsum_out = rs;
     }
     if (threadIdx.x == 0) *gamma_out = gm;
 }
 
 template <bool BF16>
 __global__ void __launch_bounds__(ACT_THREADS) quant_act_kernel(const void* __restrict__ x, int K,
-                                                                int8_t* __restrict__ x_q, float* __restrict__ gamma) {
+                                                                int8_t* __restrict__ x_q, float* __restrict__ gamma,
+                                                                int* __restrict__ rowsum) {
     __shared__ unsigned sm[ACT_THREADS / 32];
     pdl_launch_dependents();
     pdl_wait();
     const long long row = blockIdx.x;
     const char* xr = reinterpret_cast<const char*>(x) + row * (long long)K * (BF16 ? 2 : 4);
-    quant_row<BF16>(xr, K, x_q + row * (long long)K, gamma + row, sm);
+    quant_row<BF16>(xr, K, x_q + row * (long long)K, gamma + row, sm, rowsum ? rowsum + row : nullptr);
 }
 
 // Group quantisation (unite.ai page, "Gruppenquantisierung und
@@ -239,10 +262,12 @@ __global__ void __launch_bounds__(ACT_THREADS) quant_act_rms_kernel(const float*
 }  // namespace
 
 cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
-                             cudaStream_t st) {
+                             cudaStream_t st, int* rowsum) {
     if (bf16)
-        return launch_pdl(quant_act_kernel<true>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
-    return launch_pdl(quant_act_kernel<false>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma);
+        return launch_pdl(quant_act_kernel<true>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma,
+                          rowsum);
+    return launch_pdl(quant_act_kernel<false>, dim3((unsigned)M), dim3(ACT_THREADS), 0, st, x, (int)K, x_q, gamma,
+                      rowsum);
 }
 
 cudaError_t launch_quant_act_grouped(const void* x, bool bf16, long long M, long long K, int G, int8_t* x_q,

@@ -99,16 +99,27 @@ struct GemmParams {
     int M, N, K, mode;
     int tiles_m, tiles_n, num_kb;
     int splits;     // K ranges per tile (1: no split)
-    int part_rows;  // rows of a partial tile in the workspace (min(M, BM))
-    int* part;      // split K: [tiles * splits][part_rows][BN] int32 partial tiles
+    int nfull;      // units 0 .. nfull - 1 are whole tiles; each later tile is cut into `splits` K ranges
+    int part_rows;  // rows of a partial tile in the workspace (min(M, tile rows))
+    int* part;      // split K: [cut tiles * splits][part_rows][BN] int32 partial tiles
 };
 
-// Work unit u: tile u / splits, K blocks [kb0, kb1) of its split u % splits.
-__device__ __forceinline__ void unit_range(const GemmParams& p, int u, int& t, int& kb0, int& kb1) {
-    t = u / p.splits;
-    const int sp = u % p.splits;
+// Work unit u: whole tile u below nfull; past it, unit v = u - nfull is K
+// blocks [kb0, kb1) of split v % splits of tile nfull + v / splits.  Returns
+// whether the unit writes a partial tile.
+__device__ __forceinline__ bool unit_range(const GemmParams& p, int u, int& t, int& kb0, int& kb1) {
+    if (u < p.nfull) {
+        t = u;
+        kb0 = 0;
+        kb1 = p.num_kb;
+        return false;
+    }
+    const int v = u - p.nfull;
+    t = p.nfull + v / p.splits;
+    const int sp = v % p.splits;
     kb0 = (int)((long long)p.num_kb * sp / p.splits);
     kb1 = (int)((long long)p.num_kb * (sp + 1) / p.splits);
+    return p.splits > 1;
 }
 
 
@@ -144,22 +155,28 @@ __global__ void __launch_bounds__(256) rowsum_kernel(const int8_t* __restrict__ 
 }
 
 // Split K: y[m, n] = (sum over the splits of the partial tiles) - rowsum_m,
-// rescaled; four consecutive n per thread (one 16-byte load per split).
+// rescaled, for the outputs of the cut tiles (tiles nfull ..); four
+// consecutive n per thread (one 16-byte load per split).
 __global__ void __launch_bounds__(256) splitk_finish_kernel(const int* __restrict__ part, int splits, int part_rows,
-                                                            int tiles_m, const int* __restrict__ rowsum,
+                                                            int nfull, int ncut, int tiles_m, int tile_rows,
+                                                            const int* __restrict__ rowsum,
                                                             const float* __restrict__ gamma,
                                                             const float* __restrict__ beta, void* __restrict__ y,
                                                             int M, int N, int mode) {
     pdl_launch_dependents();
     pdl_wait();
     const float b = mode == Y_ACC ? 0.0f : __ldg(beta);
-    const int nq = (N + 3) / 4;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)M * nq;
+    constexpr int NQ = BN / 4;  // quads per tile row
+    const long long per_tile = (long long)part_rows * NQ;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)ncut * per_tile;
          e += (long long)gridDim.x * blockDim.x) {
-        const int m = (int)(e / nq), n = (int)(e % nq) * 4;
-        const int mb = m / BM, r = m % BM, nb = n / BN, c = n % BN;
-        const int t = mb + nb * tiles_m;
-        const int4* src = reinterpret_cast<const int4*>(part + ((size_t)t * splits * part_rows + r) * BN + c);
+        const int tt = (int)(e / per_tile);
+        const int rem = (int)(e - (long long)tt * per_tile);
+        const int r = rem / NQ, c = (rem % NQ) * 4;
+        const int t = nfull + tt;
+        const int m = (t % tiles_m) * tile_rows + r, n = (t / tiles_m) * BN + c;
+        if (m >= M || n >= N) continue;
+        const int4* src = reinterpret_cast<const int4*>(part + ((size_t)tt * splits * part_rows + r) * BN + c);
         int4 acc = make_int4(0, 0, 0, 0);
         for (int sp = 0; sp < splits; ++sp) {
             const int4 v = __ldcg(src + (size_t)sp * part_rows * BN / 4);
@@ -239,7 +256,7 @@ __global__ void __launch_bounds__(gemm_threads<MT>(), 1)
     GemmHdr& h = *reinterpret_cast<GemmHdr*>(base);
     unsigned char* stages = base + HDR_BYTES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_units = p.tiles_m * p.tiles_n * p.splits;
+    const int num_units = p.nfull + (p.tiles_m * p.tiles_n - p.nfull) * p.splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -387,7 +404,7 @@ __global__ void __launch_bounds__(gemm_threads<MT>(), 1)
         int acc_it = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++acc_it) {
             int t, kb0, kb1;
-            unit_range(p, u, t, kb0, kb1);
+            const bool cut = unit_range(p, u, t, kb0, kb1);
             const int mb = t % p.tiles_m, nb = t / p.tiles_m;
             const int b = acc_it % SETS;
             const uint32_t aph = (acc_it / SETS) & 1;
@@ -403,7 +420,7 @@ __global__ void __launch_bounds__(gemm_threads<MT>(), 1)
                 if (p.mode != Y_ACC) f = __fdiv_rn(__fmul_rn(beta, __ldg(p.gamma + m)), 127.0f);
             }
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((b * MT + sub) * BN);
-            if (MT > 1 || p.splits == 1) {
+            if (!cut) {
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
                     int v[32];
@@ -416,7 +433,7 @@ __global__ void __launch_bounds__(gemm_threads<MT>(), 1)
                 continue;
             }
             // split K: this unit's partial tile to the workspace
-            int* mine = p.part + ((size_t)u * p.part_rows + r) * BN;
+            int* mine = p.part + ((size_t)(u - p.nfull) * p.part_rows + r) * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 int v[32];
@@ -464,8 +481,12 @@ constexpr int SPLIT_UNITS_TARGET = 148;
 // Two sub-tiles per tile from this many tokens on (when K is not cut).
 constexpr long long MT2_MIN_M = 256;
 
+// A last round of at most half the SMs is cut along K into at most this
+// many ranges, so that it fills the SMs.
+constexpr int TAIL_SPLIT_MAX = 4;
+
 struct GemmPlan {
-    int mt, tiles_m, tiles_n, num_kb, splits, part_rows;
+    int mt, tiles_m, tiles_n, num_kb, splits, nfull, part_rows;
     size_t rowsum_bytes, part_bytes;
 };
 
@@ -477,13 +498,28 @@ GemmPlan gemm_plan(long long M, long long N, long long K, bool allow_split) {
     g.num_kb = (int)((K + BK - 1) / BK);
     const long long tiles = (long long)g.tiles_m * g.tiles_n;
     g.splits = allow_split ? (int)std::max<long long>(1, std::min<long long>(SPLIT_UNITS_TARGET / tiles, g.num_kb)) : 1;
-    if (g.splits == 1 && M >= MT2_MIN_M) {
-        g.mt = 2;
-        g.tiles_m = (int)((M + 2 * BM - 1) / (2 * BM));
+    g.nfull = 0;
+    if (g.splits == 1) {
+        if (M >= MT2_MIN_M) {
+            g.mt = 2;
+            g.tiles_m = (int)((M + 2 * BM - 1) / (2 * BM));
+        }
+        const long long all = (long long)g.tiles_m * g.tiles_n;
+        g.nfull = (int)all;
+        const long long tail = all % SPLIT_UNITS_TARGET;
+        if (allow_split && all > SPLIT_UNITS_TARGET && tail > 0 && tail <= SPLIT_UNITS_TARGET / 2) {
+            const int s = (int)std::min<long long>(std::min<long long>(SPLIT_UNITS_TARGET / tail, g.num_kb),
+                                                   TAIL_SPLIT_MAX);
+            if (s > 1) {
+                g.nfull = (int)(all - tail);
+                g.splits = s;
+            }
+        }
     }
-    g.part_rows = (int)std::min<long long>(M, BM);
+    const long long cut = (long long)g.tiles_m * g.tiles_n - g.nfull;
+    g.part_rows = (int)std::min<long long>(M, (long long)g.mt * BM);
     g.rowsum_bytes = (size_t)((M * 4 + 255) / 256 * 256);
-    g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.part_rows * BN * 4 : 0;
+    g.part_bytes = g.splits > 1 ? (size_t)cut * g.splits * g.part_rows * BN * 4 : 0;
     return g;
 }
 
@@ -494,7 +530,7 @@ size_t gemm_ws_bytes(long long M, long long N, long long K) {
 
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
                         int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits,
-                        bool allow_split) {
+                        bool allow_split, bool rowsum_ready) {
     if (wbits != 1 && wbits != 2) return cudaErrorInvalidValue;
     EncodeTiled enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
@@ -525,8 +561,11 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     }
     int* rowsum = reinterpret_cast<int*>(ws);
     int* part = plan.splits > 1 ? reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + plan.rowsum_bytes) : nullptr;
-    cudaError_t e = launch_pdl(rowsum_kernel, dim3((M + 7) / 8), dim3(256), 0, st, x_q, M, K, rowsum);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!rowsum_ready) {
+        e = launch_pdl(rowsum_kernel, dim3((M + 7) / 8), dim3(256), 0, st, x_q, M, K, rowsum);
+        if (e != cudaSuccess) return e;
+    }
 
     GemmParams p;
     p.gamma = gamma;
@@ -541,9 +580,11 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     p.tiles_n = plan.tiles_n;
     p.num_kb = plan.num_kb;
     p.splits = plan.splits;
+    p.nfull = plan.nfull;
     p.part_rows = plan.part_rows;
     p.part = part;
-    const int units = p.tiles_m * p.tiles_n * p.splits;
+    const int ncut = p.tiles_m * p.tiles_n - p.nfull;
+    const int units = p.nfull + ncut * p.splits;
     const int grid = std::max(1, std::min(units, dev.num_sms));
     auto kernel = plan.mt == 1 ? (wbits == 2 ? gemm_kernel<2, 1> : gemm_kernel<1, 1>)
                                : (wbits == 2 ? gemm_kernel<2, 2> : gemm_kernel<1, 2>);
@@ -552,10 +593,11 @@ cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, con
     if (e != cudaSuccess) return e;
     e = launch_pdl(kernel, dim3(grid), dim3(threads), (size_t)smem, st, ta, tb, p);
     if (e != cudaSuccess || plan.splits == 1) return e;
-    const long long quads = (long long)M * ((N + 3) / 4);
+    const long long quads = (long long)ncut * plan.part_rows * (BN / 4);
     const int fgrid = (int)std::max<long long>(1, std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8));
     return launch_pdl(splitk_finish_kernel, dim3(fgrid), dim3(256), 0, st, (const int*)part, plan.splits,
-                      plan.part_rows, plan.tiles_m, (const int*)rowsum, gamma, beta, y, M, N, (int)mode);
+                      plan.part_rows, plan.nfull, ncut, plan.tiles_m, plan.mt * BM, (const int*)rowsum, gamma, beta,
+                      y, M, N, (int)mode);
 }
 
 }  // namespace bl

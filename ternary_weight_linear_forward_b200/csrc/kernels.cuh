@@ -32,8 +32,9 @@ cudaError_t launch_binarize_weights(const float* W, long long n, int8_t* W_b, fl
 cudaError_t launch_pack_bits(const int8_t* W_b, long long nwords, uint32_t* W_p, int num_sms, cudaStream_t st);
 
 // k_act.cu
+// rowsum (may be null): the sum of every token's codes, int32 [M]
 cudaError_t launch_quant_act(const void* x, bool bf16, long long M, long long K, int8_t* x_q, float* gamma,
-                             cudaStream_t st);
+                             cudaStream_t st, int* rowsum = nullptr);
 cudaError_t launch_quant_act_grouped(const void* x, bool bf16, long long M, long long K, int G, int8_t* x_q,
                                      float* gamma, cudaStream_t st);
 cudaError_t launch_quant_act_rms(const float* a, const float* b, int combine, long long M, long long K, float* h,
@@ -94,9 +95,11 @@ cudaError_t launch_decode_cuda(const GemvProblem* probs, int count, int M, int x
 // (allow_split), the per-tile counters and partial tiles; gemm_ws_bytes
 // sizes it for allow_split, and M int32 suffice without.
 size_t gemm_ws_bytes(long long M, long long N, long long K);
+// rowsum_ready: the row sums of x_q are already at the start of ws (written
+// by the quantiser), so no row-sum kernel runs.
 cudaError_t launch_gemm(const int8_t* x_q, const float* gamma, int M, int K, const uint32_t* W_p, const float* beta,
                         int N, void* y, YMode mode, void* ws, const DevInfo& dev, cudaStream_t st, int wbits = 2,
-                        bool allow_split = true);
+                        bool allow_split = true, bool rowsum_ready = false);
 
 // k_group.cu  (group quantisation along K)
 size_t regroup_ws_bytes(long long N, long long K);

@@ -26,19 +26,29 @@ import oracle
 BM, BN, BK = 128, 256, 128
 SPLIT_UNITS_TARGET = 148
 MT2_MIN_M = 256
+TAIL_SPLIT_MAX = 4
 
 
 def plan(M, N, K, allow_split=True):
     tiles_m, tiles_n, num_kb = (M + BM - 1) // BM, (N + BN - 1) // BN, (K + BK - 1) // BK
     tiles = tiles_m * tiles_n
     splits = max(1, min(SPLIT_UNITS_TARGET // tiles, num_kb)) if allow_split else 1
-    mt = 1
-    if splits == 1 and M >= MT2_MIN_M:
-        mt, tiles_m = 2, (M + 2 * BM - 1) // (2 * BM)
-    part_rows = min(M, BM)
+    mt, nfull = 1, 0
+    if splits == 1:
+        if M >= MT2_MIN_M:
+            mt, tiles_m = 2, (M + 2 * BM - 1) // (2 * BM)
+        nfull = tiles_m * tiles_n
+        tail = nfull % SPLIT_UNITS_TARGET       # a short last round is cut along K
+        if allow_split and nfull > SPLIT_UNITS_TARGET and 0 < tail <= SPLIT_UNITS_TARGET // 2:
+            s = min(SPLIT_UNITS_TARGET // tail, num_kb, TAIL_SPLIT_MAX)
+            if s > 1:
+                nfull, splits = nfull - tail, s
+    cut = tiles_m * tiles_n - nfull
+    part_rows = min(M, mt * BM)
     rowsum_bytes = (M * 4 + 255) // 256 * 256
-    part_bytes = tiles * splits * part_rows * BN * 4 if splits > 1 else 0
-    return dict(mt=mt, tiles_m=tiles_m, tiles_n=tiles_n, num_kb=num_kb, splits=splits, part_rows=part_rows,
+    part_bytes = cut * splits * part_rows * BN * 4 if splits > 1 else 0
+    return dict(mt=mt, nfull=nfull, tiles_m=tiles_m, tiles_n=tiles_n, num_kb=num_kb, splits=splits,
+                part_rows=part_rows,
                 ws_bytes=rowsum_bytes + part_bytes, part_off=rowsum_bytes)
 
 
@@ -65,15 +75,18 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
     xq_u8 = x_q.view(np.uint8)
     rowsum = x_q.astype(np.int64).sum(1)
     y = np.full((M, N), -(2 ** 40), np.int64)
-    units = tiles_m * tiles_n * splits
+    nfull = pl["nfull"]
+    units = nfull + (tiles_m * tiles_n - nfull) * splits
     part_ints = (pl["ws_bytes"] - pl["part_off"]) // 4
     part = rng.integers(-2 ** 31, 2 ** 31, max(part_ints, 1), dtype=np.int64)   # garbage on entry
     kb_seen = np.zeros((tiles_m * tiles_n, num_kb), np.int64)
     for cta in range(grid):
         for u in range(cta, units, grid):
-            t = u // splits
-            sp = u % splits
-            kb0, kb1 = num_kb * sp // splits, num_kb * (sp + 1) // splits
+            if u < nfull:                             # a whole tile
+                t, sp, kb0, kb1, cut = u, 0, 0, num_kb, False
+            else:                                     # a K range of a cut tile
+                t, sp = nfull + (u - nfull) // splits, (u - nfull) % splits
+                kb0, kb1, cut = num_kb * sp // splits, num_kb * (sp + 1) // splits, splits > 1
             mb, nb = t % tiles_m, t // tiles_m
             D = np.zeros((TBM, BN), np.int64)             # MT accumulators of 128 rows
             for kb in range(kb0, kb1):
@@ -110,27 +123,30 @@ def emulate(x_q, W_p, K, N, wbits, grid, rng, allow_split=False):
                                   for r in range(BM)]).view(np.int8).astype(np.int64)
                     for k in range(BK // 32):
                         D[a * BM:(a + 1) * BM] += A[:, 32 * k:32 * k + 32] @ B[:, 32 * k:32 * k + 32].T
-            if splits == 1:
+            if not cut:
                 for r in range(TBM):                  # epilogue warp (sub-tile r // 128, lanes of r % 128)
                     m = mb * TBM + r
                     if m < M:
                         n0, n1 = nb * BN, min(N, nb * BN + BN)
                         y[m, n0:n1] = D[r, :n1 - n0] - rowsum[m]
                 continue
-            for r in range(BM):                       # this unit's partial tile
-                if r < part_rows and mb * BM + r < M:
-                    o = (u * part_rows + r) * BN
+            for r in range(TBM):                      # this unit's partial tile
+                if r < part_rows and mb * TBM + r < M:
+                    o = ((u - nfull) * part_rows + r) * BN
                     assert o + BN <= part_ints
                     part[o:o + BN] = D[r]
     assert np.all(kb_seen == 1)                       # every (tile, K-block) exactly once
-    if splits > 1:                                    # the finishing kernel: four columns per thread
-        for m in range(M):
-            for n in range(0, N, 4):
-                mb, r, nb, c = m // BM, m % BM, n // BN, n % BN
-                t = mb + nb * tiles_m
+    if splits > 1:                                    # the finishing kernel over the cut tiles' outputs
+        ncut = tiles_m * tiles_n - nfull
+        for e in range(ncut * part_rows * (BN // 4)):
+            tt, rem = divmod(e, part_rows * (BN // 4))
+            r, c = rem // (BN // 4), rem % (BN // 4) * 4
+            t = nfull + tt
+            m, n = (t % tiles_m) * TBM + r, (t // tiles_m) * BN + c
+            if m < M and n < N:
                 tot = np.zeros(4, np.int64)
                 for s2 in range(splits):
-                    o = ((t * splits + s2) * part_rows + r) * BN + c
+                    o = ((tt * splits + s2) * part_rows + r) * BN + c
                     assert o + 4 <= part_ints
                     tot += part[o:o + 4]
                 for j in range(4):
@@ -168,8 +184,8 @@ def test_split_k_plan_of_the_small_batch_shapes():
     for M in (16, 64):
         assert plan(M, 4096, 4096)["splits"] == 9
         assert plan(M, 11008, 4096)["splits"] == 3
-    # prefill: enough tiles, no split
-    assert plan(2048, 4096, 4096)["splits"] == 1 and plan(2048, 11008, 4096)["splits"] == 1
+    # prefill: enough tiles, no split but that of a short last round
+    assert plan(2048, 4096, 4096)["splits"] == 1 and plan(2048, 11008, 4096)["nfull"] == 296
 
 
 @pytest.mark.parametrize("M,K,N,grid", [(130, 384, 300, 2), (5, 128, 260, 1)])
@@ -203,5 +219,26 @@ def test_two_sub_tile_gemm_emulation_matches_the_oracle(M, K, N, grid, wbits, sp
 def test_sub_tiles_of_the_prefill_shapes():
     for N in (4096, 11008):
         pl = plan(2048, N, 4096)
-        assert pl["mt"] == 2 and pl["tiles_m"] == 8 and pl["splits"] == 1
+        assert pl["mt"] == 2 and pl["tiles_m"] == 8
     assert plan(64, 4096, 4096)["mt"] == 1 and plan(200, 4096, 4096)["mt"] == 1
+
+
+def test_cut_last_round_gemm_emulation_matches_the_oracle():
+    # 160 two-sub-tile tiles: a last round of 12 tiles on 148 SMs is cut into
+    # K ranges, summed by the finishing pass; the other 148 are stored whole
+    M, K, N = 256, 256, 256 * 160
+    pl = plan(M, N, K)
+    assert pl["mt"] == 2 and pl["nfull"] == 148 and pl["splits"] == 2
+    rng = np.random.default_rng(11)
+    W = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    np.testing.assert_array_equal(emulate(x_q, oracle.pack(W), K, N, 2, 148, rng, allow_split=True),
+                                  oracle.ternary_acc(x_q, W))
+
+
+def test_cut_last_round_plan_of_the_prefill_shapes():
+    pb = plan(2048, 11008, 4096)          # 344 tiles: 296 whole, the last 48 cut in 3
+    assert (pb["nfull"], pb["splits"]) == (296, 3)
+    assert pb["ws_bytes"] - pb["part_off"] == 48 * 3 * 256 * 256 * 4
+    pa = plan(2048, 4096, 4096)           # 128 tiles: one round, nothing cut
+    assert (pa["nfull"], pa["splits"], pa["ws_bytes"] - pa["part_off"]) == (128, 1, 0)
