@@ -57,19 +57,20 @@ MIXED_LANES_PER_CLK = 85
 NOMINAL_SM_HZ = 1.965e9
 
 
-def small_batch_bound(M, K, N, nbytes, hbm_gbs, sms):
-    """Lower bounds (us) of one small-batch call on the path it takes: HBM
-    time of its algorithmic bytes, and the compute time of the path's own
+def small_batch_bound(M, K, N, nbytes, hbm_gbs, sms, path):
+    """Lower bounds (us) of one small-batch call on the path it takes
+    ("cuda_cores", "swap_ab" or "gemm", as the library reports it): HBM time
+    of its algorithmic bytes, and the compute time of the path's own
     instruction stream spread evenly over the SMs -- dp4a + mask per 4 trits
-    on CUDA cores (M <= 4), 128 weight rows x 32 k per MMA for the swap-AB
-    kernel (M <= 16), 128 tokens x 256 weight rows x 32 k per MMA for the
-    GEMM.  The bound is the larger."""
+    on CUDA cores, 128 weight rows x 32 k per MMA for the swap-AB kernel,
+    128 tokens x 256 weight rows x 32 k per MMA for the GEMM.  The bound is
+    the larger."""
     hbm_us = nbytes / (hbm_gbs * 1e3)
-    if M <= 4:
+    if path == "cuda_cores":
         dp4a, lop3 = N * K / 16 * 4 * M, N * K / 16 * 4
         clk = max(dp4a / DP4A_LANES_PER_CLK, (dp4a + lop3) / MIXED_LANES_PER_CLK) / sms
         comp_us, kind = clk / NOMINAL_SM_HZ * 1e6, "alu (dp4a + mask)"
-    elif M <= 16:
+    elif path == "swap_ab":
         mmas = N * K / (128 * 32)
         comp_us, kind = mmas / sms * MMA_CYCLES / NOMINAL_SM_HZ * 1e6, "tensor (swap-AB, 128 rows x 32 k per MMA)"
     else:
@@ -718,12 +719,15 @@ def main():
             t = timed_run([g])
             gbs = s.algorithmic_bytes * reps / t / 1e9
             us = t / reps * 1e6
-            rl = small_batch_bound(s.M, s.K, s.N, s.algorithmic_bytes, peaks["hbm_gbs"], props.multi_processor_count)
+            path = bl.forward_path(s.M, s.N, s.K)
+            rl = small_batch_bound(s.M, s.K, s.N, s.algorithmic_bytes, peaks["hbm_gbs"], props.multi_processor_count,
+                                   path)
             rl["frac_of_bound"] = rl["bound_us"] / us
             small[s.name] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                              "roofline": rl,
-                             "path": "CUDA-core GEMV" if s.M <= 4 else
-                                     ("tcgen05 swap-AB decode" if s.M <= 16 else "tcgen05 GEMM")}
+                             "path": {"cuda_cores": "CUDA-core GEMV, quantiser fused",
+                                      "swap_ab": "quantiser + tcgen05 swap-AB decode",
+                                      "gemm": "quantiser writing the row sums + tcgen05 GEMM, K split + finishing pass"}[path]}
             del g, W_ps, W_p0, x, y, ws
 
     part("block")

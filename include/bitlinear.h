@@ -481,7 +481,9 @@ bl_status bitlinear_glu_forward(const float* x, int64_t M, int64_t D, int64_t F,
 enum {
     BL_ENGINE_AUTO = 0,          /* the library picks per shape (default): the CUDA-core GEMV
                                     for M <= 4, the swap-AB decode kernel for 5 <= M <= 16
-                                    where it fits, the tcgen05 GEMM otherwise */
+                                    where it fits (for one problem of more than 8 tokens only
+                                    while each CTA's rows fit one 128-lane tile), the tcgen05
+                                    GEMM otherwise */
     BL_ENGINE_CUDA_CORES = 1,    /* M <= 64 on CUDA cores (masked byte dot products) */
     BL_ENGINE_TENSOR_CORES = 2,  /* M <= 16 on the swap-AB tcgen05 decode kernel where it
                                     fits (weight rows on the MMA's 128 lanes), else as AUTO */
@@ -503,6 +505,23 @@ bl_status bitlinear_set_decode_engine(int engine);
 
 /* The engine last set (BL_ENGINE_AUTO initially). */
 int bitlinear_get_decode_engine(void);
+
+/* Kernel families of the forward. */
+enum {
+    BL_PATH_CUDA_CORES = 0,  /* CUDA-core GEMV (masked byte dot products) */
+    BL_PATH_SWAP_AB = 1,     /* tcgen05 swap-AB decode kernel (weight rows on the MMA lanes) */
+    BL_PATH_GEMM = 2         /* tcgen05 int8 GEMM (x_q rows on the MMA lanes) */
+};
+
+/*
+ * Which kernel family bitlinear_forward / _fp / _acc would run for one
+ * problem of M tokens, K input channels and N outputs on the current device
+ * under the current engine, written to *path (a BL_PATH_* value).  An
+ * implementation query, not a feature of the pages.  Errors: BL_ERR_NULL
+ * (path null), BL_ERR_SHAPE (M < 1, N < 1, K < 64 or K % 64 != 0),
+ * BL_ERR_DEVICE (no usable device).
+ */
+bl_status bitlinear_forward_path(int64_t M, int64_t N, int64_t K, int* path);
 
 /* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */

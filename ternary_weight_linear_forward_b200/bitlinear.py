@@ -61,6 +61,7 @@ SIGNATURES = {
     "bitlinear_forward_binary_fp": (_I, [_P, _I, _I64, _I64, _P, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_set_decode_engine": (_I, [_I]),
     "bitlinear_get_decode_engine": (_I, []),
+    "bitlinear_forward_path": (_I, [_I64, _I64, _I64, _P]),
     "bitlinear_device_status": (_I, [_P]),
     "bitlinear_num_sms": (_I, []),
     "bitlinear_test_expire_next_wait": (_I, [_I]),
@@ -544,6 +545,17 @@ def set_decode_engine(name: str):
     if name not in ENGINES:
         raise ValueError(f"unknown decode engine {name!r}")
     _check("bitlinear_set_decode_engine", lib().bitlinear_set_decode_engine(ENGINES[name]))
+
+
+PATHS = {0: "cuda_cores", 1: "swap_ab", 2: "gemm"}
+
+
+def forward_path(M: int, N: int, K: int) -> str:
+    """The kernel family the forward runs for one [M, K] x [N, K] problem on the
+    current device under the current engine: "cuda_cores", "swap_ab" or "gemm"."""
+    v = ctypes.c_int(-1)
+    _check("bitlinear_forward_path", lib().bitlinear_forward_path(M, N, K, ctypes.byref(v)))
+    return PATHS[v.value]
 
 
 def get_decode_engine() -> str:

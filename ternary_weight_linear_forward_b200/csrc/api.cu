@@ -95,6 +95,12 @@ std::atomic<int> g_expire_next_wait{0};
 // and the CUDA cores (17-105 us); beyond that the GEMM wins (M = 64: 23-26 us
 // against 193-482 us on CUDA cores).
 constexpr int AUTO_CUDA_MAX_M = 4;
+// Above this many tokens, one problem whose CTAs hold more rows than one
+// 128-lane tile goes to the split-K GEMM: the swap-AB kernel then issues its
+// MMAs tile after tile at 16 x S columns each, and measured slower (K = 4096,
+// N = 11008: 18.8-19.1 us at M = 16 against 16.9 us for the GEMM; at
+// M = 6-8, 16.2 us for both; at N = 4096, one tile, 11.1 us against 12.3).
+constexpr int AUTO_TC_ONE_TILE_ABOVE_M = 8;
 
 DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
     if (M > GEMV_MAX_M) return PATH_GEMM;
@@ -104,6 +110,9 @@ DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& 
     if (tc_first && M <= decode_tc_max_m()) {
         bool ok = true;
         for (int i = 0; i < count; ++i) ok = ok && decode_tc_supported(M, probs[i].K, probs[i].N, count, dev);
+        if (ok && engine == BL_ENGINE_AUTO && count == 1 && M > AUTO_TC_ONE_TILE_ABOVE_M &&
+            decode_tc_row_tiles(M, probs[0].K, probs[0].N, dev) > 1)
+            return PATH_GEMM;
         if (ok) return PATH_TC;
     }
     return M <= AUTO_CUDA_MAX_M ? PATH_CUDA : PATH_GEMM;
@@ -825,6 +834,20 @@ bl_status bitlinear_set_decode_engine(int engine) {
 }
 
 int bitlinear_get_decode_engine(void) { return g_engine.load(std::memory_order_relaxed); }
+
+bl_status bitlinear_forward_path(int64_t M, int64_t N, int64_t K, int* path) {
+    if (!path) return BL_ERR_NULL;
+    if (M < 1 || M > (int64_t)INT32_MAX) return BL_ERR_SHAPE;
+    bl_status s = check_nk(N, K, 64);
+    if (s) return s;
+    DevInfo dev;
+    s = current_device(dev);
+    if (s) return s;
+    const GemvProblem prob = {nullptr, nullptr, nullptr, nullptr, nullptr, (int)K, (int)N};
+    const DecodePath p = pick_path((int)M, &prob, 1, dev);
+    *path = p == PATH_CUDA ? BL_PATH_CUDA_CORES : p == PATH_TC ? BL_PATH_SWAP_AB : BL_PATH_GEMM;
+    return BL_OK;
+}
 
 bl_status bitlinear_test_expire_next_wait(int enable) {
     g_expire_next_wait.store(enable ? 1 : 0, std::memory_order_relaxed);

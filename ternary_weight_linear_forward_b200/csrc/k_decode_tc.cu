@@ -662,6 +662,13 @@ bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev) {
            dtc_configure(p, G, M, K, N, dev, group_budget(dev, count), grid, smem);
 }
 
+int decode_tc_row_tiles(int M, int K, int N, const DevInfo& dev) {
+    DtcParams p = {};
+    int G = 0, grid;
+    size_t smem;
+    return dtc_configure(p, G, M, K, N, dev, group_budget(dev, 1), grid, smem) ? p.ntiles : 0;
+}
+
 cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode, const DevInfo& dev,
                              cudaStream_t st) {
     // x_dtype: 0 fp32, 1 bf16 (quantiser fused), 2 int8 x_q with gamma

@@ -481,10 +481,6 @@ constexpr int SPLIT_UNITS_TARGET = 148;
 // Two sub-tiles per tile from this many tokens on (when K is not cut).
 constexpr long long MT2_MIN_M = 256;
 
-// A last round of at most half the SMs is cut along K into at most this
-// many ranges, so that it fills the SMs.
-constexpr int TAIL_SPLIT_MAX = 4;
-
 struct GemmPlan {
     int mt, tiles_m, tiles_n, num_kb, splits, nfull, part_rows;
     size_t rowsum_bytes, part_bytes;
@@ -504,17 +500,7 @@ GemmPlan gemm_plan(long long M, long long N, long long K, bool allow_split) {
             g.mt = 2;
             g.tiles_m = (int)((M + 2 * BM - 1) / (2 * BM));
         }
-        const long long all = (long long)g.tiles_m * g.tiles_n;
-        g.nfull = (int)all;
-        const long long tail = all % SPLIT_UNITS_TARGET;
-        if (allow_split && all > SPLIT_UNITS_TARGET && tail > 0 && tail <= SPLIT_UNITS_TARGET / 2) {
-            const int s = (int)std::min<long long>(std::min<long long>(SPLIT_UNITS_TARGET / tail, g.num_kb),
-                                                   TAIL_SPLIT_MAX);
-            if (s > 1) {
-                g.nfull = (int)(all - tail);
-                g.splits = s;
-            }
-        }
+        g.nfull = g.tiles_m * g.tiles_n;  // every tile whole
     }
     const long long cut = (long long)g.tiles_m * g.tiles_n - g.nfull;
     g.part_rows = (int)std::min<long long>(M, (long long)g.mt * BM);

@@ -79,6 +79,8 @@ bool take_wait_expiry_request();
 // k_decode_tc.cu  (M <= 16, tcgen05 int8 tensor cores)
 int decode_tc_max_m();
 bool decode_tc_supported(int M, int K, int N, int count, const DevInfo& dev);
+// row tiles per CTA of one swap-AB problem (0 if it does not fit)
+int decode_tc_row_tiles(int M, int K, int N, const DevInfo& dev);
 cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode, const DevInfo& dev,
                              cudaStream_t st);
 // api.cu: the kernel that runs a problem set with M tokens under the

@@ -247,3 +247,12 @@ def test_grouped_validation():
     assert h(P(A1), 0, 3, 512, 4, P(A3), P(A4), 100, P(A5), 0, P(A6), wsf - 1, None) == WS
 
 
+
+
+def test_forward_path_validation():
+    f = _L().bitlinear_forward_path
+    p = ctypes.c_int(-1)
+    assert f(4, 4096, 4096, None) == NULL
+    assert f(0, 4096, 4096, ctypes.byref(p)) == SHAPE
+    assert f(4, 4096, 100, ctypes.byref(p)) == SHAPE
+    assert f(4, 4096, 4096, ctypes.byref(p)) == DEVICE

@@ -26,7 +26,6 @@ import oracle
 BM, BN, BK = 128, 256, 128
 SPLIT_UNITS_TARGET = 148
 MT2_MIN_M = 256
-TAIL_SPLIT_MAX = 4
 
 
 def plan(M, N, K, allow_split=True):
@@ -37,12 +36,7 @@ def plan(M, N, K, allow_split=True):
     if splits == 1:
         if M >= MT2_MIN_M:
             mt, tiles_m = 2, (M + 2 * BM - 1) // (2 * BM)
-        nfull = tiles_m * tiles_n
-        tail = nfull % SPLIT_UNITS_TARGET       # a short last round is cut along K
-        if allow_split and nfull > SPLIT_UNITS_TARGET and 0 < tail <= SPLIT_UNITS_TARGET // 2:
-            s = min(SPLIT_UNITS_TARGET // tail, num_kb, TAIL_SPLIT_MAX)
-            if s > 1:
-                nfull, splits = nfull - tail, s
+        nfull = tiles_m * tiles_n               # every tile whole
     cut = tiles_m * tiles_n - nfull
     part_rows = min(M, mt * BM)
     rowsum_bytes = (M * 4 + 255) // 256 * 256
@@ -184,8 +178,8 @@ def test_split_k_plan_of_the_small_batch_shapes():
     for M in (16, 64):
         assert plan(M, 4096, 4096)["splits"] == 9
         assert plan(M, 11008, 4096)["splits"] == 3
-    # prefill: enough tiles, no split but that of a short last round
-    assert plan(2048, 4096, 4096)["splits"] == 1 and plan(2048, 11008, 4096)["nfull"] == 296
+    # prefill: enough tiles, no split
+    assert plan(2048, 4096, 4096)["splits"] == 1 and plan(2048, 11008, 4096)["splits"] == 1
 
 
 @pytest.mark.parametrize("M,K,N,grid", [(130, 384, 300, 2), (5, 128, 260, 1)])
@@ -221,24 +215,3 @@ def test_sub_tiles_of_the_prefill_shapes():
         pl = plan(2048, N, 4096)
         assert pl["mt"] == 2 and pl["tiles_m"] == 8
     assert plan(64, 4096, 4096)["mt"] == 1 and plan(200, 4096, 4096)["mt"] == 1
-
-
-def test_cut_last_round_gemm_emulation_matches_the_oracle():
-    # 160 two-sub-tile tiles: a last round of 12 tiles on 148 SMs is cut into
-    # K ranges, summed by the finishing pass; the other 148 are stored whole
-    M, K, N = 256, 256, 256 * 160
-    pl = plan(M, N, K)
-    assert pl["mt"] == 2 and pl["nfull"] == 148 and pl["splits"] == 2
-    rng = np.random.default_rng(11)
-    W = rng.integers(-1, 2, (N, K)).astype(np.int8)
-    x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
-    np.testing.assert_array_equal(emulate(x_q, oracle.pack(W), K, N, 2, 148, rng, allow_split=True),
-                                  oracle.ternary_acc(x_q, W))
-
-
-def test_cut_last_round_plan_of_the_prefill_shapes():
-    pb = plan(2048, 11008, 4096)          # 344 tiles: 296 whole, the last 48 cut in 3
-    assert (pb["nfull"], pb["splits"]) == (296, 3)
-    assert pb["ws_bytes"] - pb["part_off"] == 48 * 3 * 256 * 256 * 4
-    pa = plan(2048, 4096, 4096)           # 128 tiles: one round, nothing cut
-    assert (pa["nfull"], pa["splits"], pa["ws_bytes"] - pa["part_off"]) == (128, 1, 0)

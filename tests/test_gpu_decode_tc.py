@@ -212,3 +212,25 @@ def test_tc_engine_is_the_one_that_runs(dev):
         if not names:
             pytest.skip("profiler reported no kernel records")
         assert any(name in n for n in names), (engine, names)
+
+
+@pytest.mark.parametrize("M,N", [(1, 4096), (4, 11008), (8, 11008), (16, 4096), (16, 11008), (64, 4096)])
+def test_forward_path_names_the_kernel_that_runs(dev, M, N):
+    # the library's path query (used by the bench for its labels and bounds)
+    # names the kernel family the forward launches, under the automatic engine
+    from kernel_trace import kernel_names
+    K = 4096
+    with bl.decode_engine("auto"):
+        path = bl.forward_path(M, N, K)
+        W_p = torch.randint(-2**31, 2**31 - 1, (N, K // 16), dtype=torch.int32, device=dev)
+        beta = torch.tensor([0.02], device=dev)
+        x = torch.randn((M, K), device=dev)
+        names = kernel_names(lambda: bl.forward_fp(x, W_p, beta))
+    if not names:
+        pytest.skip("profiler reported no kernel records")
+    want = {"cuda_cores": "gemv_small_kernel", "swap_ab": "decode_tc_kernel", "gemm": "gemm_kernel"}[path]
+    assert any(want in n for n in names), (M, N, path, names)
+    if M == 16 and N == 11008:
+        assert path == "gemm"
+    if M == 16 and N == 4096:
+        assert path == "swap_ab"
