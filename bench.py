@@ -149,9 +149,11 @@ def upload_graphs(gs, stream) -> bool:
 
 def lead_cycles(n_graphs: int) -> int:
     """Device-side spin queued ahead of a timed region: long enough (about
-    50 us plus 25 us per graph at ~2 GHz) for the host to submit the graphs
-    before the start event is reached."""
-    return int((50 + 25 * n_graphs) * 2000)
+    1 ms plus 100 us per graph at ~2 GHz) for the host to submit the graphs
+    before the start event is reached, even on a busy host.  (A 75 us spin
+    was once outrun by the host's submission of a single graph: the 20
+    timed steps then read 13.6 instead of 9.0 us each.)"""
+    return int((1000 + 100 * n_graphs) * 2000)
 
 
 class ClockSampler:
