@@ -13,20 +13,27 @@
 // the unpack differs.
 //   y       = (float)acc * ((beta * gamma_m) / 127)
 //
-// Persistent kernel, one CTA per SM, 128 x 256 output tiles, K in blocks of
-// 128 bytes.  Warp roles:
-//   warp 0      TMA producer: x_q tile (128 x 128 B, 128-byte swizzle) and the
-//               packed weight tile (256 rows x 8 words) per K-block, no multicast;
+// Persistent kernel, one CTA per SM, output tiles of MT sub-tiles of 128 rows
+// x 256 weight rows (MT = 2 from 256 tokens on, else 1), K in blocks of 128
+// bytes.  Warp roles:
+//   warp 0      TMA producer: x_q tile (128 MT x 128 B, 128-byte swizzle) and
+//               the packed weight tile (256 rows x 8 words) per K-block, no
+//               multicast;
 //   warp 1      TMEM allocation and the single-thread tcgen05.mma issuer
-//               (4 MMAs of K = 32 per K-block), tcgen05.commit to free stages;
+//               (4 MMAs of K = 32 per K-block and sub-tile), tcgen05.commit to
+//               free stages;
 //   warps 2-9   unpack (UNPACK_WARPS = 8): packed word -> four registers of
 //               codes (w >> 2s) & 0x03030303, i.e. 16 consecutive-k bytes,
 //               stored as one 16-byte chunk into the 128-byte-swizzled
 //               K-major operand layout;
-//   warps 10-13 epilogue: tcgen05.ld of the int32 accumulators (32 TMEM lanes
-//               per warp), rowsum correction, rescale, bf16/fp32 store.
-// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap
-// the main loop of tile t + 1.  Every mbarrier wait is bounded.
+//   warps 10..  epilogue, 4 MT warps: tcgen05.ld of the int32 accumulators (32
+//               TMEM lanes per warp), rowsum correction, rescale, bf16/fp32
+//               store.
+// With MT = 1 two TMEM accumulators (2 x 256 columns) let the epilogue of
+// tile t overlap the main loop of tile t + 1; with MT = 2 they are the two
+// sub-tiles' accumulators, which share every unpacked B block (half the
+// unpack and packed-weight traffic per output).  Every mbarrier wait is
+// bounded.
 //
 // Few tiles (a few tokens: M <= 128 gives N / 256 tiles for 148 SMs) are cut
 // along K: a work unit is (tile, K range) and writes its int32 tile to a
