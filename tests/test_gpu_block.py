@@ -37,7 +37,11 @@ def close(got, ref):
         assert rel.max() <= REL_TOL, rel.max()
 
 
-@pytest.mark.parametrize("M,K", [(1, 2560), (1, 6912), (3, 1024), (1, 16)])
+# up to 64 rows a row is shared by a cluster of 8 CTAs (K = 64: most CTAs have
+# an empty slice; K = 98304: 48 KiB slices); from 65 rows, or beyond 98304
+# channels, one CTA per row
+@pytest.mark.parametrize("M,K", [(1, 2560), (1, 6912), (3, 1024), (1, 16), (2, 64), (64, 2560), (65, 1024),
+                                 (1, 98304), (1, 100000)])
 def test_quant_act_rms_none(dev, M, K):
     x = workloads.activations(M + K, M, K, outliers=True)
     h, x_q, g = bl.quant_act_rms(T(x, dev), want_h=True)
