@@ -146,9 +146,10 @@ size_t bitlinear_forward_workspace(int64_t M, int64_t N, int64_t K);
  *   ws    >= bitlinear_forward_workspace(M, N, K) bytes (may be NULL when that is 0)
  * K % 64 == 0, K <= BL_MAX_K.  By default M <= 4 runs the decode GEMV on
  * CUDA cores, 5 <= M <= 16 a decode kernel on the tcgen05 int8 tensor cores
- * (where x_hat fits its shared memory) and larger M the GEMM on the tensor
- * cores (bitlinear_set_decode_engine selects other kernels for M <= 64).  All
- * give identical results.
+ * (where x_hat fits its shared memory; above 8 tokens only while each CTA's
+ * rows fit one 128-lane tile) and larger M the GEMM on the tensor cores
+ * (bitlinear_set_decode_engine selects other kernels for M <= 64;
+ * bitlinear_forward_path reports the choice).  All give identical results.
  *
  * The forward kernels begin streaming W_p and read beta before the kernel
  * queued ahead of them on the stream has finished (programmatic dependent

@@ -118,8 +118,8 @@ DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& 
     return M <= AUTO_CUDA_MAX_M ? PATH_CUDA : PATH_GEMM;
 }
 
-// rowsum_ready: on the GEMM path, the quantiser has written the row sums of
-// x_q at the start of ws.
+// rowsum_ready: the quantiser has written the row sums of x_q at the start
+// of ws (read by the tensor-core paths).
 bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t K, const uint32_t* W_p,
                       const float* beta, int64_t N, void* y, YMode mode, void* ws, size_t ws_bytes, void* stream,
                       bool rowsum_ready = false) {
@@ -130,8 +130,9 @@ bl_status run_forward(const int8_t* x_q, const float* gamma, int64_t M, int64_t 
     bl_status s = current_device(dev);
     if (s) return s;
     cudaError_t e;
-    const GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
+    GemvProblem prob = {x_q, gamma, W_p, beta, y, (int)K, (int)N};
     const DecodePath path = pick_path((int)M, &prob, 1, dev);
+    if (rowsum_ready) prob.rowsum = reinterpret_cast<const int*>(ws);
     if (path == PATH_TC)
         e = launch_decode_tc(&prob, 1, (int)M, BL_I8, mode, dev, as_stream(stream));
     else if (path == PATH_CUDA)
@@ -428,14 +429,15 @@ bl_status bitlinear_forward_fp(const void* x, int x_dtype, int64_t M, int64_t K,
     int8_t* x_q = reinterpret_cast<int8_t*>(ws);
     float* gamma = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256((size_t)M * K));
     char* fws = reinterpret_cast<char*>(gamma) + round256((size_t)M * 4);
-    // on the GEMM path the quantiser also writes the row sums the GEMM needs
-    // (at the start of its workspace), which saves the row-sum launch
-    const bool gemm = pick_path((int)M, &prob, 1, dev) == PATH_GEMM;
+    // on the tensor-core paths the quantiser also writes the row sums of x_q
+    // (at the start of the forward's workspace): the GEMM then needs no
+    // row-sum launch and the swap-AB kernel no read-back of x_hat
+    const bool rows = pick_path((int)M, &prob, 1, dev) != PATH_CUDA;
     cudaError_t e = launch_quant_act(x, x_dtype == BL_BF16, M, K, x_q, gamma, as_stream(stream),
-                                     gemm ? reinterpret_cast<int*>(fws) : nullptr);
+                                     rows ? reinterpret_cast<int*>(fws) : nullptr);
     if (e != cudaSuccess) return BL_ERR_CUDA;
     return run_forward(x_q, gamma, M, K, W_p, beta, N, y, mode, fws, ws_bytes - (fws - reinterpret_cast<char*>(ws)),
-                       stream, gemm);
+                       stream, rows);
 }
 
 bl_status bitlinear_forward_fp_batch(const bl_problem* problems, int count, int64_t M, int x_dtype, int y_dtype,

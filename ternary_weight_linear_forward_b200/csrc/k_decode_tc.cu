@@ -90,6 +90,7 @@ struct DtcHdr {
     float gam[DTC_MAX_M];
     float xscale[DTC_MAX_M];         // 127 / gamma
     float fscale[DTC_MAX_M];
+    float beta;                      // read at CTA start (a weight input)
 };
 static_assert(sizeof(DtcHdr) <= DTC_HDR, "decode header too large");
 
@@ -100,6 +101,7 @@ struct alignas(64) DtcParams {
     const void* x;     // fp32 / bf16 activations (quantised in the prologue)
     const int8_t* x_q;
     const float* gamma;
+    const int* rowsum_in;  // row sums of x_q when the quantiser wrote them (else null)
     const float* beta;
     void* y;
     int M, K, N, mode;
@@ -211,6 +213,14 @@ __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part
     const int ctid = threadIdx.x, lane = ctid & 31, warp = ctid >> 5;
     const size_t xrow = (size_t)p.K * (XM == X_BF16 ? 2 : XM == X_F32 ? 4 : 1);
     const char* xbase = XM == X_QUANTISED ? reinterpret_cast<const char*>(p.x_q) : reinterpret_cast<const char*>(p.x);
+    // gamma and the given row sums (written by the preceding quantiser) load
+    // while x_hat is staged
+    float gq = 0.0f;
+    int rsq = 0;
+    if (XM == X_QUANTISED && ctid < MP && ctid < p.M) {
+        if (p.mode != Y_ACC) gq = __ldg(p.gamma + ctid);
+        if (p.rowsum_in) rsq = __ldg(p.rowsum_in + ctid);
+    }
     const int rows = p.S * MP;                // B rows per K-block before the G expansion
     const int KC = p.T * (DTC_STAGE_K / 16);  // chunks per B row
     const uint32_t bs = smem_u32(Bs);
@@ -261,7 +271,7 @@ __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part
             }
         }
         cp_async_wait_all();
-        for (int j = warp; j < rows; j += NW) {
+        for (int j = warp; j < rows && !p.rowsum_in; j += NW) {
             const int m = j % MP;
             int rs = 0;
             for (int kc = lane; kc < KC; kc += 32) {
@@ -308,10 +318,11 @@ __device__ __forceinline__ void stage_b(const DtcParams& p, DtcHdr& h, int* part
         const int m = ctid;
         float f = 0.0f;
         if (p.mode != Y_ACC && m < p.M) {
-            const float g = XM == X_QUANTISED ? __ldg(p.gamma + m) : h.gam[m];
-            f = __fdiv_rn(__fmul_rn(__ldg(p.beta), g), 127.0f);
+            const float g = XM == X_QUANTISED ? gq : h.gam[m];
+            f = __fdiv_rn(__fmul_rn(h.beta, g), 127.0f);
         }
         h.fscale[m] = f;
+        if (XM == X_QUANTISED && p.rowsum_in && m < p.M) h.rowsum[m] = rsq;
     }
     unpack_sync();
     if (ctid == 0) mbar_arrive(&h.b_ready);
@@ -487,6 +498,7 @@ __device__ __forceinline__ void dtc_body(const DtcParams& p, int cta) {
         mbar_init(&h.drain, 1);
         h.abort_flag = 0;
         for (int m = 0; m < DTC_MAX_M; ++m) h.rowsum[m] = h.amax[m] = 0;
+        h.beta = p.mode == Y_ACC ? 0.0f : __ldg(p.beta);
         fence_mbar_init();
         prefetch_tmap(&p.tmap);
         produce(p, h, ring, r0, 0, 1, pol);
@@ -715,6 +727,7 @@ cudaError_t launch_decode_tc(const GemvProblem* probs, int count, int M, int x_d
         if (xm == X_QUANTISED) {
             p.x_q = static_cast<const int8_t*>(q.x);
             p.gamma = q.gamma;
+            p.rowsum_in = q.rowsum;
         } else {
             p.x = q.x;
         }

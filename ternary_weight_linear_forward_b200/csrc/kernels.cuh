@@ -60,6 +60,7 @@ struct GemvProblem {
     const float* beta;
     void* y;
     int K, N;
+    const int* rowsum;   // with x_q: the row sums of x_q when already known, else null
 };
 int gemv_group_max();
 cudaError_t launch_gemv_fused_group(const GemvProblem* probs, int count, int M, int x_dtype, YMode mode,
