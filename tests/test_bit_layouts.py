@@ -132,3 +132,20 @@ def test_gemm_unpack_codes_and_swizzled_placement():
         np.testing.assert_array_equal(un2, W_t[n].astype(np.int64) + 1)
         un1 = np.concatenate([row1[((c ^ (n & 7)) * 16):((c ^ (n & 7)) * 16) + 16] for c in range(8)])
         np.testing.assert_array_equal(un1, W_b[n].astype(np.int64) + 1)
+
+
+def test_rms_cluster_slices_cover_every_chunk_once():
+    # The RMS-folded quantiser shares a row among a cluster of 8 CTAs: CTA r
+    # takes 16-element chunks [G r / 8, G (r + 1) / 8) and keeps them in a
+    # shared-memory slice sized for ceil(G / 8) chunks (at most 40 KiB).
+    C = 8
+    for K in list(range(16, 4096, 16)) + [6912, 11008, 65536, 81920]:
+        G = K // 16
+        cap = (G + C - 1) // C
+        assert cap * 16 * 4 <= 40 * 1024
+        seen = []
+        for r in range(C):
+            g0, g1 = G * r // C, G * (r + 1) // C
+            assert 0 <= g1 - g0 <= cap
+            seen += range(g0, g1)
+        assert seen == list(range(G))
