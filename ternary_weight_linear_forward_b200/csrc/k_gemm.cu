@@ -22,11 +22,11 @@
 //   warp 1      TMEM allocation and the single-thread tcgen05.mma issuer
 //               (4 MMAs of K = 32 per K-block and sub-tile), tcgen05.commit to
 //               free stages;
-//   warps 2-9   unpack (UNPACK_WARPS = 8): packed word -> four registers of
+//   warps 2-5   unpack (UNPACK_WARPS = 4): packed word -> four registers of
 //               codes (w >> 2s) & 0x03030303, i.e. 16 consecutive-k bytes,
 //               stored as one 16-byte chunk into the 128-byte-swizzled
 //               K-major operand layout;
-//   warps 10..  epilogue, 4 MT warps: tcgen05.ld of the int32 accumulators (32
+//   warps 6..   epilogue, 4 MT warps: tcgen05.ld of the int32 accumulators (32
 //               TMEM lanes per warp), rowsum correction, rescale, bf16/fp32
 //               store.
 // With MT = 1 two TMEM accumulators (2 x 256 columns) let the epilogue of
@@ -60,7 +60,7 @@ constexpr int BC_BYTES = BN * BK;             // 32 KiB unpacked codes
 constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words (2-bit; 1-bit uses half)
 constexpr int HDR_BYTES = 1024;
 constexpr int MAX_STAGES = 4;
-constexpr int UNPACK_WARPS = 8;
+constexpr int UNPACK_WARPS = 4;  // measured: 4 beat 8 and 16 (fewer warps contending for shared memory)
 constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;  // epilogue warps EPI_WARP0 .. EPI_WARP0 + 4 MT - 1
 
