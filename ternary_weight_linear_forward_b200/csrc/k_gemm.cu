@@ -60,7 +60,7 @@ constexpr int BC_BYTES = BN * BK;             // 32 KiB unpacked codes
 constexpr int BP_BYTES = BN * (BK / 16) * 4;  // 8 KiB packed words (2-bit; 1-bit uses half)
 constexpr int HDR_BYTES = 1024;
 constexpr int MAX_STAGES = 4;
-constexpr int UNPACK_WARPS = 4;  // measured: 4 beat 8 and 16 (fewer warps contending for shared memory)
+constexpr int UNPACK_WARPS = 4;  // measured: 4 beat 2, 8 and 16
 constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;  // epilogue warps EPI_WARP0 .. EPI_WARP0 + 4 MT - 1
 
