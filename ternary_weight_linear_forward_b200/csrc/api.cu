@@ -98,8 +98,9 @@ constexpr int AUTO_CUDA_MAX_M = 4;
 // Above this many tokens, one problem whose CTAs hold more rows than one
 // 128-lane tile goes to the split-K GEMM: the swap-AB kernel then issues its
 // MMAs tile after tile at 16 x S columns each, and measured slower (K = 4096,
-// N = 11008: 18.8-19.1 us at M = 16 against 16.9 us for the GEMM; at
-// M = 6-8, 16.2 us for both; at N = 4096, one tile, 11.1 us against 12.3).
+// N = 11008: ~19 us at M = 16 against 16.4 us for the GEMM, while at M = 6-8
+// the swap-AB kernel takes 15.5 us; at N = 4096, one tile, 9.6 us against
+// ~12 us for the GEMM).
 constexpr int AUTO_TC_ONE_TILE_ABOVE_M = 8;
 
 DecodePath pick_path(int M, const GemvProblem* probs, int count, const DevInfo& dev) {
