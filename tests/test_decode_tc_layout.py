@@ -263,3 +263,18 @@ def test_staging_row_sums_match_the_token_sums():
         x_q = rng.integers(-127, 128, (M, K)).astype(np.int8)
         rows = row_rowsum(x_q, M, K, mp, S, T * (STAGE_K // 16), Lfull)
         assert rows == [int(x_q[m].astype(np.int64).sum()) if m < M else 0 for m in range(mp)]
+
+
+def test_lone_problem_takes_the_whole_sm_when_its_ring_is_short():
+    # At two CTAs per SM a problem whose ring cannot hold all of its stages
+    # (M = 16, N = 11008: 6 stages of 16 KiB, 2 slots) is laid out for the
+    # whole SM instead, where every stage is in flight at once.
+    FULL = 232448 - 1024
+    half = configure(16, 4096, 11008, 148, BUDGET)
+    assert half["slots"] < half["ntiles"] * half["T"]
+    full = configure(16, 4096, 11008, 148, FULL)
+    assert full["slots"] == full["ntiles"] * full["T"]
+    assert full["smem"] + 1024 <= 232448
+    # one tile of a 4096-row problem already fits two CTAs per SM
+    p = configure(16, 4096, 4096, 148, BUDGET)
+    assert p["slots"] == p["ntiles"] * p["T"]
