@@ -8,7 +8,9 @@ channels):
 both through one call of the batched C-ABI entry bitlinear_forward_fp_batch
 (one kernel launch per step; the projections are independent).  Weights are prepared once (absmean ternarisation + 2-bit
 packing, outside the timed region) and rotate over enough copies that every
-step reads its weights from HBM (working set > L2).
+step reads its weights from HBM (working set > L2).  The timed steps are CUDA
+graphs uploaded to the device before the start event, behind a ~1 ms
+device-side spin, so the timed region holds exactly the replayed steps.
 
 Printed metric: algorithmic GB/s (packed weights + activations + outputs per
 step / step time), whole job over all ranks, plus the roofline of the GEMV
