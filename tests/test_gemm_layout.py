@@ -215,3 +215,18 @@ def test_sub_tiles_of_the_prefill_shapes():
         pl = plan(2048, N, 4096)
         assert pl["mt"] == 2 and pl["tiles_m"] == 8
     assert plan(64, 4096, 4096)["mt"] == 1 and plan(200, 4096, 4096)["mt"] == 1
+
+
+@pytest.mark.parametrize("unpack_warps", [4, 8])
+@pytest.mark.parametrize("mt", [1, 2])
+def test_epilogue_warps_cover_every_tile_row_once(unpack_warps, mt):
+    # Epilogue warps start after the producer, the MMA issuer and the unpack
+    # warps; warp w may read only TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so
+    # it takes those lanes of sub-tile (w - first) / 4.  Every row of the
+    # 128 MT-row tile must be read by exactly one thread.
+    first = 2 + unpack_warps
+    rows = []
+    for w in range(first, first + 4 * mt):
+        sub, q = (w - first) // 4, w % 4
+        rows += [sub * BM + q * 32 + lane for lane in range(32)]
+    assert sorted(rows) == list(range(BM * mt))
